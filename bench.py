@@ -1,0 +1,405 @@
+"""Throughput of the spatial-spectral coupling (fwd + bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload dense_60k|geo_60k|...] [--need-dv]
+
+One step = the whole hot path over one synthetic shape pair resident in HBM:
+the dense coupling forward (O, lse) and backward (dQ, dK) at n = 60,000,
+d = 128, k = 196 (the headline), followed in the same line by the
+Geo-FlashAttention step at the same size (patch scores + top-R selection,
+forward, backward).  Throughput is effective TFLOP/s counted the
+FlashAttention way (executed flops including the S recompute of the
+backward): per (i, j) pair 2(d + k) forward and 2(2d + k) + 2d backward.
+
+Under torchrun every rank runs its own shape pair (independent problems, weak
+scaling, no collective on the data path); the time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded row sample of the
+same workload and extrapolates to the full size.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "coupling fwd+bwd ms & TFLOP/s at n=60k (dense, geo); % of bf16 tensor peak"
+
+
+def pair_flops(d, k, need_dv):
+    fwd = 2 * (d + k)
+    bwd = 2 * (2 * d + k) + 2 * d + (2 * k if need_dv else 0)
+    return fwd, bwd
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(tflops=j["bf16_tflops"], tflops_sustained=j["bf16_tflops_sustained"],
+                    hbm=j["hbm_gbs"], source="measured")
+    return dict(tflops=1590.0, tflops_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(ngpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, ws, rank, local):
+    import torch
+    from spatial_spectral_attention_b200 import api, synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pair = synth.make_workload(args.workload)
+    gpair = synth.make_workload("geo_60k") if args.with_geo else None
+    bf = lambda a: torch.tensor(a).to(torch.bfloat16)
+    host = dict(Q=bf(pair.F_N).pin_memory(), K=bf(pair.F_M).pin_memory(),
+                V=bf(pair.Phi_M).pin_memory(), dO=torch.tensor(pair.dO).pin_memory())
+    Q, K, V, dO = (host[x].to(dev) for x in ("Q", "K", "V", "dO"))
+    n, d, k = pair.n, pair.d, pair.k
+    scale = pair.scale
+    ws_bytes = api.lib().ssc_dense_coupling_workspace_size(n, n, d, k, 0)
+    wsb = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+    fpp, bpp = pair_flops(d, k, args.need_dv)
+    flops_step = float(n) * n * (fpp + bpp)
+
+    def dense_step(Qd, Kd, Vd, dOd, ev=None):
+        if ev:
+            ev[0].record(stream)
+        O, lse = api.ssc_dense_coupling_fwd(Qd, Kd, Vd, scale, workspace=wsb)
+        if ev:
+            ev[1].record(stream)
+        g = api.ssc_dense_coupling_bwd(Qd, Kd, Vd, O, lse, dOd, scale, need_dV=args.need_dv,
+                                       workspace=wsb)
+        if ev:
+            ev[2].record(stream)
+        return O, lse, g
+
+    # geo inputs and tables (tables per shape, computed once: they depend on geometry only)
+    geo = None
+    if gpair is not None:
+        gQ, gK, gV = bf(gpair.F_N).to(dev), bf(gpair.F_M).to(dev), bf(gpair.Phi_M).to(dev)
+        gdO = torch.tensor(gpair.dO).to(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        _, _, offN, memN = api.ssc_fps_patches(torch.tensor(gpair.pts_N).to(dev), gpair.P)
+        _, _, offM, memM = api.ssc_fps_patches(torch.tensor(gpair.pts_M).to(dev), gpair.P)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        fps_ms = t0.elapsed_time(t1) / 2
+        gws = torch.empty(api.lib().ssc_geo_coupling_workspace_size(
+            gpair.n, gpair.n, gpair.d, gpair.k, gpair.P, gpair.P, gpair.R, 0),
+            dtype=torch.uint8, device=dev)
+        geo = dict(Q=gQ, K=gK, V=gV, dO=gdO, offN=offN, memN=memN, offM=offM, memM=memM,
+                   fps_ms=fps_ms, ws=gws)
+
+    def geo_step():
+        g = geo
+        topk = api.ssc_patch_scores_topk(g["Q"], g["K"], g["offN"], g["memN"], g["offM"],
+                                         g["memM"], gpair.R)
+        O, lse = api.ssc_geo_coupling_fwd(g["Q"], g["K"], g["V"], gpair.scale, g["offN"],
+                                          g["memN"], g["offM"], g["memM"], topk, workspace=g["ws"])
+        api.ssc_geo_coupling_bwd(g["Q"], g["K"], g["V"], O, lse, g["dO"], gpair.scale, g["offN"],
+                                 g["memN"], g["offM"], g["memM"], topk, need_dV=args.need_dv,
+                                 workspace=g["ws"])
+        return topk
+
+    for _ in range(args.warmup):
+        dense_step(Q, K, V, dO)
+        if geo:
+            geo_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+
+    # ---- timed region: device-resident inputs, L2 flushed between steps (untimed)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    launches0 = api.ssc_kernel_launches()
+    torch.cuda.reset_peak_memory_stats(dev)
+    mem0 = torch.cuda.memory_allocated(dev)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        for s in range(args.steps):
+            flush.zero_()
+            dense_step(Q, K, V, dO, evs[s])
+            if geo:
+                flush.zero_()
+                gev[s][0].record(stream)
+                geo_step()
+                gev[s][1].record(stream)
+        torch.cuda.synchronize()
+    launches = api.ssc_kernel_launches() - launches0
+    peak_gib = (torch.cuda.max_memory_allocated(dev) - mem0 + ws_bytes) / 2**30
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
+    dense_ms = max_over_ranks(float(np.mean(step_ms)), ws)
+    geo_ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in gev])), ws) if geo else None
+    barrier(ws)
+
+    # ---- end to end through the public API with host buffers
+    out_host = dict(O=torch.empty((n, k), dtype=torch.float32).pin_memory(),
+                    lse=torch.empty(n, dtype=torch.float32).pin_memory(),
+                    dQ=torch.empty((n, d), dtype=torch.float32).pin_memory(),
+                    dK=torch.empty((n, d), dtype=torch.float32).pin_memory())
+    e2e_steps = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Qd, Kd, Vd, dOd = (host[x].to(dev, non_blocking=True) for x in ("Q", "K", "V", "dO"))
+        O, lse, (dQ, dK, _) = dense_step(Qd, Kd, Vd, dOd)
+        out_host["O"].copy_(O, non_blocking=True)
+        out_host["lse"].copy_(lse, non_blocking=True)
+        out_host["dQ"].copy_(dQ, non_blocking=True)
+        out_host["dK"].copy_(dK, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
+    h2d = sum(host[x].numel() * host[x].element_size() for x in ("Q", "K", "V", "dO"))
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+
+    pk = peaks()
+    tflops = ws * flops_step / (dense_ms * 1e-3) / 1e12
+    # dominant kernel: the backward (2/3 of the flops); its window also holds the
+    # small prep kernels, so the achieved rate is a slight underestimate
+    bwd_flops = float(n) * n * bpp
+    bwd_mean = float(np.mean(bwd_ms))
+    achieved = bwd_flops / (bwd_mean * 1e-3) / 1e12
+    res = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dense_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded sphere workload: random-Fourier-feature descriptors, "
+                "spherical-harmonic eigenbasis)",
+        "config": {"workload": pair.name, "n": n, "d": d, "k": k, "need_dV": args.need_dv,
+                   "flops_per_step": flops_step, "flop_convention":
+                   "executed, fwd 2(d+k) + bwd 2(2d+k)+2d per (i,j) pair",
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{ws} (independent shape pairs)"},
+        "dense": {"fwd_ms": round(float(np.mean(fwd_ms)), 4),
+                  "bwd_ms": round(float(np.mean(bwd_ms)), 4),
+                  "fwd_tflops": round(float(n) * n * fpp / (np.mean(fwd_ms) * 1e-3) / 1e12, 2),
+                  "bwd_tflops": round(achieved, 2),
+                  "frac_of_peak": round(tflops / ws / pk["tflops"], 4),
+                  "peak_gib": round(peak_gib, 3)},
+        "roofline": {"bound": "tensor", "kernel": "tc_bwd_kernel (dense backward)",
+                     "achieved": round(achieved, 2), "peak": pk["tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["tflops"], 4), "peak_source": pk["source"] +
+                     " burst bf16 (MEASURED_PEAKS.json bf16_tflops)", "traffic": None},
+        "e2e": {"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if geo:
+        U = float(np.mean(np.diff(geo["offM"].cpu().numpy()))) * gpair.R
+        gflops = float(gpair.n) * U * (fpp + bpp)
+        res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_ms, 4),
+                      "tflops": round(gflops / (geo_ms * 1e-3) / 1e12, 2),
+                      "support_per_row": round(U, 1), "fps_ms_per_shape": round(geo["fps_ms"], 3),
+                      "note": "step = scores/top-R + fwd + bwd; FPS per shape, outside the step"}
+    return res
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(pair, budget_s, need_dv):
+    """Time the oracle's dense fwd+bwd on a row sample; extrapolate to all rows."""
+    import oracle
+    import torch
+    bf = lambda a: torch.tensor(a).to(torch.bfloat16).double().numpy()
+    Q, K, V = bf(pair.F_N), bf(pair.F_M), bf(pair.Phi_M)
+    dO = bf(pair.dO)
+    rows = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.dense_bwd(Q[:rows], K, V, dO[:rows], pair.scale)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or rows >= pair.n:
+            break
+        rows = min(pair.n, rows * 4)
+    full_s = dt * pair.n / rows
+    fpp, bpp = pair_flops(pair.d, pair.k, need_dv)
+    tflops = float(pair.n) * pair.n * (fpp + bpp) / full_s / 1e12
+    return tflops, full_s * 1e3, rows, dt
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, ws, rank):
+    from spatial_spectral_attention_b200 import synth
+    pair = synth.make_workload(args.workload)
+    vals, times = [], []
+    for s in range(args.warmup + args.steps):
+        tf, ms, rows, dt = oracle_sample(pair, args.ref_budget, args.need_dv)
+        if s >= args.warmup:
+            vals.append(tf)
+            times.append(ms)
+    v = float(np.mean(vals))
+    cores = cpu_cores()
+    sample = f"{rows} of {pair.n} target rows per step (all {pair.n} source rows), extrapolated"
+    return {
+        "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(float(np.mean(times)), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": pair.name, "n": pair.n, "d": pair.d, "k": pair.k,
+                   "need_dV": args.need_dv},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dense_60k")
+    ap.add_argument("--need-dv", action="store_true")
+    ap.add_argument("--no-geo", dest="with_geo", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle time per step")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, ws, rank)), flush=True)
+        return
+    res = run_ours(args, ws, rank, local)
+    if rank == 0:
+        if args.cpu_baseline:
+            from spatial_spectral_attention_b200 import synth
+            tf, ms, rows, dt = oracle_sample(synth.make_workload(args.workload), 12.0, args.need_dv)
+            res["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cpu_cores(),
+                                   "kind": "oracle", "ms_full_step_est": round(ms, 1),
+                                   "sample": f"{rows} of {res['config']['n']} target rows "
+                                             f"({dt:.1f} s), extrapolated to all rows"}
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * ssc.h -- C ABI of the spatial-spectral coupling library (libssc.so), sm_100a.
+ *
+ * The library evaluates the spatial-spectral coupling of deep functional maps,
+ *     O = Pi_NM Phi_M = softmax(s * F_N F_M^T) Phi_M,
+ * as scaled dot-product attention with Q = F_N (target descriptors),
+ * K = F_M (source descriptors) and V = Phi_M (source Laplace-Beltrami
+ * eigenbasis) without ever storing the n_N x n_M map Pi_NM
+ * ("Spatial-Spectral Coupling as Attention", project page, sections "The
+ * bottleneck" and "Spatial-spectral coupling is attention").  It also provides
+ * Geo-FlashAttention (same page, section "Geo-FlashAttention"): both shapes are
+ * partitioned into geodesic patches, patch-mean descriptors are scored, each
+ * target patch keeps its top R source patches, and the exact softmax runs over
+ * the vertices of those patches only.
+ *
+ * Conventions shared by every call
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, unless a
+ *    comment says otherwise.  The library never allocates device memory: each
+ *    call that needs scratch space has a *_workspace_size query, and the caller
+ *    passes a device buffer `ws` of at least that many bytes (256-byte aligned).
+ *  - Work is enqueued on `stream` (a cudaStream_t, passed as void*) and runs
+ *    asynchronously; no call synchronises the host.  Device-side failures
+ *    (a bounded wait that ran out) are recorded in a library status word that
+ *    ssc_device_status() reads back.
+ *  - Matrices are row-major with an explicit leading dimension (`ld*`, in
+ *    elements, >= the row length).  bf16 Q and K need 16-byte aligned base
+ *    pointers and leading dimensions that are multiples of 8 elements (the
+ *    tensor-memory-accelerator reads them in place); bf16 V may have any
+ *    stride (it is re-packed into the workspace when its rows are not 16-byte
+ *    aligned); fp32 inputs need 4-byte alignment; fp32 outputs need 16-byte
+ *    aligned base pointers.
+ *  - Index tables that are inconsistent (an index out of range, offsets that
+ *    decrease or exceed n, repeated top-R entries) never cause an out-of-range
+ *    access: the offending entries are dropped, results are unspecified and
+ *    ssc_device_status() reports SSC_ERR_INVALID_ARG.
+ *  - `dtype` selects the input type of Q, K, V: SSC_BF16 (bf16 inputs, tensor
+ *    cores, fp32 accumulation) or SSC_F32 (fp32 inputs on CUDA cores, a check
+ *    mode held to a 1e-4 tolerance).  Outputs are always fp32.
+ *  - Sizes: n >= 1, d in {64, 128}, 1 <= k <= 256, 1 <= R <= P <= n,
+ *    P <= 65535.  Violations return SSC_ERR_INVALID_ARG or SSC_ERR_UNSUPPORTED
+ *    before any work is enqueued; outputs are then untouched.
+ *  - Vertex indices and patch tables are int32.
+ */
+#ifndef SSC_H_
+#define SSC_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* ssc_stream_t; /* a cudaStream_t; NULL = the legacy default stream */
+
+enum ssc_status_code {
+  SSC_OK = 0,
+  SSC_ERR_INVALID_ARG = 1,  /* bad size, null pointer, bad index table */
+  SSC_ERR_UNSUPPORTED = 2,  /* d or k outside what the kernels implement */
+  SSC_ERR_ALIGNMENT = 3,    /* base pointer or leading dimension misaligned */
+  SSC_ERR_WORKSPACE = 4,    /* workspace missing or smaller than the query */
+  SSC_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed */
+  SSC_ERR_TIMEOUT = 6       /* a device-side wait hit its limit (see ssc_device_status) */
+};
+
+enum ssc_dtype { SSC_BF16 = 0, SSC_F32 = 1 };
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* ssc_status_string(int status);
+
+/* Library version, (major << 16) | minor. */
+int ssc_version(void);
+
+/* Running count of the CUDA kernels this library has enqueued (host-side
+ * counter, all devices and streams); lets a caller attribute launches. */
+unsigned long long ssc_kernel_launches(void);
+
+/* Synchronises `stream`, then stores into *status the device status word that
+ * kernels set when a bounded wait ran out (SSC_OK or SSC_ERR_TIMEOUT) and, if
+ * `clear` is non-zero, resets it.  Returns SSC_ERR_CUDA if the sync failed. */
+int ssc_device_status(ssc_stream_t stream, int clear, int* status);
+
+/* Sets the time limit of every device-side wait, in nanoseconds (default
+ * 2e9).  Intended for tests; 0 restores the default. */
+int ssc_set_wait_limit_ns(unsigned long long ns);
+
+/* Test hook of the bounded-wait machinery: launches one block that waits on a
+ * barrier nothing will ever arrive on.  The wait gives up after `limit_ns`,
+ * records SSC_ERR_TIMEOUT in the device status word and the kernel returns.
+ * No GPU fault, trap or hang is involved. */
+int ssc_debug_wait_timeout(unsigned long long limit_ns, ssc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Geodesic patches.                                                        */
+/* Source: digest "Interpretation" (geodesic farthest-point sampling) and    */
+/* project page "Geo-FlashAttention" (partition each surface into geodesic   */
+/* patches).  On the unit sphere the geodesic distance is the great-circle   */
+/* distance, a decreasing function of the dot product, so every ranking is   */
+/* made on the fp64 dot ((x0*y0 + x1*y1) + x2*y2) of the fp32 coordinates.   */
+/* ------------------------------------------------------------------------ */
+
+/* Scratch bytes ssc_fps_patches needs for n points and P patches. */
+size_t ssc_fps_patches_workspace_size(int n, int P);
+
+/* Farthest-point sampling plus nearest-centre (Voronoi) assignment.
+ *   pts      [n,3] fp32 unit vectors, row-major, contiguous
+ *   seed_vertex  first centre (the synthetic workloads use vertex 0)
+ * Outputs (all int32, caller-allocated):
+ *   centers  [P]   centre t = the not-yet-chosen vertex whose largest dot to
+ *                  centres 0..t-1 is smallest; ties -> lowest vertex index
+ *   owner    [n]   patch of each vertex = index of its nearest centre (largest
+ *                  dot), ties -> lowest patch index; a centre owns itself
+ *   offsets  [P+1] patch p holds members[offsets[p] .. offsets[p+1])
+ *   members  [n]   vertices grouped by patch, ascending vertex id in a patch
+ * Results are bit-identical to the fp64 definition.  Requires 1 <= P <= n,
+ * P <= 65535, n <= 2^24. */
+int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex,
+                    int* centers, int* owner, int* offsets, int* members,
+                    void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* Scratch bytes ssc_patch_scores_topk needs. */
+size_t ssc_patch_scores_topk_workspace_size(int PN, int PM, int d);
+
+/* Pool, score and select (project page "Geo-FlashAttention": pool source
+ * keys, score source patches using descriptors, keep the top R per target).
+ *   FN [nN, ldn], FM [nM, ldm]   descriptors (bf16 or fp32 per dtype)
+ *   offN/memN, offM/memM          patch tables from ssc_fps_patches
+ * Computes in fp64, in a fixed order (bit-exact):
+ *   mu_N(p) = mean over members of p of F_N (ascending vertex order, one divide)
+ *   score(p,q) = sum_{c=0..d-1} mu_N(p)_c * mu_M(q)_c  (in order, no FMA)
+ * Outputs: topk [PN,R] int32, per row the R best q by (score desc, q asc);
+ * scores [PN,PM] fp64 (nullable; when NULL the matrix lives in `ws`). */
+int ssc_patch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int ldm, int nM,
+                          int d, int dtype,
+                          const int* offN, const int* memN, int PN,
+                          const int* offM, const int* memM, int PM,
+                          int R, int* topk, double* scores,
+                          void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Dense coupling (project page, "Spatial-spectral coupling is attention").  */
+/*   S = scale * Q K^T, Pi = row softmax of S, O = Pi V,                     */
+/*   lse_i = ln sum_j exp(S_ij) (natural log).                               */
+/* Q [nN, ldq], K [nM, ldk], V [nM, ldv] in `dtype`; O [nN, ldo] fp32 and    */
+/* lse [nN] fp32.                                                            */
+/* ------------------------------------------------------------------------ */
+
+size_t ssc_dense_coupling_workspace_size(int nN, int nM, int d, int k, int dtype);
+
+int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk,
+                           const void* V, int ldv, int nN, int nM, int d, int k,
+                           float scale, int dtype, float* O, int ldo, float* lse,
+                           void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* Backward of a loss L with dL/dO = dO (fp32 [nN, lddo]), given the forward's
+ * O and lse.  Textbook softmax-matmul gradient with recompute from lse:
+ *   D_i = <dO_i, O_i>, P_ij = exp(S_ij - lse_i), dP_ij = <dO_i, V_j>,
+ *   dS_ij = P_ij (dP_ij - D_i), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO.
+ * On the bf16 path dO is rounded to bf16 once and that value is used
+ * throughout (D included).  dV may be NULL (the eigenbasis is not learned);
+ * dQ [nN, lddq], dK [nM, lddk], dV [nM, lddv] fp32 are overwritten. */
+int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
+                           const void* V, int ldv, int nN, int nM, int d, int k,
+                           float scale, int dtype, const float* O, int ldo,
+                           const float* lse, const float* dO, int lddo,
+                           float* dQ, int lddq, float* dK, int lddk,
+                           float* dV, int lddv,
+                           void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Geo-FlashAttention (project page, "Geo-FlashAttention"; digest,           */
+/* "Interpretation": each target patch computes the exact softmax over only  */
+/* its highest-scoring source patches).  Row i of target patch p attends to  */
+/* U(p) = union of the members of source patches topk[p, 0..R-1]; the        */
+/* softmax is normalised over U(p).  Patch tables as from ssc_fps_patches,   */
+/* topk as from ssc_patch_scores_topk (entries must be distinct).  Outputs   */
+/* are in vertex order, like the dense calls.                                */
+/* ------------------------------------------------------------------------ */
+
+size_t ssc_geo_coupling_workspace_size(int nN, int nM, int d, int k, int PN, int PM,
+                                       int R, int dtype);
+
+int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk,
+                         const void* V, int ldv, int nN, int nM, int d, int k,
+                         float scale, int dtype,
+                         const int* offN, const int* memN, int PN,
+                         const int* offM, const int* memM, int PM,
+                         const int* topk, int R,
+                         float* O, int ldo, float* lse,
+                         void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
+                         const void* V, int ldv, int nN, int nM, int d, int k,
+                         float scale, int dtype,
+                         const int* offN, const int* memN, int PN,
+                         const int* offM, const int* memM, int PM,
+                         const int* topk, int R,
+                         const float* O, int ldo, const float* lse,
+                         const float* dO, int lddo,
+                         float* dQ, int lddq, float* dK, int lddk,
+                         float* dV, int lddv,
+                         void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSC_H_ */

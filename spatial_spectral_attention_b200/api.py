@@ -1,0 +1,200 @@
+"""Python binding of libssc: the C calls of include/ssc.h under the same names.
+
+Argument marshalling only: every step of the computation runs in libssc's CUDA
+kernels.  PyTorch provides device memory (outputs and workspaces are allocated
+with torch) and the current CUDA stream.  Inputs must be CUDA tensors; nothing
+here falls back to a CPU computation.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._abi import check, lib
+
+SSC_BF16 = 0
+SSC_F32 = 1
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libssc calls take CUDA tensors")
+
+
+def _rowmajor(t):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D row-major tensor (unit column stride)")
+    return t.stride(0)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SSC_BF16
+    if t.dtype == torch.float32:
+        return SSC_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _workspace(nbytes, device):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def ssc_version():
+    return lib().ssc_version()
+
+
+def ssc_kernel_launches():
+    """Running count of the kernels libssc has enqueued."""
+    return int(lib().ssc_kernel_launches())
+
+
+def ssc_device_status(clear=True):
+    """Synchronises the current stream and returns the device status word as a
+    status code (0 ok, 6 a bounded wait ran out, 1 a bad index table entry)."""
+    out = ctypes.c_int(0)
+    check("ssc_device_status", lib().ssc_device_status(_stream(), int(clear), ctypes.byref(out)))
+    return out.value
+
+
+def ssc_set_wait_limit_ns(ns):
+    check("ssc_set_wait_limit_ns", lib().ssc_set_wait_limit_ns(int(ns)))
+
+
+def ssc_debug_wait_timeout(limit_ns):
+    check("ssc_debug_wait_timeout", lib().ssc_debug_wait_timeout(int(limit_ns), _stream()))
+
+
+def ssc_fps_patches(pts, P, seed_vertex=0):
+    """Geodesic FPS + Voronoi patches.  pts: fp32 [n,3] CUDA tensor.
+    Returns (centers [P], owner [n], offsets [P+1], members [n]) int32."""
+    _cuda(pts)
+    pts = pts.contiguous()
+    n = pts.shape[0]
+    dev = pts.device
+    centers = torch.empty(P, dtype=torch.int32, device=dev)
+    owner = torch.empty(n, dtype=torch.int32, device=dev)
+    offsets = torch.empty(P + 1, dtype=torch.int32, device=dev)
+    members = torch.empty(n, dtype=torch.int32, device=dev)
+    nb = lib().ssc_fps_patches_workspace_size(n, P)
+    ws = _workspace(nb, dev)
+    check("ssc_fps_patches", lib().ssc_fps_patches(
+        _ptr(pts), n, P, seed_vertex, _ptr(centers), _ptr(owner), _ptr(offsets), _ptr(members),
+        _ptr(ws), ws.numel(), _stream()))
+    return centers, owner, offsets, members
+
+
+def ssc_patch_scores_topk(FN, FM, offN, memN, offM, memM, R, return_scores=False):
+    """Patch-mean scores and the top-R source patches of every target patch."""
+    _cuda(FN, FM, offN, memN, offM, memM)
+    d = FN.shape[1]
+    PN, PM = offN.numel() - 1, offM.numel() - 1
+    dev = FN.device
+    topk = torch.empty((PN, R), dtype=torch.int32, device=dev)
+    scores = torch.empty((PN, PM), dtype=torch.float64, device=dev) if return_scores else None
+    ws = _workspace(lib().ssc_patch_scores_topk_workspace_size(PN, PM, d), dev)
+    check("ssc_patch_scores_topk", lib().ssc_patch_scores_topk(
+        _ptr(FN), _rowmajor(FN), FN.shape[0], _ptr(FM), _rowmajor(FM), FM.shape[0], d,
+        _dtype_code(FN), _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, R,
+        _ptr(topk), _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return (topk, scores) if return_scores else topk
+
+
+def _qkv(Q, K, V):
+    _cuda(Q, K, V)
+    if not (Q.dtype == K.dtype == V.dtype):
+        raise ValueError("Q, K and V must share one dtype")
+    return _rowmajor(Q), _rowmajor(K), _rowmajor(V), _dtype_code(Q)
+
+
+def ssc_dense_coupling_fwd(Q, K, V, scale, workspace=None):
+    """Dense coupling: O = softmax(scale Q K^T) V (fp32 [nN,k]) and lse (fp32 [nN])."""
+    ldq, ldk, ldv, dt = _qkv(Q, K, V)
+    nN, d = Q.shape
+    nM, k = V.shape
+    O = torch.empty((nN, k), dtype=torch.float32, device=Q.device)
+    lse = torch.empty(nN, dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_dense_coupling_workspace_size(nN, nM, d, k, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    check("ssc_dense_coupling_fwd", lib().ssc_dense_coupling_fwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(O), k, _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return O, lse
+
+
+def ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=None):
+    """Gradients (dQ, dK, dV or None) of the dense coupling for upstream dO (fp32)."""
+    ldq, ldk, ldv, dt = _qkv(Q, K, V)
+    _cuda(O, lse, dO)
+    nN, d = Q.shape
+    nM, k = V.shape
+    dev = Q.device
+    dQ = torch.empty((nN, d), dtype=torch.float32, device=dev)
+    dK = torch.empty((nM, d), dtype=torch.float32, device=dev)
+    dV = torch.empty((nM, k), dtype=torch.float32, device=dev) if need_dV else None
+    O, dO, lse = O.contiguous(), dO.contiguous(), lse.contiguous()
+    nb = lib().ssc_dense_coupling_workspace_size(nN, nM, d, k, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    check("ssc_dense_coupling_bwd", lib().ssc_dense_coupling_bwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(O), O.stride(0), _ptr(lse), _ptr(dO), dO.stride(0),
+        _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(), _stream()))
+    return dQ, dK, dV
+
+
+def _patches(offN, memN, offM, memM, topk):
+    _cuda(offN, memN, offM, memM, topk)
+    for t in (offN, memN, offM, memM, topk):
+        if t.dtype != torch.int32:
+            raise ValueError("patch tables must be int32")
+    return offN.numel() - 1, offM.numel() - 1, topk.shape[1]
+
+
+def ssc_geo_coupling_fwd(Q, K, V, scale, offN, memN, offM, memM, topk, workspace=None):
+    """Geo-FlashAttention forward: (O fp32 [nN,k], lse fp32 [nN]) in vertex order."""
+    ldq, ldk, ldv, dt = _qkv(Q, K, V)
+    PN, PM, R = _patches(offN, memN, offM, memM, topk)
+    nN, d = Q.shape
+    nM, k = V.shape
+    O = torch.empty((nN, k), dtype=torch.float32, device=Q.device)
+    lse = torch.empty(nN, dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_geo_coupling_workspace_size(nN, nM, d, k, PN, PM, R, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    topk = topk.contiguous()
+    check("ssc_geo_coupling_fwd", lib().ssc_geo_coupling_fwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
+        _ptr(O), k, _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return O, lse
+
+
+def ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, scale, offN, memN, offM, memM, topk,
+                         need_dV=False, workspace=None):
+    """Geo-FlashAttention backward: (dQ, dK, dV or None) in vertex order."""
+    ldq, ldk, ldv, dt = _qkv(Q, K, V)
+    PN, PM, R = _patches(offN, memN, offM, memM, topk)
+    _cuda(O, lse, dO)
+    nN, d = Q.shape
+    nM, k = V.shape
+    dev = Q.device
+    dQ = torch.empty((nN, d), dtype=torch.float32, device=dev)
+    dK = torch.empty((nM, d), dtype=torch.float32, device=dev)
+    dV = torch.empty((nM, k), dtype=torch.float32, device=dev) if need_dV else None
+    O, dO, lse, topk = O.contiguous(), dO.contiguous(), lse.contiguous(), topk.contiguous()
+    nb = lib().ssc_geo_coupling_workspace_size(nN, nM, d, k, PN, PM, R, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    check("ssc_geo_coupling_bwd", lib().ssc_geo_coupling_bwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
+        _ptr(O), O.stride(0), _ptr(lse), _ptr(dO), dO.stride(0),
+        _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(), _stream()))
+    return dQ, dK, dV

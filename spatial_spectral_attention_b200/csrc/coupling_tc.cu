@@ -1,0 +1,860 @@
+// coupling_tc.cu -- the bf16 coupling on 5th-generation tensor cores (sm_100a).
+//
+// Operation ("Spatial-Spectral Coupling as Attention", project page, section
+// "Spatial-spectral coupling is attention"): O = softmax(s Q K^T) V with
+// Q = F_N, K = F_M, V = Phi_M, plus lse; its backward with recompute from lse
+// (a training step, section "Results").  Geo-FlashAttention (section
+// "Geo-FlashAttention") is the same kernel driven by a different tile
+// schedule: each row tile of a target patch visits only the key rows of its
+// selected source patches, which the patch-major gather made contiguous.
+//
+// Work unit: a RowTile (<= 128 query rows) and its list of KeySegs (<= 128
+// key rows each).  CTAs are persistent (one per SM: the kernel claims all 512
+// TMEM columns) and walk the tile list round-robin.
+//
+// Forward, per CTA (warp roles):
+//   warp 0      TMA producer: Q tile once per row tile, K/V tiles into a
+//               2-stage ring (128B-swizzled boxes of 64 columns; the k % 64
+//               remainder of V in a 32B/64B-swizzled box).
+//   warp 1      MMA issuer (one thread) and TMEM owner:
+//                 S_j = Q K_j^T            (SS, K-major x K-major, M=N=128)
+//                 O  += P_j V_j            (TS: P from TMEM, V MN-major)
+//               with S double-buffered in TMEM columns [0,128) and [128,256)
+//               and O in [256, 256+kp).
+//   warps 2-5   softmax, one thread per query row (TMEM lane): row max, exp2,
+//               row sum, P written back over S as packed bf16; O is rescaled in
+//               TMEM only when the running max grows by more than 2^8
+//               (otherwise the stale max is kept, which bounds P by 256);
+//               epilogue O / l and lse.
+// Backward (query-stationary, one row tile per pass, key tiles streamed):
+//                 dP_j = dO V_j^T          (SS, K-major, K = kp)
+//                 S_j  = Q K_j^T
+//   compute     P = exp2(S s log2e - lse log2e), dS = P (dP - D) -> bf16 in a
+//               128B-swizzled smem tile [q][keys]
+//                 dQ  += dS K_j            (SS, dS K-major, K_j MN-major)
+//                 dKp  = dS^T Q            (SS, both MN-major views)
+//   compute     dKp (TMEM) -> scale -> fp32 vector atomics into dK
+//   end         dQ (TMEM) -> scale -> store.
+//   A second pass with kDV computes dV = P^T dO the same way when requested.
+//
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
+// SSC timeout in the status word, every role leaves its loop, the MMA thread
+// drains its tensor-core work and TMEM is freed before the CTA exits.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+namespace ssc {
+namespace {
+
+constexpr int kChunk = 128 * 128;  // bytes of a 128-row x 64-col bf16 swizzled box
+constexpr int kThreadsFwd = 192;
+constexpr int kThreadsBwd = 192;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct TensorMaps {
+  CUtensorMap q;     // box {64, 128}, SW128
+  CUtensorMap k;     // box {64, 128}, SW128
+  CUtensorMap v;     // box {64, 128}, SW128
+  CUtensorMap vr;    // box {vr, 128}, SW32/SW64 (remainder columns of V)
+  CUtensorMap g;     // dO: box {64, 128}, SW128
+  CUtensorMap gr;    // dO remainder
+};
+
+struct TcParams {
+  const RowTile* tiles;
+  const KeySeg* segs;
+  const int* ntiles_dev;
+  int ntiles_host;
+  const int* row_map;
+  const int* col_map;
+  int d, k, kp, qch, vf, vr;
+  int nq, nk;        // rows of Q (and of the outputs O, lse, dQ) and of K/V (dK, dV)
+  float scale_log2;  // scale * log2(e)
+  float scale;
+  float* O;
+  int ldo;
+  float* lse;
+  // backward
+  const float* lse_in;  // row order of Q
+  const float* Dvec;
+  float* dQ;
+  int lddq;
+  float* dK;
+  int lddk;
+  float* dV;
+  int lddv;
+  int vec_atomics;
+  WaitCtl ctl;
+};
+
+__device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, uint32_t col) {
+  return base + ((uint32_t)(32 * (warp & 3)) << 16) + col;
+}
+
+// Bytes of one V (or dO) tile in shared memory: vf full 64-col chunks plus the
+// remainder box.
+__host__ __device__ inline int vtile_bytes(int vf, int vr) { return vf * kChunk + 128 * vr * 2; }
+__host__ __device__ inline uint32_t rem_swizzle(int vr) { return vr == 16 ? kSw32 : kSw64; }
+
+// ------------------------------------------------------------------ forward
+__global__ void __launch_bounds__(kThreadsFwd, 1)
+    tc_fwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_q_full, bar_q_empty, bar_kv_full[2], bar_kv_empty[2], bar_s_full[2],
+      bar_p_full[2], bar_o_full, bar_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
+  const int qbytes = p.qch * kChunk;
+  const int vbytes = vtile_bytes(p.vf, p.vr);
+  const uint32_t sQ = sbase;
+  const uint32_t sK0 = sQ + qbytes;
+  const uint32_t sV0 = sK0 + 2 * qbytes;
+  (void)gbase;
+  const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_kv_full[i], 1);
+      mbar_init(&bar_kv_empty[i], 1);
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_p_full[i], 128);
+    }
+    mbar_init(&bar_o_full, 1);
+    mbar_init(&bar_drain, 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm.q);
+    tma_prefetch_desc(&tm.k);
+    tma_prefetch_desc(&tm.v);
+    if (p.vr) tma_prefetch_desc(&tm.vr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      int q_issued = -1;
+      const uint32_t kv_bytes = qbytes + vbytes;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
+        const RowTile tile = p.tiles[t];
+        if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        mbar_arrive_expect_tx(&bar_q_full, qbytes);
+        for (int c = 0; c < p.qch; ++c)
+          tma_load_2d(smem_raw + (sQ - smem_u32(smem_raw)) + c * kChunk, &tm.q, 64 * c, tile.row0,
+                      &bar_q_full);
+        q_issued = (int)tcount;
+        bool ok = true;
+        for (int j = 0; j < tile.nseg; ++j, ++it) {
+          const KeySeg sg = p.segs[tile.seg0 + j];
+          const int st = it & 1;
+          if (it >= 2 && !mbar_wait(&bar_kv_empty[st], ((it >> 1) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_kv_full[st], kv_bytes);
+          uint8_t* dk = smem_raw + (sK0 - smem_u32(smem_raw)) + st * qbytes;
+          uint8_t* dv = smem_raw + (sV0 - smem_u32(smem_raw)) + st * vbytes;
+          for (int c = 0; c < p.qch; ++c)
+            tma_load_2d(dk + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_kv_full[st]);
+          for (int c = 0; c < p.vf; ++c)
+            tma_load_2d(dv + c * kChunk, &tm.v, 64 * c, sg.key0, &bar_kv_full[st]);
+          if (p.vr) tma_load_2d(dv + p.vf * kChunk, &tm.vr, 64 * p.vf, sg.key0, &bar_kv_full[st]);
+        }
+        if (!ok) break;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        if (q_issued >= 0) mbar_wait(&bar_q_full, q_issued & 1, p.ctl, &never);
+        for (uint32_t g = it >= 2 ? it - 2 : 0; g < it; ++g)
+          mbar_wait(&bar_kv_full[g & 1], (g >> 1) & 1, p.ctl, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (p.vf > 0 ? p.vf : 1), 0, 1);
+      const uint32_t idesc_pvr = make_idesc_bf16(128, p.vr > 0 ? p.vr : 16, 0, 1);
+      const uint32_t o_col = tmem + 256;
+      const uint32_t rsw = rem_swizzle(p.vr);
+      const uint32_t rrow = (uint32_t)p.vr * 2;  // bytes per row of the remainder box
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      auto issue_s = [&](uint32_t g) -> bool {
+        const int st = g & 1;
+        if (!mbar_wait(&bar_kv_full[st], (g >> 1) & 1, p.ctl, abort)) return false;
+        tc_fence_after();
+        const uint32_t sk = sK0 + st * qbytes;
+        const uint32_t d_tmem = tmem + (g & 1) * 128;
+        for (int kk = 0; kk < p.d / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+          mma_ss(d_tmem, make_sdesc(sQ + off, 16, 1024, kSw128), make_sdesc(sk + off, 16, 1024, kSw128),
+                 idesc_s, kk > 0);
+        }
+        mma_commit(&bar_s_full[g & 1]);
+        return true;
+      };
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+        const RowTile tile = p.tiles[t];
+        const int nk = tile.nseg;
+        if (!mbar_wait(&bar_q_full, tcount & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < std::min(2, nk) && ok; ++j) ok = issue_s(it + j);
+        for (int j = 0; j < nk && ok; ++j) {
+          const uint32_t g = it + j;
+          const int buf = g & 1, st = g & 1;
+          if (!mbar_wait(&bar_p_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sv = sV0 + st * vbytes;
+          const uint32_t a_tmem = tmem + buf * 128;
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            if (p.vf > 0)
+              mma_ts(o_col, a_tmem + kk * 8, make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128),
+                     idesc_pv, acc);
+            if (p.vr > 0)
+              mma_ts(o_col + 64 * p.vf, a_tmem + kk * 8,
+                     make_sdesc(sv + p.vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+                     idesc_pvr, acc);
+          }
+          mma_commit(&bar_kv_empty[st]);
+          mma_commit(&bar_o_full);
+          if (j + 2 < nk) ok = issue_s(g + 2);
+        }
+        mma_commit(&bar_q_empty);
+        it += nk;
+      }
+      // drain: wait until every tensor-core op issued here has completed
+      mma_commit(&bar_drain);
+      WaitCtl c2 = p.ctl;
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, c2, &never);
+    }
+  } else {
+    // ---------------- softmax / epilogue (warps 2..5)
+    const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = row within the tile
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const RowTile tile = p.tiles[t];
+      const int nk = tile.nseg;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nk; ++j) {
+        const uint32_t g = it + j;
+        const int buf = g & 1;
+        if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nkeys = p.segs[tile.seg0 + j].nkeys;
+        uint32_t r[4][32];
+        const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(sa + 32 * c, r[c]);
+        tmem_ld_wait();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float x = __uint_as_float(r[c][i]);
+            if (32 * c + i >= nkeys) x = -INFINITY;
+            r[c][i] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        const float m_new = fmaxf(m, mx * p.scale_log2);
+        const bool need = m_new > m + 8.0f;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds P_0..P_{j-1} V: wait for PV_{j-1}, then rescale in TMEM
+          if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = need ? ex2_approx(m - m_new) : 1.0f;
+          const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
+          for (int c0 = 0; c0 < p.kp; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(oa + c0, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st16(oa + c0, o);
+          }
+          tmem_st_wait();
+          l *= f;
+          if (need) m = m_new;
+        } else if (need) {
+          m = m_new;
+        }
+        const float neg_m = -m;
+        float rs = 0.f;
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i]), p.scale_log2, neg_m));
+            const float a1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i + 1]), p.scale_log2, neg_m));
+            rs += a0 + a1;
+            pk[c][i] = pack_bf16x2(a0, a1);
+          }
+        l += rs;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(sa + 16 * c, pk[c]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[buf]);
+      }
+      if (!ok) break;
+      // epilogue: O / l, lse
+      const uint32_t glast = it + nk - 1;
+      if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      const int row = tile.row0 + lrow;
+      int orow = (lrow < tile.nrows && row < p.nq) ? (p.row_map ? p.row_map[row] : row) : -1;
+      if (orow >= p.nq) orow = -1;
+      const bool live = orow >= 0;
+      if (!live) orow = 0;
+      float* optr = p.O + (size_t)orow * p.ldo;
+      const float inv = 1.0f / l;
+      const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
+      for (int c0 = 0; c0 < p.kp; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(oa + c0, o);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+        }
+      }
+      if (live) p.lse[orow] = (m + log2f(l)) * kLn2;
+      it += nk;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ backward
+// kDV = false: dQ (stored) and dK (atomics).  kDV = true: dV (atomics).
+template <bool kDV>
+__global__ void __launch_bounds__(kThreadsBwd, 1)
+    tc_bwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_qg_full, bar_qg_empty, bar_k_full, bar_k_empty, bar_v_full, bar_v_empty,
+      bar_sdp_full, bar_ds_full, bar_dkp_full, bar_dq_full, bar_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  const int qbytes = p.qch * kChunk;
+  const int vbytes = vtile_bytes(p.vf, p.vr);
+  const uint32_t sQ = sbase;
+  const uint32_t sG = sQ + qbytes;           // dO tile
+  const uint32_t sK = sG + vbytes;
+  const uint32_t sV = sK + qbytes;           // unused in the dV pass
+  const uint32_t sS = sV + (kDV ? 0 : vbytes);  // dS (or P) tile [q][keys], 2 chunks
+  auto gptr = [&](uint32_t s) { return smem_raw + (s - base_u); };
+  const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_qg_full, 1);
+    mbar_init(&bar_qg_empty, 1);
+    mbar_init(&bar_k_full, 1);
+    mbar_init(&bar_k_empty, 1);
+    mbar_init(&bar_v_full, 1);
+    mbar_init(&bar_v_empty, 1);
+    mbar_init(&bar_sdp_full, 1);
+    mbar_init(&bar_ds_full, 128);
+    mbar_init(&bar_dkp_full, 1);
+    mbar_init(&bar_dq_full, 1);
+    mbar_init(&bar_drain, 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+  // TMEM columns
+  const uint32_t c_s = 0, c_dp = 128, c_dq = 256, c_dkp = kDV ? 256 : 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      int q_issued = -1, k_last = -1, v_last = -1;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
+        const RowTile tile = p.tiles[t];
+        if (tcount > 0 && !mbar_wait(&bar_qg_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        q_issued = (int)tcount;
+        mbar_arrive_expect_tx(&bar_qg_full, qbytes + vbytes);
+        for (int c = 0; c < p.qch; ++c)
+          tma_load_2d(gptr(sQ) + c * kChunk, &tm.q, 64 * c, tile.row0, &bar_qg_full);
+        for (int c = 0; c < p.vf; ++c)
+          tma_load_2d(gptr(sG) + c * kChunk, &tm.g, 64 * c, tile.row0, &bar_qg_full);
+        if (p.vr) tma_load_2d(gptr(sG) + p.vf * kChunk, &tm.gr, 64 * p.vf, tile.row0, &bar_qg_full);
+        bool ok = true;
+        for (int j = 0; j < tile.nseg; ++j, ++it) {
+          const KeySeg sg = p.segs[tile.seg0 + j];
+          if (!kDV) {
+            if (it >= 1 && !mbar_wait(&bar_v_empty, (it - 1) & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bar_v_full, vbytes);
+            for (int c = 0; c < p.vf; ++c)
+              tma_load_2d(gptr(sV) + c * kChunk, &tm.v, 64 * c, sg.key0, &bar_v_full);
+            if (p.vr) tma_load_2d(gptr(sV) + p.vf * kChunk, &tm.vr, 64 * p.vf, sg.key0, &bar_v_full);
+            v_last = (int)it;
+          }
+          if (it >= 1 && !mbar_wait(&bar_k_empty, (it - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_k_full, qbytes);
+          for (int c = 0; c < p.qch; ++c)
+            tma_load_2d(gptr(sK) + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_k_full);
+          k_last = (int)it;
+        }
+        if (!ok) break;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        if (q_issued >= 0) mbar_wait(&bar_qg_full, q_issued & 1, p.ctl, &never);
+        if (k_last >= 0) mbar_wait(&bar_k_full, k_last & 1, p.ctl, &never);
+        if (v_last >= 0) mbar_wait(&bar_v_full, v_last & 1, p.ctl, &never);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_dq = make_idesc_bf16(128, p.d, 0, 1);
+      const uint32_t idesc_dkp = make_idesc_bf16(128, p.d, 1, 1);
+      const uint32_t idesc_dv = make_idesc_bf16(128, 64 * (p.vf > 0 ? p.vf : 1), 1, 1);
+      const uint32_t idesc_dvr = make_idesc_bf16(128, p.vr > 0 ? p.vr : 16, 1, 1);
+      const uint32_t rsw = rem_swizzle(p.vr);
+      const uint32_t rrow = (uint32_t)p.vr * 2;
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+        const RowTile tile = p.tiles[t];
+        if (!mbar_wait(&bar_qg_full, tcount & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < tile.nseg && ok; ++j, ++it) {
+          if (!kDV) {
+            // dP = dO V^T (K = kp)
+            if (!mbar_wait(&bar_v_full, it & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            int kk = 0;
+            for (int c = 0; c < p.vf; ++c)
+              for (int u = 0; u < 4; ++u, ++kk) {
+                const uint32_t off = c * kChunk + u * 32;
+                mma_ss(tmem + c_dp, make_sdesc(sG + off, 16, 1024, kSw128),
+                       make_sdesc(sV + off, 16, 1024, kSw128), idesc_s, kk > 0);
+              }
+            for (int u = 0; u < p.vr / 16; ++u, ++kk) {
+              const uint32_t off = p.vf * kChunk + u * 32;
+              mma_ss(tmem + c_dp, make_sdesc(sG + off, 16, 8 * rrow, rsw),
+                     make_sdesc(sV + off, 16, 8 * rrow, rsw), idesc_s, kk > 0);
+            }
+            mma_commit(&bar_v_empty);
+          }
+          // S = Q K^T
+          if (!mbar_wait(&bar_k_full, it & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int kk = 0; kk < p.d / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + c_s, make_sdesc(sQ + off, 16, 1024, kSw128),
+                   make_sdesc(sK + off, 16, 1024, kSw128), idesc_s, kk > 0);
+          }
+          mma_commit(&bar_sdp_full);
+          // wait for dS (or P) in shared memory
+          if (!mbar_wait(&bar_ds_full, it & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!kDV) {
+            // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t aoff = (kk >> 2) * kChunk + (kk & 3) * 32;
+              mma_ss(tmem + c_dq, make_sdesc(sS + aoff, 16, 1024, kSw128),
+                     make_sdesc(sK + kk * 2048, kChunk, 1024, kSw128), idesc_dq,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bar_k_empty);
+            // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                     make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
+          } else {
+            mma_commit(&bar_k_empty);
+            // dVp = P^T dO : A = P viewed MN-major (M = keys), B = dO MN-major (N = k)
+            for (int kk = 0; kk < 8; ++kk) {
+              if (p.vf > 0)
+                mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                       make_sdesc(sG + kk * 2048, kChunk, 1024, kSw128), idesc_dv, kk > 0);
+              if (p.vr > 0)
+                mma_ss(tmem + c_dkp + 64 * p.vf, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                       make_sdesc(sG + p.vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+                       idesc_dvr, kk > 0);
+            }
+          }
+          mma_commit(&bar_dkp_full);
+        }
+        if (!ok) break;
+        mma_commit(&bar_dq_full);
+        mma_commit(&bar_qg_empty);
+      }
+      mma_commit(&bar_drain);
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
+    }
+  } else {
+    // ---------------- compute (warps 2..5): one thread per query row for S/dP,
+    // one thread per key row for the dK / dV flush.
+    const int lrow = 32 * (warp & 3) + lane;
+    uint32_t it = 0, tcount = 0;
+    const int kt_out = kDV ? p.kp : p.d;  // columns of the partial to flush
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+      const RowTile tile = p.tiles[t];
+      const int qrow = tile.row0 + lrow;
+      const bool live_row = lrow < tile.nrows && qrow < p.nq;
+      const float lse2 = live_row ? p.lse_in[qrow] * kLog2e : 0.f;
+      const float Di = (!kDV && live_row) ? p.Dvec[qrow] : 0.f;
+      bool ok = true;
+      for (int j = 0; j < tile.nseg; ++j, ++it) {
+        const KeySeg sg = p.segs[tile.seg0 + j];
+        if (!mbar_wait(&bar_sdp_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem_lane_addr(tmem, warp, 0);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], dp[32];
+          tmem_ld32(ta + c_s + 32 * c, s);
+          if (!kDV) tmem_ld32(ta + c_dp + 32 * c, dp);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float v2[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int col = 32 * c + 2 * i + h;
+              float pr = ex2_approx(fmaf(__uint_as_float(s[2 * i + h]), p.scale_log2, -lse2));
+              if (col >= sg.nkeys || !live_row) pr = 0.f;
+              v2[h] = kDV ? pr : pr * (__uint_as_float(dp[2 * i + h]) - Di);
+            }
+            pk[i] = pack_bf16x2(v2[0], v2[1]);
+          }
+          // row lrow, keys [32c, 32c+32): chunk c/2, 16-byte units (c&1)*4 + 0..3
+          const uint32_t rowb = sS + (c >> 1) * kChunk + lrow * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t unit = ((c & 1) * 4 + u) ^ (lrow & 7);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(rowb + unit * 16),
+                         "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar_ds_full);
+        // flush the partial dK (or dV) of this key tile: thread = key row
+        if (!mbar_wait(&bar_dkp_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int krow = sg.key0 + lrow;
+        int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
+        if (okey >= p.nk) okey = -1;
+        const bool live_key = okey >= 0;
+        if (!live_key) okey = 0;
+        float* dst = kDV ? p.dV + (size_t)okey * p.lddv : p.dK + (size_t)okey * p.lddk;
+        const int ncols = kDV ? p.k : p.d;
+        const float mul = kDV ? 1.0f : p.scale;
+        for (int c0 = 0; c0 < kt_out; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(ta + c_dkp + c0, o);
+          tmem_ld_wait();
+          if (live_key) {
+            if (p.vec_atomics && c0 + 16 <= ncols) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4) {
+                float4 v = make_float4(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul,
+                                       __uint_as_float(o[i + 2]) * mul,
+                                       __uint_as_float(o[i + 3]) * mul);
+                atomicAdd(reinterpret_cast<float4*>(dst + c0 + i), v);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (c0 + i < ncols) atomicAdd(dst + c0 + i, __uint_as_float(o[i]) * mul);
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      if (!kDV) {
+        if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
+        tc_fence_after();
+        // TMEM loads are warp-collective: every lane loads, live rows store
+        int orow = live_row ? (p.row_map ? p.row_map[qrow] : qrow) : -1;
+        const bool store_row = orow >= 0 && orow < p.nq;
+        if (!store_row) orow = 0;
+        float* dq = p.dQ + (size_t)orow * p.lddq;
+        const uint32_t ta = tmem_lane_addr(tmem, warp, c_dq);
+        for (int c0 = 0; c0 < p.d; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(ta + c0, o);
+          tmem_ld_wait();
+          if (store_row) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dq[c0 + i] = __uint_as_float(o[i]) * p.scale;
+          }
+        }
+      } else {
+        if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+__global__ void wait_probe_kernel(WaitCtl ctl) {
+  __shared__ uint64_t bar;
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl, &s_abort);  // nothing ever arrives
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] with leading dimension ld (elements); box of
+// {box_cols, 128}; columns >= cols and rows >= rows read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_cols,
+              CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle rem_sw_host(int vr) {
+  return vr == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
+}
+
+int padded_k(int k) {
+  int kp = (k + 15) / 16 * 16;
+  if (kp % 64 == 48) kp += 16;
+  return kp;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+void fill_common(const TcArgs& a, TcParams& p) {
+  std::memset(&p, 0, sizeof(p));
+  p.tiles = a.tiles;
+  p.segs = a.segs;
+  p.ntiles_dev = a.ntiles_dev;
+  p.ntiles_host = a.ntiles_host;
+  p.row_map = a.row_map;
+  p.col_map = a.col_map;
+  p.d = a.d;
+  p.k = a.k;
+  p.nq = a.nQrows;
+  p.nk = a.nKrows;
+  p.kp = padded_k(a.k);
+  p.qch = a.d / 64;
+  p.vf = p.kp / 64;
+  p.vr = p.kp % 64;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+}
+
+}  // namespace
+
+bool tc_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
+
+cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
+                          const WaitCtl& ctl) {
+  TcParams p;
+  fill_common(a, p);
+  p.O = O;
+  p.ldo = ldo;
+  p.lse = lse;
+  p.ctl = ctl;
+  TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (!make_map(&tm.q, a.Q, a.nQrows, a.d, a.ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.k, a.K, a.nKrows, a.d, a.ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.v, a.V, a.nKrows, a.k, a.ldv, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (p.vr && !make_map(&tm.vr, a.V, a.nKrows, a.k, a.ldv, p.vr, rem_sw_host(p.vr)))
+    return cudaErrorInvalidValue;
+  const int smem = 1024 + p.qch * kChunk * 3 + 2 * vtile_bytes(p.vf, p.vr);
+  cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
+  const int grid = std::max(1, std::min(work, num_sms()));
+  tc_fwd_kernel<<<grid, kThreadsFwd, smem, st>>>(tm, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,
+                          const float* D, float* dQ, int lddq, float* dK, int lddk, float* dV,
+                          int lddv, cudaStream_t st, const WaitCtl& ctl) {
+  TcParams p;
+  fill_common(a, p);
+  p.lse_in = lse;
+  p.Dvec = D;
+  p.dQ = dQ;
+  p.lddq = lddq;
+  p.dK = dK;
+  p.lddk = lddk;
+  p.dV = dV;
+  p.lddv = lddv;
+  p.ctl = ctl;
+  TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (!make_map(&tm.q, a.Q, a.nQrows, a.d, a.ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.k, a.K, a.nKrows, a.d, a.ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.v, a.V, a.nKrows, a.k, a.ldv, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.g, dOb, a.nQrows, a.k, lddob, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (p.vr && (!make_map(&tm.vr, a.V, a.nKrows, a.k, a.ldv, p.vr, rem_sw_host(p.vr)) ||
+               !make_map(&tm.gr, dOb, a.nQrows, a.k, lddob, p.vr, rem_sw_host(p.vr))))
+    return cudaErrorInvalidValue;
+  const int vb = vtile_bytes(p.vf, p.vr);
+  const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
+  const int grid = std::max(1, std::min(work, num_sms()));
+  {
+    p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
+    const int smem = 1024 + 2 * p.qch * kChunk + 2 * vb + 2 * kChunk;
+    cudaError_t e =
+        cudaFuncSetAttribute(tc_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tc_bwd_kernel<false><<<grid, kThreadsBwd, smem, st>>>(tm, p);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (dV) {
+    p.vec_atomics = (lddv % 4 == 0) && (reinterpret_cast<uintptr_t>(dV) % 16 == 0);
+    const int smem = 1024 + 2 * p.qch * kChunk + vb + 2 * kChunk;
+    cudaError_t e =
+        cudaFuncSetAttribute(tc_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tc_bwd_kernel<true><<<grid, kThreadsBwd, smem, st>>>(tm, p);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl) {
+  wait_probe_kernel<<<1, 32, 0, st>>>(ctl);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ssc

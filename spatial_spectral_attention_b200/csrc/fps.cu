@@ -1,0 +1,434 @@
+// fps.cu -- geodesic farthest-point sampling, nearest-centre assignment and
+// the patch tables (offsets + members), bit-exact in fp64.
+//
+// Source: "Spatial-Spectral Coupling as Attention" digest, "Interpretation"
+// (the surface is partitioned with geodesic farthest-point sampling) and the
+// project page, "Geo-FlashAttention" (partition both shapes into patches).
+// On the unit sphere geodesic distance is the great-circle distance, which
+// falls as the dot product rises, so the kernel ranks on the fp64 dot
+// ((x0*y0 + x1*y1) + x2*y2) of the fp32 coordinates.
+//
+// Design: FPS is P dependent rounds (argmax of a running minimum distance), so
+// its cost is round latency, not bandwidth.  One thread-block cluster of CL
+// CTAs (16 where the GPU allows it) holds every point on chip: coordinates in
+// shared memory, the running largest dot and patch of each point in registers.
+// Each round a CTA reduces its candidate, pushes it into every CTA's shared
+// memory through DSMEM, and one cluster barrier later every CTA knows the next
+// centre.  No grid-wide synchronisation.
+#include <cfloat>
+#include <climits>
+#include <cooperative_groups.h>
+
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace ssc {
+namespace {
+
+constexpr int kFpsThreads = 1024;
+
+struct Cand {
+  double val;
+  int idx;
+};
+
+// a precedes b: smaller largest-dot (farther), ties to the lower vertex.
+__device__ __forceinline__ bool cand_before(const Cand& a, const Cand& b) {
+  return a.val < b.val || (a.val == b.val && a.idx < b.idx);
+}
+
+__device__ __forceinline__ double dot3_rn(float a0, float a1, float a2, float b0, float b1,
+                                          float b2) {
+  double p0 = __dmul_rn((double)a0, (double)b0);
+  double p1 = __dmul_rn((double)a1, (double)b1);
+  double p2 = __dmul_rn((double)a2, (double)b2);
+  return __dadd_rn(__dadd_rn(p0, p1), p2);
+}
+
+__device__ __forceinline__ Cand warp_min(Cand c) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Cand x;
+    x.val = __shfl_xor_sync(0xffffffffu, c.val, o);
+    x.idx = __shfl_xor_sync(0xffffffffu, c.idx, o);
+    if (cand_before(x, c)) c = x;
+  }
+  return c;
+}
+
+// Cluster FPS: the CTA of rank r owns points [r*per, min(n,(r+1)*per));
+// their coordinates sit in shared memory (structure of arrays), the running
+// largest dot and patch of each point in registers (PPT points per thread).
+template <int PPT>
+__global__ void __launch_bounds__(kFpsThreads, 1)
+    fps_cluster_kernel(const float* __restrict__ pts, int n, int P, int seed, int per,
+                       int* __restrict__ centers, int* __restrict__ owner) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  extern __shared__ float sx[];  // [3][PPT * kFpsThreads]
+  __shared__ Cand warp_c[kFpsThreads / 32];
+  __shared__ Cand slots[2][16];
+  __shared__ int s_next;
+
+  const int tid = threadIdx.x;
+  const int cap = PPT * kFpsThreads;
+  const int v0 = rank * per;
+  const int cnt = max(0, min(n - v0, per));
+  for (int i = tid; i < cnt; i += kFpsThreads) {
+    sx[i] = pts[3 * (size_t)(v0 + i)];
+    sx[cap + i] = pts[3 * (size_t)(v0 + i) + 1];
+    sx[2 * cap + i] = pts[3 * (size_t)(v0 + i) + 2];
+  }
+  double best[PPT];
+  int own[PPT];
+  uint32_t chosen = 0;
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    best[i] = -DBL_MAX;
+    own[i] = -1;
+    if (i * kFpsThreads + tid >= cnt) chosen |= 1u << i;  // padding never competes
+  }
+  __syncthreads();
+  int c = seed;
+  for (int t = 0; t < P; ++t) {
+    if (rank == 0 && tid == 0) centers[t] = c;
+    const float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
+                c2 = __ldg(pts + 3 * (size_t)c + 2);
+    Cand mine{DBL_MAX, INT_MAX};
+#pragma unroll
+    for (int i = 0; i < PPT; ++i) {
+      const int li = i * kFpsThreads + tid;
+      if (v0 + li == c) {
+        chosen |= 1u << i;
+        own[i] = t;
+      }
+      if (!(chosen >> i & 1u)) {
+        double g = dot3_rn(sx[li], sx[cap + li], sx[2 * cap + li], c0, c1, c2);
+        if (g > best[i]) {
+          best[i] = g;
+          own[i] = t;
+        }
+        Cand me{best[i], v0 + li};
+        if (cand_before(me, mine)) mine = me;
+      }
+    }
+    if (t + 1 == P) break;
+    mine = warp_min(mine);
+    if ((tid & 31) == 0) warp_c[tid >> 5] = mine;
+    __syncthreads();
+    if (tid < 32) {
+      Cand w = warp_c[tid];
+      w = warp_min(w);
+      if (tid < CL) {
+        // push this CTA's candidate into slot `rank` of CTA `tid`
+        Cand* dst = cluster.map_shared_rank(&slots[t & 1][rank], tid);
+        dst->val = w.val;
+        dst->idx = w.idx;
+      }
+    }
+    cluster.sync();
+    if (tid < 32) {
+      Cand w{DBL_MAX, INT_MAX};
+      if (tid < CL) w = slots[t & 1][tid];
+      w = warp_min(w);
+      if (tid == 0) s_next = w.idx;
+    }
+    __syncthreads();
+    c = s_next;
+  }
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    const int li = i * kFpsThreads + tid;
+    if (li < cnt) owner[v0 + li] = own[i];
+  }
+  cluster.sync();  // no CTA leaves while others may still write its slots
+}
+
+// Fallback for n beyond what the cluster holds on chip: the same rounds with
+// the per-point state in global memory.
+__global__ void __launch_bounds__(kFpsThreads, 1)
+    fps_cluster_mem_kernel(const float* __restrict__ pts, int n, int P, int seed,
+                           int* __restrict__ centers, int* __restrict__ owner,
+                           double* __restrict__ best, unsigned char* __restrict__ chosen) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  __shared__ Cand warp_c[kFpsThreads / 32];
+  __shared__ Cand slots[2][16];
+  __shared__ int s_next;
+  const int tid = threadIdx.x;
+  const int stride = CL * kFpsThreads;
+  for (int v = rank * kFpsThreads + tid; v < n; v += stride) {
+    best[v] = -DBL_MAX;
+    chosen[v] = 0;
+    owner[v] = -1;
+  }
+  int c = seed;
+  for (int t = 0; t < P; ++t) {
+    if (rank == 0 && tid == 0) centers[t] = c;
+    const float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
+                c2 = __ldg(pts + 3 * (size_t)c + 2);
+    Cand mine{DBL_MAX, INT_MAX};
+    for (int v = rank * kFpsThreads + tid; v < n; v += stride) {
+      if (v == c) {
+        chosen[v] = 1;
+        owner[v] = t;
+      }
+      if (!chosen[v]) {
+        double g = dot3_rn(pts[3 * (size_t)v], pts[3 * (size_t)v + 1], pts[3 * (size_t)v + 2], c0,
+                           c1, c2);
+        double b = best[v];
+        if (g > b) {
+          b = g;
+          best[v] = g;
+          owner[v] = t;
+        }
+        Cand me{b, v};
+        if (cand_before(me, mine)) mine = me;
+      }
+    }
+    if (t + 1 == P) break;
+    mine = warp_min(mine);
+    if ((tid & 31) == 0) warp_c[tid >> 5] = mine;
+    __syncthreads();
+    if (tid < 32) {
+      Cand w = warp_min(warp_c[tid]);
+      if (tid < CL) {
+        Cand* dst = cluster.map_shared_rank(&slots[t & 1][rank], tid);
+        dst->val = w.val;
+        dst->idx = w.idx;
+      }
+    }
+    cluster.sync();
+    if (tid < 32) {
+      Cand w{DBL_MAX, INT_MAX};
+      if (tid < CL) w = slots[t & 1][tid];
+      w = warp_min(w);
+      if (tid == 0) s_next = w.idx;
+    }
+    __syncthreads();
+    c = s_next;
+  }
+  cluster.sync();
+}
+
+// ---- patch tables
+__global__ void count_kernel(const int* __restrict__ owner, int n, int* __restrict__ counts) {
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < n; v += gridDim.x * blockDim.x)
+    atomicAdd(counts + owner[v], 1);
+}
+
+// Single-block exclusive scan: offsets[0] = 0, offsets[p+1] = sum counts[0..p].
+__global__ void __launch_bounds__(1024) scan_offsets_kernel(const int* __restrict__ counts, int P,
+                                                            int* __restrict__ offsets,
+                                                            int* __restrict__ cursor) {
+  __shared__ int part[1024];
+  const int tid = threadIdx.x;
+  const int per = (P + 1023) / 1024;
+  const int b = tid * per, e = min(P, b + per);
+  int s = 0;
+  for (int p = b; p < e; ++p) s += counts[p];
+  part[tid] = s;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    int x = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += x;
+    __syncthreads();
+  }
+  int run = part[tid] - s;
+  for (int p = b; p < e; ++p) {
+    offsets[p] = run;
+    cursor[p] = run;
+    run += counts[p];
+  }
+  if (tid == 1023) offsets[P] = part[1023];
+}
+
+__global__ void fill_kernel(const int* __restrict__ owner, int n, int* __restrict__ cursor,
+                            int* __restrict__ members) {
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < n; v += gridDim.x * blockDim.x)
+    members[atomicAdd(cursor + owner[v], 1)] = v;
+}
+
+constexpr int kSortCap = 4096;
+
+// Puts the members of every patch in ascending vertex order: a bitonic sort in
+// shared memory for patches up to kSortCap vertices, an ordered compaction of
+// the owner array for larger ones (there are at most n / kSortCap of those).
+__global__ void __launch_bounds__(512) sort_segments_kernel(const int* __restrict__ owner, int n,
+                                                            const int* __restrict__ offsets,
+                                                            int* __restrict__ members) {
+  __shared__ int buf[kSortCap];
+  __shared__ int warp_tot[16];
+  const int p = blockIdx.x;
+  const int b = offsets[p], len = offsets[p + 1] - b;
+  const int tid = threadIdx.x;
+  if (len <= 1) return;
+  if (len <= kSortCap) {
+    int m = 1;
+    while (m < len) m <<= 1;
+    for (int i = tid; i < m; i += blockDim.x) buf[i] = i < len ? members[b + i] : INT_MAX;
+    __syncthreads();
+    for (int size = 2; size <= m; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < m; i += blockDim.x) {
+          int j = i ^ stride;
+          if (j > i) {
+            bool up = (i & size) == 0;
+            int a = buf[i], c = buf[j];
+            if ((a > c) == up) {
+              buf[i] = c;
+              buf[j] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = tid; i < len; i += blockDim.x) members[b + i] = buf[i];
+    return;
+  }
+  // ordered compaction over all vertices
+  int base = b;
+  for (int v0 = 0; v0 < n; v0 += blockDim.x) {
+    int v = v0 + tid;
+    int flag = (v < n && owner[v] == p) ? 1 : 0;
+    unsigned bal = __ballot_sync(0xffffffffu, flag);
+    int lane = tid & 31, w = tid >> 5;
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int i = 0; i < (int)(blockDim.x / 32); ++i) {
+      if (i < w) before += warp_tot[i];
+      total += warp_tot[i];
+    }
+    if (flag) members[base + before + __popc(bal & ((1u << lane) - 1u))] = v;
+    base += total;
+    __syncthreads();
+  }
+}
+
+int fps_cluster_size() {
+  static int cl = -1;
+  if (cl < 0) {
+    cl = 8;
+    if (cudaFuncSetAttribute(fps_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1) == cudaSuccess)
+      cl = 16;
+    cudaGetLastError();
+  }
+  return cl;
+}
+
+template <int PPT>
+cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, int* owner, int CL,
+                       cudaStream_t st) {
+  auto kern = fps_cluster_kernel<PPT>;
+  const int smem = 3 * PPT * kFpsThreads * (int)sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  const int per = (n + CL - 1) / CL;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL);
+  cfg.blockDim = dim3(kFpsThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, pts, n, P, seed, per, centers, owner);
+}
+
+}  // namespace
+
+size_t fps_workspace_bytes(int n, int P) {
+  Carve c(nullptr);
+  c.take<int>(P);       // counts
+  c.take<int>(P);       // cursor
+  c.take<double>(n);    // best (memory-resident fallback)
+  c.take<uint8_t>(n);   // chosen
+  return c.used + 256;
+}
+
+cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* centers, int* owner,
+                               int* offsets, int* members, void* ws, cudaStream_t st,
+                               const WaitCtl&) {
+  Carve c(ws);
+  int* counts = c.take<int>(P);
+  int* cursor = c.take<int>(P);
+  double* best = c.take<double>(n);
+  uint8_t* chosen = c.take<uint8_t>(n);
+  int CL = fps_cluster_size();
+  if (CL == 16) {
+    // make sure a 16-CTA cluster of this shape can be resident, else use 8
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(16);
+    q.blockDim = dim3(kFpsThreads);
+    q.dynamicSmemBytes = 3 * 16 * kFpsThreads * sizeof(float);
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 16;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int nclusters = 0;
+    cudaFuncSetAttribute(fps_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)q.dynamicSmemBytes);
+    cudaFuncSetAttribute(fps_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (cudaOccupancyMaxActiveClusters(&nclusters, fps_cluster_kernel<16>, &q) != cudaSuccess ||
+        nclusters < 1)
+      CL = 8;
+    cudaGetLastError();
+  }
+  const long per = (n + CL - 1) / CL;
+  const long ppt = (per + kFpsThreads - 1) / kFpsThreads;
+  cudaError_t e;
+  if (ppt <= 1) e = launch_reg<1>(pts, n, P, seed, centers, owner, CL, st);
+  else if (ppt <= 2) e = launch_reg<2>(pts, n, P, seed, centers, owner, CL, st);
+  else if (ppt <= 4) e = launch_reg<4>(pts, n, P, seed, centers, owner, CL, st);
+  else if (ppt <= 8) e = launch_reg<8>(pts, n, P, seed, centers, owner, CL, st);
+  else if (ppt <= 16) e = launch_reg<16>(pts, n, P, seed, centers, owner, CL, st);
+  else {
+    if (CL > 8)
+      cudaFuncSetAttribute(fps_cluster_mem_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                           1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL);
+    cfg.blockDim = dim3(kFpsThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launch();
+    e = cudaLaunchKernelEx(&cfg, fps_cluster_mem_kernel, pts, n, P, seed, centers, owner, best,
+                           chosen);
+  }
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(counts, 0, sizeof(int) * P, st)) != cudaSuccess) return e;
+  const int nb = (int)std::min<long>(1184, (n + 255) / 256);
+  count_kernel<<<nb, 256, 0, st>>>(owner, n, counts);
+  count_launch();
+  scan_offsets_kernel<<<1, 1024, 0, st>>>(counts, P, offsets, cursor);
+  count_launch();
+  fill_kernel<<<nb, 256, 0, st>>>(owner, n, cursor, members);
+  count_launch();
+  sort_segments_kernel<<<P, 512, 0, st>>>(owner, n, offsets, members);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ssc

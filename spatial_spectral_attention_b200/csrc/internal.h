@@ -1,0 +1,166 @@
+// internal.h -- launch interfaces between the C ABI (ssc_api.cu) and the
+// kernel files.  Host-side only types; no torch, no allocation.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace ssc {
+
+// Number of kernels this library has launched (all devices, all streams).
+inline std::atomic<unsigned long long> g_launches{0};
+inline void count_launch(unsigned n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// One unit of coupling work: query rows [row0, row0+nrows) (nrows <= 128) of
+// the (possibly patch-major) Q buffer attend to the key segments
+// segs[seg0 .. seg0+nseg).
+struct RowTile {
+  int row0, nrows, seg0, nseg;
+};
+// A run of consecutive key rows [key0, key0+nkeys), nkeys <= 128.
+struct KeySeg {
+  int key0, nkeys;
+};
+
+constexpr int kTileRows = 128;
+
+// Round x up to a multiple of a.
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Sequential carve-out of a caller workspace (256-byte aligned pieces).
+struct Carve {
+  char* base;
+  size_t used = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    used = round_up(used, 256);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+// ------------------------------------------------------------ fps.cu
+size_t fps_workspace_bytes(int n, int P);
+cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* centers, int* owner,
+                               int* offsets, int* members, void* ws, cudaStream_t st,
+                               const WaitCtl& ctl);
+
+// ------------------------------------------------------------ patch_topk.cu
+size_t scores_topk_workspace_bytes(int PN, int PM, int d);
+cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int ldm, int nM,
+                               int d, int dtype, const int* offN, const int* memN, int PN,
+                               const int* offM, const int* memM, int PM, int R, int* topk,
+                               double* scores, void* ws, unsigned* status, cudaStream_t st);
+
+// ------------------------------------------------------------ prep.cu
+// out[r, 0..cols) = in[map ? map[r] : r, 0..cols) converted to bf16 (in is
+// bf16 or fp32 per in_f32), zero-filled up to out_ld.
+// A map entry outside [0, src_rows) yields a zero row and sets the
+// bad-index bit of the status word.
+cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const int* map, int rows,
+                                    int src_rows, int cols, __nv_bfloat16* out, int out_ld,
+                                    unsigned* status, cudaStream_t st);
+// fp32 variant (check mode).
+cudaError_t launch_gather_rows_f32(const float* in, int in_ld, const int* map, int rows,
+                                   int src_rows, int cols, float* out, int out_ld, unsigned* status,
+                                   cudaStream_t st);
+// Backward preparation of row r (source row src = map ? map[r] : r):
+//   dOb[r, 0..k) = bf16(dO[src]) (zero-padded to ldb) when dOb != nullptr,
+//   dOf[r, 0..k) = dO[src] when dOf != nullptr,
+//   D[r] = <dO'[src], O[src]> with dO' the bf16-rounded value on the bf16 path,
+//   lse_out[r] = lse[src].
+cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, const float* lse,
+                            const int* map, int rows, int src_rows, int k, __nv_bfloat16* dOb,
+                            int ldb, float* dOf, int ldf, float* D, float* lse_out,
+                            unsigned* status, cudaStream_t st);
+// Dense schedule: ceil(nN/128) row tiles, all pointing at ceil(nM/128) segments.
+int dense_num_tiles(int nN);
+int dense_num_segs(int nM);
+cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, cudaStream_t st);
+// Geo schedule: per target patch ceil(|p|/128) row tiles that share the list of
+// 128-row pieces of the patch's selected source patches.  Writes the counts to
+// counts[0] (tiles) and counts[1] (segments).  Upper bounds for sizing:
+int geo_max_tiles(int nN, int PN);
+int geo_max_segs(int nM, int PM, int PN, int R);
+// topk entries outside [0, PM) are skipped and set the bad-index bit.
+// Offsets outside [0, n] or decreasing are clamped and set the bad-index bit.
+cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
+                                const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
+                                int* scratch, unsigned* status, cudaStream_t st);
+size_t geo_schedule_scratch_ints(int PN);
+// Transposed selection (for the key-stationary fp32 backward): for every
+// source patch q the ascending list of target patches p with q in topk[p].
+size_t invert_topk_scratch_ints(int PM);
+cudaError_t launch_invert_topk(const int* topk, int PN, int R, int PM, int* inv_off, int* inv_p,
+                               int* scratch, cudaStream_t st);
+
+// ------------------------------------------------------------ coupling_simt.cu (fp32)
+struct SimtArgs {
+  const float* Q;
+  const float* K;
+  const float* V;
+  int ldq, ldk, ldv;
+  int nN, nM, d, k;
+  float scale;
+  const RowTile* tiles;
+  const KeySeg* segs;
+  const int* ntiles_dev;  // nullable: number of tiles read on the device
+  int ntiles_host;        // used when ntiles_dev == nullptr
+  const int* row_map;     // output row r -> vertex (nullable = identity)
+  const int* col_map;     // key row j -> vertex (nullable = identity)
+};
+cudaError_t launch_simt_fwd(const SimtArgs& a, float* O, int ldo, float* lse, cudaStream_t st);
+// dQ: query-stationary.  Needs D and lse in the (permuted) row order.
+cudaError_t launch_simt_bwd_dq(const SimtArgs& a, const float* dO, int lddo, const float* lse,
+                               const float* D, float* dQ, int lddq, cudaStream_t st);
+// dK/dV: key-stationary.  Dense when inv_off == nullptr (every row attends);
+// otherwise key row j of source patch q is seen by the rows of the target
+// patches inv_p[inv_off[q] .. inv_off[q+1]).
+struct SimtKeyArgs {
+  const int* offM;     // source patch offsets (patch-major key rows), nullable for dense
+  int PM;
+  const int* offN;     // target patch offsets (patch-major query rows)
+  const int* inv_off;
+  const int* inv_p;
+  unsigned* status;    // bad-index reports
+};
+cudaError_t launch_simt_bwd_dkdv(const SimtArgs& a, const SimtKeyArgs& g, const float* dO,
+                                 int lddo, const float* lse, const float* D, float* dK, int lddk,
+                                 float* dV, int lddv, cudaStream_t st);
+
+// ------------------------------------------------------------ coupling_tc.cu (bf16, tcgen05)
+struct TcArgs {
+  const __nv_bfloat16* Q;  // [nQrows, ldq]
+  const __nv_bfloat16* K;  // [nKrows, ldk]
+  const __nv_bfloat16* V;  // [nKrows, ldv]
+  int ldq, ldk, ldv;
+  int nQrows, nKrows;
+  int d, k;
+  float scale;
+  const RowTile* tiles;
+  const KeySeg* segs;
+  const int* ntiles_dev;  // nullable
+  int ntiles_host;
+  const int* row_map;
+  const int* col_map;
+};
+bool tc_supported(int d, int k);
+cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
+                          const WaitCtl& ctl);
+// dQ written (scaled), dK accumulated with atomics (caller zeroes it).
+// dOb: bf16 [nQrows, lddob] (k padded with zeros), lse/D in row order.
+cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,
+                          const float* D, float* dQ, int lddq, float* dK, int lddk, float* dV,
+                          int lddv, cudaStream_t st, const WaitCtl& ctl);
+
+// Test hook: a kernel that waits on a barrier nothing arrives on.
+cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl);
+
+}  // namespace ssc

@@ -1,0 +1,382 @@
+// prep.cu -- data movement around the coupling kernels: row gathers into the
+// patch-major order Geo-FlashAttention works in, the backward preparation
+// (bf16 upstream gradient and D_i = <dO_i, O_i>), and the tile schedules.
+//
+// Patch-major order (project page, "Geo-FlashAttention": each target patch
+// attends to its selected source patches): after the gather, the rows of patch
+// p are the contiguous range offsets[p] .. offsets[p+1] of the gathered
+// buffer, so every selected source patch is a run of consecutive key rows that
+// one TMA box can fetch.  All kernels here are HBM-bound copies: 16-byte
+// vector accesses, one warp per row.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace ssc {
+namespace {
+
+// Patch p of a table with n rows, clamped into [0, n] and non-decreasing;
+// an inconsistent table sets the bad-index bit (and yields empty patches).
+__device__ __forceinline__ int2 patch_range(const int* off, int p, int n, unsigned* status) {
+  int b = off[p], e = off[p + 1];
+  if (b < 0 || e < b || e > n) {
+    atomicOr(status, kStatusBadIndex);
+    b = min(max(b, 0), n);
+    e = min(max(e, b), n);
+  }
+  return make_int2(b, e);
+}
+
+__device__ __forceinline__ int checked_src(const int* map, int r, int src_rows, unsigned* status) {
+  const int src = map ? map[r] : r;
+  if (src < 0 || src >= src_rows) {
+    atomicOr(status, kStatusBadIndex);
+    return -1;
+  }
+  return src;
+}
+
+__global__ void gather_bf16_from_bf16(const __nv_bfloat16* __restrict__ in, int in_ld,
+                                      const int* __restrict__ map, int rows, int src_rows, int cols,
+                                      __nv_bfloat16* __restrict__ out, int out_ld, int vec_ok,
+                                      unsigned* status) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int src = checked_src(map, r, src_rows, status);
+    __nv_bfloat16* o = out + (size_t)r * out_ld;
+    if (src < 0) {
+      for (int c = lane; c < out_ld; c += 32) o[c] = __float2bfloat16(0.f);
+      continue;
+    }
+    const __nv_bfloat16* a = in + (size_t)src * in_ld;
+    if (vec_ok) {
+      const int nvec = cols >> 3;  // full 8-element chunks
+      for (int v = lane; v < nvec; v += 32)
+        reinterpret_cast<uint4*>(o)[v] = __ldg(reinterpret_cast<const uint4*>(a) + v);
+      for (int c = (nvec << 3) + lane; c < out_ld; c += 32)
+        o[c] = c < cols ? a[c] : __float2bfloat16(0.f);
+    } else {
+      for (int c = lane; c < out_ld; c += 32) o[c] = c < cols ? a[c] : __float2bfloat16(0.f);
+    }
+  }
+}
+
+__global__ void gather_bf16_from_f32(const float* __restrict__ in, int in_ld,
+                                     const int* __restrict__ map, int rows, int src_rows, int cols,
+                                     __nv_bfloat16* __restrict__ out, int out_ld, unsigned* status) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int src = checked_src(map, r, src_rows, status);
+    const float* a = in + (size_t)(src < 0 ? 0 : src) * in_ld;
+    __nv_bfloat16* o = out + (size_t)r * out_ld;
+    for (int c = lane; c < out_ld; c += 32)
+      o[c] = __float2bfloat16((c < cols && src >= 0) ? a[c] : 0.f);
+  }
+}
+
+__global__ void gather_f32_kernel(const float* __restrict__ in, int in_ld,
+                                  const int* __restrict__ map, int rows, int src_rows, int cols,
+                                  float* __restrict__ out, int out_ld, unsigned* status) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int src = checked_src(map, r, src_rows, status);
+    const float* a = in + (size_t)(src < 0 ? 0 : src) * in_ld;
+    float* o = out + (size_t)r * out_ld;
+    for (int c = lane; c < out_ld; c += 32) o[c] = (c < cols && src >= 0) ? a[c] : 0.f;
+  }
+}
+
+__global__ void bwd_prep_kernel(const float* __restrict__ dO, int lddo, const float* __restrict__ O,
+                                int ldo, const float* __restrict__ lse, const int* __restrict__ map,
+                                int rows, int src_rows, int k, __nv_bfloat16* __restrict__ dOb,
+                                int ldb, float* __restrict__ dOf, int ldf, float* __restrict__ D,
+                                float* __restrict__ lse_out, unsigned* status) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int src0 = checked_src(map, r, src_rows, status);
+    const int src = src0 < 0 ? 0 : src0;
+    const float* g = dO + (size_t)src * lddo;
+    const float* o = O + (size_t)src * ldo;
+    float acc = 0.f;
+    for (int c = lane; c < k; c += 32) {
+      float v = src0 < 0 ? 0.f : g[c];
+      if (dOb) {
+        __nv_bfloat16 b = __float2bfloat16(v);
+        dOb[(size_t)r * ldb + c] = b;
+        v = __bfloat162float(b);
+      }
+      if (dOf) dOf[(size_t)r * ldf + c] = v;
+      acc = fmaf(v, o[c], acc);
+    }
+    if (dOb)
+      for (int c = k + lane; c < ldb; c += 32) dOb[(size_t)r * ldb + c] = __float2bfloat16(0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      D[r] = acc;
+      if (lse_out) lse_out[r] = src0 < 0 ? 0.f : lse[src];
+    }
+  }
+}
+
+__global__ void dense_schedule_kernel(int nN, int nM, RowTile* __restrict__ tiles,
+                                      KeySeg* __restrict__ segs) {
+  const int nt = (nN + kTileRows - 1) / kTileRows, ns = (nM + kTileRows - 1) / kTileRows;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < max(nt, ns); i += gridDim.x * blockDim.x) {
+    if (i < nt) tiles[i] = RowTile{i * kTileRows, min(kTileRows, nN - i * kTileRows), 0, ns};
+    if (i < ns) segs[i] = KeySeg{i * kTileRows, min(kTileRows, nM - i * kTileRows)};
+  }
+}
+
+// pieces[p] = row tiles of target patch p; nsegs[p] = 128-row pieces of its
+// selected source patches.
+__global__ void geo_count_kernel(const int* __restrict__ offN, int PN, int nN,
+                                 const int* __restrict__ offM, int PM, int nM,
+                                 const int* __restrict__ topk, int R, int* __restrict__ pieces,
+                                 int* __restrict__ nsegs, unsigned* status) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < PN; p += gridDim.x * blockDim.x) {
+    const int2 pr = patch_range(offN, p, nN, status);
+    const int rows = pr.y - pr.x;
+    pieces[p] = (rows + kTileRows - 1) / kTileRows;
+    int s = 0;
+    for (int r = 0; r < R; ++r) {
+      const int q = topk[(size_t)p * R + r];
+      if (q < 0 || q >= PM) {
+        atomicOr(status, kStatusBadIndex);
+        continue;
+      }
+      const int2 qr = patch_range(offM, q, nM, status);
+      s += (qr.y - qr.x + kTileRows - 1) / kTileRows;
+    }
+    nsegs[p] = s;
+  }
+}
+
+// Single-block exclusive scan of two int arrays of length m; totals[0..1].
+__global__ void __launch_bounds__(1024) scan2_kernel(const int* __restrict__ a, const int* __restrict__ b,
+                                                     int m, int* __restrict__ abase,
+                                                     int* __restrict__ bbase,
+                                                     int* __restrict__ totals) {
+  __shared__ int pa[1024], pb[1024];
+  const int tid = threadIdx.x;
+  const int per = (m + 1023) / 1024;
+  const int lo = tid * per, hi = min(m, lo + per);
+  int sa = 0, sb = 0;
+  for (int i = lo; i < hi; ++i) {
+    sa += a[i];
+    sb += b ? b[i] : 0;
+  }
+  pa[tid] = sa;
+  pb[tid] = sb;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    int xa = tid >= o ? pa[tid - o] : 0, xb = tid >= o ? pb[tid - o] : 0;
+    __syncthreads();
+    pa[tid] += xa;
+    pb[tid] += xb;
+    __syncthreads();
+  }
+  int ra = pa[tid] - sa, rb = pb[tid] - sb;
+  for (int i = lo; i < hi; ++i) {
+    abase[i] = ra;
+    ra += a[i];
+    if (b) {
+      bbase[i] = rb;
+      rb += b[i];
+    }
+  }
+  if (tid == 1023) {
+    totals[0] = pa[1023];
+    totals[1] = pb[1023];
+  }
+}
+
+// Writes beyond the capacities (possible only for inconsistent tables, e.g.
+// repeated entries in a topk row) are dropped and set the bad-index bit.
+__global__ void geo_fill_kernel(const int* __restrict__ offN, int PN, int nN,
+                                const int* __restrict__ offM, int PM, int nM,
+                                const int* __restrict__ topk, int R, unsigned* status,
+                                const int* __restrict__ tbase, const int* __restrict__ sbase,
+                                const int* __restrict__ nsegs, RowTile* __restrict__ tiles,
+                                KeySeg* __restrict__ segs, int tile_cap, int seg_cap) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < PN; p += gridDim.x * blockDim.x) {
+    const int2 pr = patch_range(offN, p, nN, status);
+    const int r0 = pr.x, rows = pr.y - pr.x;
+    const int sb = sbase[p];
+    const int ns = max(0, min(nsegs[p], seg_cap - sb));
+    if (ns < nsegs[p]) atomicOr(status, kStatusBadIndex);
+    for (int t = 0, i = 0; t < rows; t += kTileRows, ++i) {
+      if (tbase[p] + i >= tile_cap) {
+        atomicOr(status, kStatusBadIndex);
+        break;
+      }
+      tiles[tbase[p] + i] = RowTile{r0 + t, min(kTileRows, rows - t), sb, ns};
+    }
+    int s = sb;
+    for (int r = 0; r < R; ++r) {
+      const int q = topk[(size_t)p * R + r];
+      if (q < 0 || q >= PM) continue;
+      const int2 qr = patch_range(offM, q, nM, status);
+      const int k0 = qr.x, kn = qr.y - qr.x;
+      for (int u = 0; u < kn && s < sb + ns; u += kTileRows)
+        segs[s++] = KeySeg{k0 + u, min(kTileRows, kn - u)};
+    }
+  }
+}
+
+__global__ void clamp_counts_kernel(int* counts, int tile_cap, int seg_cap) {
+  counts[0] = min(counts[0], tile_cap);
+  counts[1] = min(counts[1], seg_cap);
+}
+
+__global__ void inv_count_kernel(const int* __restrict__ topk, int n, int PM, int* __restrict__ cnt) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int q = topk[i];
+    if (q >= 0 && q < PM) atomicAdd(cnt + q, 1);
+  }
+}
+__global__ void inv_fill_kernel(const int* __restrict__ topk, int PN, int R, int PM,
+                                int* __restrict__ cursor, int* __restrict__ inv_p) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < PN * R; i += gridDim.x * blockDim.x) {
+    const int q = topk[i];
+    if (q >= 0 && q < PM) inv_p[atomicAdd(cursor + q, 1)] = i / R;
+  }
+}
+__global__ void inv_sort_kernel(const int* __restrict__ inv_off, int PM, int* __restrict__ inv_p) {
+  for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < PM; q += gridDim.x * blockDim.x) {
+    const int b = inv_off[q], e = inv_off[q + 1];
+    for (int i = b + 1; i < e; ++i) {
+      int x = inv_p[i], j = i - 1;
+      while (j >= b && inv_p[j] > x) {
+        inv_p[j + 1] = inv_p[j];
+        --j;
+      }
+      inv_p[j + 1] = x;
+    }
+  }
+}
+__global__ void copy_offsets_kernel(const int* __restrict__ base, const int* __restrict__ totals,
+                                    int m, int* __restrict__ off, int* __restrict__ cursor) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= m; i += gridDim.x * blockDim.x) {
+    const int v = i < m ? base[i] : totals[0];
+    off[i] = v;
+    if (i < m) cursor[i] = v;
+  }
+}
+
+int grid_for(long work, int per_block) {
+  long b = (work + per_block - 1) / per_block;
+  return (int)std::max<long>(1, std::min<long>(b, 148L * 16));
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const int* map, int rows,
+                                    int src_rows, int cols, __nv_bfloat16* out, int out_ld,
+                                    unsigned* status, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int g = grid_for(rows, 8);
+  if (in_f32) {
+    gather_bf16_from_f32<<<g, 256, 0, st>>>(static_cast<const float*>(in), in_ld, map, rows,
+                                            src_rows, cols, out, out_ld, status);
+    count_launch();
+  } else {
+    const int vec_ok = (in_ld % 8 == 0) && (out_ld % 8 == 0) &&
+                       (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(out) % 16 == 0);
+    gather_bf16_from_bf16<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), in_ld, map,
+                                             rows, src_rows, cols, out, out_ld, vec_ok, status);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows_f32(const float* in, int in_ld, const int* map, int rows,
+                                   int src_rows, int cols, float* out, int out_ld, unsigned* status,
+                                   cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  gather_f32_kernel<<<grid_for(rows, 8), 256, 0, st>>>(in, in_ld, map, rows, src_rows, cols, out,
+                                                        out_ld, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, const float* lse,
+                            const int* map, int rows, int src_rows, int k, __nv_bfloat16* dOb,
+                            int ldb, float* dOf, int ldf, float* D, float* lse_out,
+                            unsigned* status, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  bwd_prep_kernel<<<grid_for(rows, 8), 256, 0, st>>>(dO, lddo, O, ldo, lse, map, rows, src_rows, k,
+                                                      dOb, ldb, dOf, ldf, D, lse_out, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int dense_num_tiles(int nN) { return (nN + kTileRows - 1) / kTileRows; }
+int dense_num_segs(int nM) { return (nM + kTileRows - 1) / kTileRows; }
+
+cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, cudaStream_t st) {
+  const int m = std::max(dense_num_tiles(nN), dense_num_segs(nM));
+  dense_schedule_kernel<<<grid_for(m, 256), 256, 0, st>>>(nN, nM, tiles, segs);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int geo_max_tiles(int nN, int PN) { return PN + (nN + kTileRows - 1) / kTileRows; }
+int geo_max_segs(int nM, int PM, int PN, int R) {
+  (void)PM;
+  const long a = (long)PN * R + (long)PN * ((nM + kTileRows - 1) / kTileRows);
+  return (int)std::min<long>(a, 0x7fffffffL);
+}
+size_t geo_schedule_scratch_ints(int PN) { return 4 * (size_t)PN + 2; }
+
+cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
+                                const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
+                                int* scratch, unsigned* status, cudaStream_t st) {
+  int* pieces = scratch;
+  int* nsegs = scratch + PN;
+  int* tbase = scratch + 2 * PN;
+  int* sbase = scratch + 3 * PN;
+  geo_count_kernel<<<grid_for(PN, 128), 128, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, pieces,
+                                                      nsegs, status);
+  count_launch();
+  scan2_kernel<<<1, 1024, 0, st>>>(pieces, nsegs, PN, tbase, sbase, counts);
+  count_launch();
+  const int tile_cap = geo_max_tiles(nN, PN), seg_cap = geo_max_segs(nM, PM, PN, R);
+  geo_fill_kernel<<<grid_for(PN, 64), 64, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, status,
+                                                    tbase, sbase, nsegs, tiles, segs, tile_cap,
+                                                    seg_cap);
+  count_launch();
+  clamp_counts_kernel<<<1, 1, 0, st>>>(counts, tile_cap, seg_cap);
+  count_launch();
+  return cudaGetLastError();
+}
+
+size_t invert_topk_scratch_ints(int PM) { return 3 * (size_t)PM + 2; }
+
+cudaError_t launch_invert_topk(const int* topk, int PN, int R, int PM, int* inv_off, int* inv_p,
+                               int* scratch, cudaStream_t st) {
+  int* cnt = scratch;            // [PM]
+  int* base = scratch + PM;      // [PM]
+  int* cursor = scratch + 2 * PM;  // [PM]
+  int* totals = scratch + 3 * PM;  // [2]
+  cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int) * PM, st);
+  if (e != cudaSuccess) return e;
+  inv_count_kernel<<<grid_for((long)PN * R, 256), 256, 0, st>>>(topk, PN * R, PM, cnt);
+  count_launch();
+  scan2_kernel<<<1, 1024, 0, st>>>(cnt, nullptr, PM, base, nullptr, totals);
+  count_launch();
+  copy_offsets_kernel<<<grid_for(PM + 1, 256), 256, 0, st>>>(base, totals, PM, inv_off, cursor);
+  count_launch();
+  inv_fill_kernel<<<grid_for((long)PN * R, 256), 256, 0, st>>>(topk, PN, R, PM, cursor, inv_p);
+  count_launch();
+  inv_sort_kernel<<<grid_for(PM, 128), 128, 0, st>>>(inv_off, PM, inv_p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace ssc

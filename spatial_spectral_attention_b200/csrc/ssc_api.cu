@@ -1,0 +1,461 @@
+// ssc_api.cu -- the C ABI of libssc (declared in include/ssc.h): argument
+// checks, workspace carving and the launch sequence of every call.  No call
+// allocates device memory and none synchronises the host (except
+// ssc_device_status, whose job is to read the status word back).
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/ssc.h"
+#include "internal.h"
+
+using namespace ssc;
+
+namespace {
+
+__device__ unsigned g_status_word;  // bit 0: a wait ran out; bit 1: bad index
+
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+unsigned* status_ptr() {
+  static unsigned* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned*>(p);
+  }
+  return ptrs[dev];
+}
+
+WaitCtl make_ctl() {
+  WaitCtl c;
+  c.status = status_ptr();
+  c.limit_ns = g_wait_limit_ns;
+  return c;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SSC_OK : SSC_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN,
+                 int nM, int d, int k, float scale, int dtype) {
+  if (!Q || !K || !V) return SSC_ERR_INVALID_ARG;
+  if (nN < 1 || nM < 1 || k < 1) return SSC_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SSC_ERR_INVALID_ARG;
+  if (dtype != SSC_BF16 && dtype != SSC_F32) return SSC_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SSC_ERR_UNSUPPORTED;
+  if (k > 256) return SSC_ERR_UNSUPPORTED;
+  if (ldq < d || ldk < d || ldv < k) return SSC_ERR_INVALID_ARG;
+  if (dtype == SSC_BF16) {
+    // Q and K are read by TMA in place; V of any stride is re-packed when needed
+    if (!aligned16(Q) || !aligned16(K)) return SSC_ERR_ALIGNMENT;
+    if (ldq % 8 || ldk % 8) return SSC_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(V) & 1u) return SSC_ERR_ALIGNMENT;
+  } else {
+    const uintptr_t m = reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
+                        reinterpret_cast<uintptr_t>(V);
+    if (m & 3u) return SSC_ERR_ALIGNMENT;
+  }
+  return SSC_OK;
+}
+
+int check_out(const float* p, int ld, int cols) {
+  if (!p) return SSC_ERR_INVALID_ARG;
+  if (ld < cols) return SSC_ERR_INVALID_ARG;
+  if (!aligned16(p)) return SSC_ERR_ALIGNMENT;
+  return SSC_OK;
+}
+
+int check_patches(const int* offN, const int* memN, int PN, int nN, const int* offM,
+                  const int* memM, int PM, int nM, const int* topk, int R) {
+  if (!offN || !memN || !offM || !memM || !topk) return SSC_ERR_INVALID_ARG;
+  if (PN < 1 || PM < 1 || PN > nN || PM > nM || PN > 65535 || PM > 65535) return SSC_ERR_INVALID_ARG;
+  if (R < 1 || R > PM) return SSC_ERR_INVALID_ARG;
+  return SSC_OK;
+}
+
+size_t kp_of(int k) {
+  size_t kp = (k + 15) / 16 * 16;
+  if (kp % 64 == 48) kp += 16;
+  return kp;
+}
+
+cudaError_t zero_matrix(float* p, int ld, int rows, int cols, cudaStream_t st) {
+  if (ld == cols) return cudaMemsetAsync(p, 0, sizeof(float) * (size_t)rows * cols, st);
+  return cudaMemset2DAsync(p, sizeof(float) * (size_t)ld, 0, sizeof(float) * (size_t)cols, rows, st);
+}
+
+// ---- workspace layouts (sizes only when base == nullptr)
+struct DenseWs {
+  RowTile* tiles;
+  KeySeg* segs;
+  __nv_bfloat16* dOb;
+  __nv_bfloat16* Vpad;  // V re-packed with a 16-byte aligned row pitch
+  float* D;
+};
+size_t dense_ws(void* base, int nN, int nM, int d, int k, int dtype, DenseWs* w) {
+  (void)d;
+  Carve c(base);
+  DenseWs x;
+  x.tiles = c.take<RowTile>(dense_num_tiles(nN));
+  x.segs = c.take<KeySeg>(dense_num_segs(nM));
+  x.dOb = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nN * kp_of(k)) : nullptr;
+  x.Vpad = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nM * kp_of(k)) : nullptr;
+  x.D = c.take<float>(nN);
+  if (w) *w = x;
+  return c.used + 256;
+}
+
+struct GeoWs {
+  void* Qp;
+  void* Kp;
+  void* Vp;
+  void* dOp;
+  float* D;
+  float* lsep;
+  RowTile* tiles;
+  KeySeg* segs;
+  int* counts;
+  int* sched_scratch;
+  int* inv_off;
+  int* inv_p;
+  int* inv_scratch;
+  int ldq, ldk, ldv, ldg;
+};
+size_t geo_ws(void* base, int nN, int nM, int d, int k, int PN, int PM, int R, int dtype, GeoWs* w) {
+  Carve c(base);
+  GeoWs x;
+  const bool bf = dtype == SSC_BF16;
+  const size_t es = bf ? 2 : 4;
+  x.ldq = d;
+  x.ldk = d;
+  x.ldv = bf ? (int)kp_of(k) : k;
+  x.ldg = bf ? (int)kp_of(k) : k;
+  x.Qp = c.take<uint8_t>((size_t)nN * x.ldq * es);
+  x.Kp = c.take<uint8_t>((size_t)nM * x.ldk * es);
+  x.Vp = c.take<uint8_t>((size_t)nM * x.ldv * es);
+  x.dOp = c.take<uint8_t>((size_t)nN * x.ldg * es);
+  x.D = c.take<float>(nN);
+  x.lsep = c.take<float>(nN);
+  x.tiles = c.take<RowTile>(geo_max_tiles(nN, PN));
+  x.segs = c.take<KeySeg>(geo_max_segs(nM, PM, PN, R));
+  x.counts = c.take<int>(2);
+  x.sched_scratch = c.take<int>(geo_schedule_scratch_ints(PN));
+  x.inv_off = c.take<int>(PM + 1);
+  x.inv_p = c.take<int>((size_t)PN * R);
+  x.inv_scratch = c.take<int>(invert_topk_scratch_ints(PM));
+  if (w) *w = x;
+  return c.used + 256;
+}
+
+bool ws_ok(void* ws, size_t have, size_t need) {
+  return ws && have >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0;
+}
+
+// The bf16 V operand as the tensor-core kernels read it: in place when its
+// rows are 16-byte aligned, else re-packed into the workspace.
+cudaError_t dense_v(const void* V, int ldv, int nM, int k, const DenseWs& w,
+                    const __nv_bfloat16** Vout, int* ldout, cudaStream_t st, unsigned* status) {
+  if (ldv % 8 == 0 && aligned16(V)) {
+    *Vout = static_cast<const __nv_bfloat16*>(V);
+    *ldout = ldv;
+    return cudaSuccess;
+  }
+  *Vout = w.Vpad;
+  *ldout = (int)kp_of(k);
+  return launch_gather_rows_bf16(V, ldv, 0, nullptr, nM, nM, k, w.Vpad, (int)kp_of(k), status, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssc_status_string(int status) {
+  switch (status) {
+    case SSC_OK: return "ok";
+    case SSC_ERR_INVALID_ARG: return "invalid argument (size, null pointer or index table)";
+    case SSC_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128, 1 <= k <= 256)";
+    case SSC_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case SSC_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SSC_ERR_CUDA: return "CUDA call failed";
+    case SSC_ERR_TIMEOUT: return "a device-side wait ran out of time";
+    default: return "unknown status";
+  }
+}
+
+int ssc_version(void) { return (0 << 16) | 1; }
+
+unsigned long long ssc_kernel_launches(void) { return g_launches.load(); }
+
+int ssc_device_status(ssc_stream_t stream, int clear, int* status) {
+  if (!status) return SSC_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSC_ERR_CUDA;
+  unsigned* p = status_ptr();
+  if (!p) return SSC_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, p, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return SSC_ERR_CUDA;
+  if (clear) {
+    unsigned zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return SSC_ERR_CUDA;
+  }
+  *status = (word & kStatusTimeout) ? SSC_ERR_TIMEOUT
+            : (word & kStatusBadIndex) ? SSC_ERR_INVALID_ARG
+                                        : SSC_OK;
+  return SSC_OK;
+}
+
+int ssc_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns = ns ? ns : 2000000000ull;
+  return SSC_OK;
+}
+
+int ssc_debug_wait_timeout(unsigned long long limit_ns, ssc_stream_t stream) {
+  WaitCtl c = make_ctl();
+  if (!c.status) return SSC_ERR_CUDA;
+  c.limit_ns = limit_ns ? limit_ns : 1000000ull;
+  return cuda_status(launch_wait_timeout_probe(static_cast<cudaStream_t>(stream), c));
+}
+
+// ------------------------------------------------------------ patches
+size_t ssc_fps_patches_workspace_size(int n, int P) {
+  if (n < 1 || P < 1) return 0;
+  return fps_workspace_bytes(n, P);
+}
+
+int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex, int* centers, int* owner,
+                    int* offsets, int* members, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  if (!pts || !centers || !owner || !offsets || !members) return SSC_ERR_INVALID_ARG;
+  if (n < 1 || P < 1 || P > n || P > 65535 || n > (1 << 24)) return SSC_ERR_INVALID_ARG;
+  if (seed_vertex < 0 || seed_vertex >= n) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, fps_workspace_bytes(n, P))) return SSC_ERR_WORKSPACE;
+  WaitCtl c = make_ctl();
+  return cuda_status(launch_fps_patches(pts, n, P, seed_vertex, centers, owner, offsets, members, ws,
+                                        static_cast<cudaStream_t>(stream), c));
+}
+
+size_t ssc_patch_scores_topk_workspace_size(int PN, int PM, int d) {
+  if (PN < 1 || PM < 1 || d < 1) return 0;
+  return scores_topk_workspace_bytes(PN, PM, d);
+}
+
+int ssc_patch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int ldm, int nM, int d,
+                          int dtype, const int* offN, const int* memN, int PN, const int* offM,
+                          const int* memM, int PM, int R, int* topk, double* scores, void* ws,
+                          size_t ws_bytes, ssc_stream_t stream) {
+  if (!FN || !FM || !offN || !memN || !offM || !memM || !topk) return SSC_ERR_INVALID_ARG;
+  if (d < 1 || d > 1024 || ldn < d || ldm < d || nN < 1 || nM < 1) return SSC_ERR_INVALID_ARG;
+  if (dtype != SSC_BF16 && dtype != SSC_F32) return SSC_ERR_INVALID_ARG;
+  if (PN < 1 || PM < 1 || PN > nN || PM > nM || PN > 65535 || PM > 65535) return SSC_ERR_INVALID_ARG;
+  if (R < 1 || R > PM) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, scores_topk_workspace_bytes(PN, PM, d))) return SSC_ERR_WORKSPACE;
+  WaitCtl c = make_ctl();
+  return cuda_status(launch_scores_topk(FN, ldn, nN, FM, ldm, nM, d, dtype, offN, memN, PN, offM,
+                                        memM, PM, R, topk, scores, ws, c.status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------ dense
+size_t ssc_dense_coupling_workspace_size(int nN, int nM, int d, int k, int dtype) {
+  if (nN < 1 || nM < 1 || k < 1) return 0;
+  return dense_ws(nullptr, nN, nM, d, k, dtype, nullptr);
+}
+
+int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                           int nN, int nM, int d, int k, float scale, int dtype, float* O, int ldo,
+                           float* lse, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, dense_ws(nullptr, nN, nM, d, k, dtype, nullptr))) return SSC_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DenseWs w;
+  dense_ws(ws, nN, nM, d, k, dtype, &w);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if (dtype == SSC_F32) {
+    SimtArgs a{static_cast<const float*>(Q), static_cast<const float*>(K),
+               static_cast<const float*>(V), ldq, ldk, ldv, nN, nM, d, k, scale, w.tiles, w.segs,
+               nullptr, dense_num_tiles(nN), nullptr, nullptr};
+    return cuda_status(launch_simt_fwd(a, O, ldo, lse, st));
+  }
+  WaitCtl ctl = make_ctl();
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
+           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), nullptr,
+           nullptr};
+  return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
+}
+
+int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                           int nN, int nM, int d, int k, float scale, int dtype, const float* O,
+                           int ldo, const float* lse, const float* dO, int lddo, float* dQ, int lddq,
+                           float* dK, int lddk, float* dV, int lddv, void* ws, size_t ws_bytes,
+                           ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, dense_ws(nullptr, nN, nM, d, k, dtype, nullptr))) return SSC_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  DenseWs w;
+  dense_ws(ws, nN, nM, d, k, dtype, &w);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if (dtype == SSC_F32) {
+    e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, nullptr, 0, nullptr, 0, w.D,
+                        nullptr, ctl.status, st);
+    if (e != cudaSuccess) return SSC_ERR_CUDA;
+    SimtArgs a{static_cast<const float*>(Q), static_cast<const float*>(K),
+               static_cast<const float*>(V), ldq, ldk, ldv, nN, nM, d, k, scale, w.tiles, w.segs,
+               nullptr, dense_num_tiles(nN), nullptr, nullptr};
+    if ((e = launch_simt_bwd_dq(a, dO, lddo, lse, w.D, dQ, lddq, st)) != cudaSuccess)
+      return SSC_ERR_CUDA;
+    SimtKeyArgs g{nullptr, 0, nullptr, nullptr, nullptr, ctl.status};
+    return cuda_status(launch_simt_bwd_dkdv(a, g, dO, lddo, lse, w.D, dK, lddk, dV, lddv, st));
+  }
+  const int kp = (int)kp_of(k);
+  e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
+                      nullptr, ctl.status, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
+           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), nullptr,
+           nullptr};
+  return cuda_status(launch_tc_bwd(a, w.dOb, kp, lse, w.D, dQ, lddq, dK, lddk, dV, lddv, st, ctl));
+}
+
+// ------------------------------------------------------------ geo
+size_t ssc_geo_coupling_workspace_size(int nN, int nM, int d, int k, int PN, int PM, int R,
+                                       int dtype) {
+  if (nN < 1 || nM < 1 || k < 1 || PN < 1 || PM < 1 || R < 1) return 0;
+  return geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr);
+}
+
+namespace {
+
+// Gathers Q, K, V into patch-major order and builds the tile schedule.
+int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN, int nM,
+              int d, int k, int dtype, const int* offN, const int* memN, int PN, const int* offM,
+              const int* memM, int PM, const int* topk, int R, const GeoWs& w, cudaStream_t st,
+              const WaitCtl& ctl) {
+  cudaError_t e;
+  if (dtype == SSC_BF16) {
+    if ((e = launch_gather_rows_bf16(Q, ldq, 0, memN, nN, nN, d, static_cast<__nv_bfloat16*>(w.Qp),
+                                     w.ldq, ctl.status, st)) != cudaSuccess ||
+        (e = launch_gather_rows_bf16(K, ldk, 0, memM, nM, nM, d, static_cast<__nv_bfloat16*>(w.Kp),
+                                     w.ldk, ctl.status, st)) != cudaSuccess ||
+        (e = launch_gather_rows_bf16(V, ldv, 0, memM, nM, nM, k, static_cast<__nv_bfloat16*>(w.Vp),
+                                     w.ldv, ctl.status, st)) != cudaSuccess)
+      return SSC_ERR_CUDA;
+  } else {
+    if ((e = launch_gather_rows_f32(static_cast<const float*>(Q), ldq, memN, nN, nN, d,
+                                    static_cast<float*>(w.Qp), w.ldq, ctl.status, st)) != cudaSuccess ||
+        (e = launch_gather_rows_f32(static_cast<const float*>(K), ldk, memM, nM, nM, d,
+                                    static_cast<float*>(w.Kp), w.ldk, ctl.status, st)) != cudaSuccess ||
+        (e = launch_gather_rows_f32(static_cast<const float*>(V), ldv, memM, nM, nM, k,
+                                    static_cast<float*>(w.Vp), w.ldv, ctl.status, st)) != cudaSuccess)
+      return SSC_ERR_CUDA;
+  }
+  e = launch_geo_schedule(offN, PN, nN, offM, PM, nM, topk, R, w.tiles, w.segs, w.counts,
+                          w.sched_scratch, ctl.status, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
+                         const int* memN, int PN, const int* offM, const int* memM, int PM,
+                         const int* topk, int R, float* O, int ldo, float* lse, void* ws,
+                         size_t ws_bytes, ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoWs w;
+  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
+  if ((rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
+                      topk, R, w, st, ctl)))
+    return rc;
+  if (dtype == SSC_F32) {
+    SimtArgs a{static_cast<const float*>(w.Qp), static_cast<const float*>(w.Kp),
+               static_cast<const float*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale, w.tiles,
+               w.segs, w.counts, 0, memN, memM};
+    return cuda_status(launch_simt_fwd(a, O, ldo, lse, st));
+  }
+  TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
+           static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
+           w.tiles, w.segs, w.counts, 0, memN, memM};
+  return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
+}
+
+int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
+                         const int* memN, int PN, const int* offM, const int* memM, int PM,
+                         const int* topk, int R, const float* O, int ldo, const float* lse,
+                         const float* dO, int lddo, float* dQ, int lddq, float* dK, int lddk,
+                         float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoWs w;
+  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
+  if ((rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
+                      topk, R, w, st, ctl)))
+    return rc;
+  cudaError_t e;
+  if (dtype == SSC_F32) {
+    e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, nullptr, 0,
+                        static_cast<float*>(w.dOp), w.ldg, w.D, w.lsep, ctl.status, st);
+    if (e != cudaSuccess) return SSC_ERR_CUDA;
+    if ((e = launch_invert_topk(topk, PN, R, PM, w.inv_off, w.inv_p, w.inv_scratch, st)) !=
+        cudaSuccess)
+      return SSC_ERR_CUDA;
+    SimtArgs a{static_cast<const float*>(w.Qp), static_cast<const float*>(w.Kp),
+               static_cast<const float*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale, w.tiles,
+               w.segs, w.counts, 0, memN, memM};
+    if ((e = launch_simt_bwd_dq(a, static_cast<const float*>(w.dOp), w.ldg, w.lsep, w.D, dQ, lddq,
+                                st)) != cudaSuccess)
+      return SSC_ERR_CUDA;
+    SimtKeyArgs g{offM, PM, offN, w.inv_off, w.inv_p, ctl.status};
+    return cuda_status(launch_simt_bwd_dkdv(a, g, static_cast<const float*>(w.dOp), w.ldg, w.lsep,
+                                            w.D, dK, lddk, dV, lddv, st));
+  }
+  e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, static_cast<__nv_bfloat16*>(w.dOp),
+                      w.ldg, nullptr, 0, w.D, w.lsep, ctl.status, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
+           static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
+           w.tiles, w.segs, w.counts, 0, memN, memM};
+  return cuda_status(launch_tc_bwd(a, static_cast<const __nv_bfloat16*>(w.dOp), w.ldg, w.lsep, w.D,
+                                   dQ, lddq, dK, lddk, dV, lddv, st, ctl));
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+"""GPU parity of the coupling O = softmax(s Q K^T) V and its gradients against
+the fp64 oracle, dense and Geo-FlashAttention, bf16 tensor-core path and fp32
+check mode ("Spatial-Spectral Coupling as Attention", project page, sections
+"Spatial-spectral coupling is attention" and "Geo-FlashAttention")."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from spatial_spectral_attention_b200 import api, synth
+
+from _util import TOL_BF16, TOL_F32, as_i32, assert_close, rounded
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(Qn, Kn, Vn, dOn, dtype):
+    Q, Q64 = rounded(Qn, dtype)
+    K, K64 = rounded(Kn, dtype)
+    V, V64 = rounded(Vn, dtype)
+    # the bf16 path rounds dO once and uses that value throughout
+    dO = torch.tensor(np.ascontiguousarray(dOn, np.float32)).cuda()
+    dO64 = (dO.to(torch.bfloat16) if dtype == "bf16" else dO).double().cpu().numpy()
+    return (Q, K, V, dO), (Q64, K64, V64, dO64)
+
+
+def _status_ok():
+    torch.cuda.synchronize()
+    assert api.ssc_device_status() == 0
+
+
+def _dense_case(Qn, Kn, Vn, dOn, scale, dtype, need_dV=True):
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(Qn, Kn, Vn, dOn, dtype)
+    O, lse = api.ssc_dense_coupling_fwd(Q, K, V, scale)
+    dQ, dK, dV = api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=need_dV)
+    _status_ok()
+    ref = oracle.dense_bwd(Q64, K64, V64, dO64, scale)
+    assert_close(O, ref["O"], tol, "O")
+    assert_close(lse, ref["lse"], tol, "lse")
+    assert_close(dQ, ref["dQ"], tol, "dQ")
+    assert_close(dK, ref["dK"], tol, "dK")
+    if need_dV:
+        assert_close(dV, ref["dV"], tol, "dV")
+
+
+def test_dense_fp32_check_mode_small_workload():
+    p = synth.make_workload("small_fp32_2k")
+    (Q, K, V, _), (Q64, K64, V64, _) = _inputs(p.F_N, p.F_M, p.Phi_M, p.dO, "f32")
+    O, lse = api.ssc_dense_coupling_fwd(Q, K, V, p.scale)
+    _status_ok()
+    O64, lse64 = oracle.dense_fwd(Q64, K64, V64, p.scale)
+    assert_close(O, O64, TOL_F32, "O")
+    assert_close(lse, lse64, TOL_F32, "lse")
+
+
+def test_dense_fp32_check_mode_backward():
+    p = synth.make_workload("small_fp32_2k", n=700)
+    _dense_case(p.F_N, p.F_M, p.Phi_M, p.dO, p.scale, "f32")
+
+
+def test_dense_bf16_workload_ragged():
+    p = synth.make_workload("dense_10k", n=3000)  # 23 full row tiles + 56 rows
+    _dense_case(p.F_N, p.F_M, p.Phi_M, p.dO, p.scale, "bf16")
+
+
+@pytest.mark.parametrize("nN,nM,d,k", [(1, 1, 128, 196), (129, 300, 64, 25), (513, 77, 128, 16),
+                                       (256, 1000, 128, 256), (200, 200, 64, 100),
+                                       (130, 260, 128, 32), (384, 129, 128, 196)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_dense_shapes(nN, nM, d, k, dtype):
+    Qn, Kn, Vn, dOn = synth.random_inputs(nN, nM, d, k, seed=nN * 7 + nM, q_scale=0.5)
+    _dense_case(Qn, Kn, Vn, dOn, 1.0 / math.sqrt(d), dtype)
+
+
+def test_dense_bf16_unaligned_v_is_repacked():
+    # k = 25 gives a 50-byte V row pitch, which the library re-packs itself
+    Qn, Kn, Vn, dOn = synth.random_inputs(300, 260, 64, 25, seed=3)
+    _dense_case(Qn, Kn, Vn, dOn, 0.125, "bf16")
+
+
+def test_dense_bf16_peaked_softmax_rescaling():
+    # a large scale makes the running max jump often: exercises the O rescale
+    Qn, Kn, Vn, dOn = synth.random_inputs(256, 1024, 128, 64, seed=9)
+    _dense_case(Qn, Kn, Vn, dOn, 0.6, "bf16")
+
+
+def test_dense_bf16_full_size_sampled():
+    p = synth.make_workload("dense_60k")
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(p.F_N, p.F_M, p.Phi_M, p.dO, "bf16")
+    O, lse = api.ssc_dense_coupling_fwd(Q, K, V, p.scale)
+    dQ, dK, dV = api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, p.scale, need_dV=True)
+    _status_ok()
+    rows = np.random.default_rng(0).choice(p.n, 384, replace=False)
+    O64, lse64 = oracle.dense_fwd(Q64, K64, V64, p.scale, rows=rows)
+    assert_close(O.cpu().numpy()[rows], O64, TOL_BF16, "O rows")
+    assert_close(lse.cpu().numpy()[rows], lse64, TOL_BF16, "lse rows")
+    # dQ of a row needs only that row's O, lse and D (row-local)
+    D = (dO64[rows] * O64).sum(1)
+    S = p.scale * (Q64[rows] @ K64.T)
+    Pi = np.exp(S - lse64[:, None])
+    dQ64 = p.scale * ((Pi * (dO64[rows] @ V64.T - D[:, None])) @ K64)
+    assert_close(dQ.cpu().numpy()[rows], dQ64, TOL_BF16, "dQ rows")
+    # properties that hold at any size: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i,
+    # sum_i <Q_i, dQ_i> = sum_j <K_j, dK_j>
+    dKn, dVn, dQn = (t.double().cpu().numpy() for t in (dK, dV, dQ))
+    assert np.abs(dKn.sum(0)).max() <= 1e-2 * np.abs(dKn).sum(0).max()
+    np.testing.assert_allclose(dVn.sum(0), dO64.sum(0), atol=0.5, rtol=2e-3)
+    a, b = (Q64 * dQn).sum(), (K64 * dKn).sum()
+    assert abs(a - b) <= 1e-2 * max(abs(a), abs(b), 1.0)
+
+
+def _geo_tables(pair, P, R, dtype):
+    FN64 = rounded(pair.F_N, dtype)[1]
+    FM64 = rounded(pair.F_M, dtype)[1]
+    return oracle.patch_pipeline(pair.pts_N, pair.pts_M, FN64, FM64, P, P, R)
+
+
+def _geo_case(pair, P, R, dtype, need_dV=True):
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    t = _geo_tables(pair, P, R, dtype)
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, dtype)
+    tabs = [as_i32(t[x]) for x in ("off_N", "mem_N", "off_M", "mem_M", "topk")]
+    O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, *tabs)
+    dQ, dK, dV = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, need_dV=need_dV)
+    _status_ok()
+    ref = oracle.geo_bwd(Q64, K64, V64, dO64, pair.scale, t["off_N"], t["mem_N"], t["off_M"],
+                         t["mem_M"], t["topk"])
+    assert_close(O, ref["O"], tol, "O")
+    assert_close(lse, ref["lse"], tol, "lse")
+    assert_close(dQ, ref["dQ"], tol, "dQ")
+    assert_close(dK, ref["dK"], tol, "dK")
+    if need_dV:
+        assert_close(dV, ref["dV"], tol, "dV")
+    return O, lse, dQ, dK, dV
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("n,P,R", [(6000, 48, 8), (2000, 5, 2), (1500, 12, 3), (300, 300, 4)])
+def test_geo_matches_oracle(dtype, n, P, R):
+    pair = synth.make_workload("geo_60k", n=n)
+    _geo_case(pair, P, R, dtype)
+
+
+def test_geo_all_patches_selected_equals_dense():
+    pair = synth.make_workload("geo_60k", n=1200)
+    P = 10
+    O, lse, dQ, dK, dV = _geo_case(pair, P, P, "bf16")
+    (Q, K, V, dO), _ = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, "bf16")
+    Od, lsed = api.ssc_dense_coupling_fwd(Q, K, V, pair.scale)
+    dQd, dKd, dVd = api.ssc_dense_coupling_bwd(Q, K, V, Od, lsed, dO, pair.scale, need_dV=True)
+    for a, b, nm in ((O, Od, "O"), (lse, lsed, "lse"), (dQ, dQd, "dQ"), (dK, dKd, "dK"),
+                     (dV, dVd, "dV")):
+        assert_close(a, b.double().cpu().numpy(), TOL_BF16, nm)
+
+
+@pytest.mark.parametrize("name", ["geo_60k", "geo_160k_warped"])
+def test_geo_bf16_full_size(name):
+    pair = synth.make_workload(name)
+    _geo_case(pair, pair.P, pair.R, "bf16", need_dV=False)
+
+
+def test_geo_end_to_end_from_gpu_tables():
+    pair = synth.make_workload("geo_60k", n=8000)
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, "bf16")
+    _, _, offN, memN = api.ssc_fps_patches(torch.tensor(pair.pts_N).cuda(), 64)
+    _, _, offM, memM = api.ssc_fps_patches(torch.tensor(pair.pts_M).cuda(), 64)
+    topk = api.ssc_patch_scores_topk(Q, K, offN, memN, offM, memM, 8)
+    O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, offN, memN, offM, memM, topk)
+    _status_ok()
+    t = oracle.patch_pipeline(pair.pts_N, pair.pts_M, Q64, K64, 64, 64, 8)
+    np.testing.assert_array_equal(topk.cpu().numpy(), t["topk"])
+    O64, lse64 = oracle.geo_fwd(Q64, K64, V64, pair.scale, t["off_N"], t["mem_N"], t["off_M"],
+                                t["mem_M"], t["topk"])
+    assert_close(O, O64, TOL_BF16, "O")
+    assert_close(lse, lse64, TOL_BF16, "lse")
+
+
+def test_constant_eigenfunction_reproduced():
+    # rows of Pi sum to one, so the constant column Y_00 of Phi comes back exactly
+    # up to the bf16 rounding of P (relative 2^-8 at worst per element)
+    p = synth.make_workload("dense_10k", n=2000)
+    (Q, K, V, _), _ = _inputs(p.F_N, p.F_M, p.Phi_M, p.dO, "bf16")
+    O, _ = api.ssc_dense_coupling_fwd(Q, K, V, p.scale)
+    y00 = float(V[0, 0].float())
+    assert np.abs(O[:, 0].cpu().numpy() - y00).max() < 4e-3 * y00
+
+
+def test_wait_timeout_reports_status_without_fault():
+    api.ssc_device_status(clear=True)
+    api.ssc_debug_wait_timeout(2_000_000)  # 2 ms, nothing ever arrives
+    assert api.ssc_device_status(clear=True) == 6
+    # the context is still usable
+    Qn, Kn, Vn, dOn = synth.random_inputs(130, 140, 64, 16, seed=1)
+    _dense_case(Qn, Kn, Vn, dOn, 0.125, "bf16", need_dV=False)
