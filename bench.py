@@ -144,8 +144,8 @@ def run_ours(args, ws, rank, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pair = synth.make_workload(args.workload)
-    gpair = synth.make_workload("geo_60k") if args.with_geo else None
+    pair = synth.make_workload(args.workload, n=args.n)
+    gpair = synth.make_workload("geo_60k", n=args.n) if args.with_geo else None
     bf = lambda a: torch.tensor(a).to(torch.bfloat16)
     host = dict(Q=bf(pair.F_N).pin_memory(), K=bf(pair.F_M).pin_memory(),
                 V=bf(pair.Phi_M).pin_memory(), dO=torch.tensor(pair.dO).pin_memory())
@@ -235,11 +235,13 @@ def run_ours(args, ws, rank, local):
     barrier(ws)
 
     # ---- end to end through the public API with host buffers
+    if not args.e2e:
+        e2e_steps = 0
     out_host = dict(O=torch.empty((n, k), dtype=torch.float32).pin_memory(),
                     lse=torch.empty(n, dtype=torch.float32).pin_memory(),
                     dQ=torch.empty((n, d), dtype=torch.float32).pin_memory(),
                     dK=torch.empty((n, d), dtype=torch.float32).pin_memory())
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = max(2, min(args.steps, 5)) if args.e2e else 0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(ws)
@@ -253,7 +255,7 @@ def run_ours(args, ws, rank, local):
         out_host["dK"].copy_(dK, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(e2e_steps, 1), ws)
     h2d = sum(host[x].numel() * host[x].element_size() for x in ("Q", "K", "V", "dO"))
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
 
@@ -344,7 +346,7 @@ def cpu_cores():
 
 def run_reference(args, ws, rank):
     from spatial_spectral_attention_b200 import synth
-    pair = synth.make_workload(args.workload)
+    pair = synth.make_workload(args.workload, n=args.n)
     vals, times = [], []
     for s in range(args.warmup + args.steps):
         tf, ms, rows, dt = oracle_sample(pair, args.ref_budget, args.need_dv)
@@ -375,6 +377,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="dense_60k")
+    ap.add_argument("--n", type=int, default=None, help="resize the workload (profiling runs)")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--need-dv", action="store_true")
     ap.add_argument("--no-geo", dest="with_geo", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
@@ -390,7 +394,8 @@ def main():
     if rank == 0:
         if args.cpu_baseline:
             from spatial_spectral_attention_b200 import synth
-            tf, ms, rows, dt = oracle_sample(synth.make_workload(args.workload), 12.0, args.need_dv)
+            tf, ms, rows, dt = oracle_sample(synth.make_workload(args.workload, n=args.n), 12.0,
+                                             args.need_dv)
             res["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cpu_cores(),
                                    "kind": "oracle", "ms_full_step_est": round(ms, 1),
                                    "sample": f"{rows} of {res['config']['n']} target rows "

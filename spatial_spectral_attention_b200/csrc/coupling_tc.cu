@@ -50,8 +50,8 @@ namespace ssc {
 namespace {
 
 constexpr int kChunk = 128 * 128;  // bytes of a 128-row x 64-col bf16 swizzled box
-constexpr int kThreadsFwd = 192;
-constexpr int kThreadsBwd = 192;
+constexpr int kFwdSoftmaxGroups = 2;  // softmax warpgroups per forward CTA
+constexpr int kBwdComputeGroups = 2;  // compute warpgroups per backward CTA
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -101,23 +101,45 @@ __host__ __device__ inline int vtile_bytes(int vf, int vr) { return vf * kChunk 
 __host__ __device__ inline uint32_t rem_swizzle(int vr) { return vr == 16 ? kSw32 : kSw64; }
 
 // ------------------------------------------------------------------ forward
-__global__ void __launch_bounds__(kThreadsFwd, 1)
+// Max of 32 values by a balanced tree (short dependency chain).
+__device__ __forceinline__ float max32(const float (&x)[32]) {
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = fmaxf(x[i], x[i + 16]);
+#pragma unroll
+  for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return t[0];
+}
+
+// NWG softmax warpgroups split every query row's 128 key columns: thread
+// (wg, lane row) owns columns [wg*CW, (wg+1)*CW) of the S tile, CW = 128/NWG.
+template <int NWG>
+__global__ void __launch_bounds__(64 + 128 * NWG, 1)
     tc_fwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr int CW = 128 / NWG;  // S columns per softmax thread
+  constexpr int NC = CW / 32;    // 32-column TMEM loads per thread
+  constexpr int NSM = 128 * NWG; // softmax threads
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_kv_full[2], bar_kv_empty[2], bar_s_full[2],
-      bar_p_full[2], bar_o_full, bar_drain;
+      bar_p_full[2], bar_o_full, bar_drain, bar_xmax, bar_xsum;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  // Partial row maxima / sums exchanged between the softmax warpgroups through
+  // mbarriers (bounded waits, unlike a named barrier).
+  __shared__ float s_pmax[2][NWG][128];  // partial row maxima, double-buffered by tile parity
+  __shared__ float s_psum[NWG][128];     // partial row sums for the epilogue
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
   const int qbytes = p.qch * kChunk;
   const int vbytes = vtile_bytes(p.vf, p.vr);
   const uint32_t sQ = sbase;
   const uint32_t sK0 = sQ + qbytes;
   const uint32_t sV0 = sK0 + 2 * qbytes;
-  (void)gbase;
   const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
 
   if (threadIdx.x == 0) {
@@ -127,10 +149,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       mbar_init(&bar_kv_full[i], 1);
       mbar_init(&bar_kv_empty[i], 1);
       mbar_init(&bar_s_full[i], 1);
-      mbar_init(&bar_p_full[i], 128);
+      mbar_init(&bar_p_full[i], NSM);
     }
     mbar_init(&bar_o_full, 1);
     mbar_init(&bar_drain, 1);
+    mbar_init(&bar_xmax, NSM);
+    mbar_init(&bar_xsum, NSM);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -161,8 +185,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         mbar_arrive_expect_tx(&bar_q_full, qbytes);
         for (int c = 0; c < p.qch; ++c)
-          tma_load_2d(smem_raw + (sQ - smem_u32(smem_raw)) + c * kChunk, &tm.q, 64 * c, tile.row0,
-                      &bar_q_full);
+          tma_load_2d(gptr(sQ) + c * kChunk, &tm.q, 64 * c, tile.row0, &bar_q_full);
         q_issued = (int)tcount;
         bool ok = true;
         for (int j = 0; j < tile.nseg; ++j, ++it) {
@@ -173,8 +196,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             break;
           }
           mbar_arrive_expect_tx(&bar_kv_full[st], kv_bytes);
-          uint8_t* dk = smem_raw + (sK0 - smem_u32(smem_raw)) + st * qbytes;
-          uint8_t* dv = smem_raw + (sV0 - smem_u32(smem_raw)) + st * vbytes;
+          uint8_t* dk = gptr(sK0) + st * qbytes;
+          uint8_t* dv = gptr(sV0) + st * vbytes;
           for (int c = 0; c < p.qch; ++c)
             tma_load_2d(dk + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_kv_full[st]);
           for (int c = 0; c < p.vf; ++c)
@@ -254,61 +277,79 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       }
       // drain: wait until every tensor-core op issued here has completed
       mma_commit(&bar_drain);
-      WaitCtl c2 = p.ctl;
       volatile int never = 0;
-      mbar_wait(&bar_drain, 0, c2, &never);
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
     }
   } else {
-    // ---------------- softmax / epilogue (warps 2..5)
+    // ---------------- softmax / correction / epilogue (NWG warpgroups)
+    const int wg = (warp - 2) >> 2;
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = row within the tile
-    uint32_t it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int col0 = wg * CW;                 // first S column of this thread
+    const int nchunk = p.kp / 16;             // 16-column chunks of O
+    uint32_t it = 0, tcount = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       const RowTile tile = p.tiles[t];
       const int nk = tile.nseg;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
+      int nkeys_next = nk > 0 ? p.segs[tile.seg0].nkeys : 0;
       for (int j = 0; j < nk; ++j) {
         const uint32_t g = it + j;
         const int buf = g & 1;
+        const int nkeys = nkeys_next;
+        if (j + 1 < nk) nkeys_next = p.segs[tile.seg0 + j + 1].nkeys;
         if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int nkeys = p.segs[tile.seg0 + j].nkeys;
-        uint32_t r[4][32];
-        const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128);
+        float x[NC][32];
+        const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(sa + 32 * c, r[c]);
+        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_ld_wait();
-        float mx = -INFINITY;
+        if (nkeys < 128) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < NC; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float x = __uint_as_float(r[c][i]);
-            if (32 * c + i >= nkeys) x = -INFINITY;
-            r[c][i] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+            for (int i = 0; i < 32; ++i)
+              if (col0 + 32 * c + i >= nkeys) x[c][i] = -INFINITY;
+        }
+        float mx = max32(x[0]);
+#pragma unroll
+        for (int c = 1; c < NC; ++c) mx = fmaxf(mx, max32(x[c]));
+        if (NWG > 1) {
+          s_pmax[g & 1][wg][lrow] = mx;
+          mbar_arrive(&bar_xmax);
+          if (!mbar_wait(&bar_xmax, g & 1, p.ctl, abort)) {
+            ok = false;
+            break;
           }
+#pragma unroll
+          for (int w = 0; w < NWG; ++w) mx = fmaxf(mx, s_pmax[g & 1][w][lrow]);
+        }
         const float m_new = fmaxf(m, mx * p.scale_log2);
         const bool need = m_new > m + 8.0f;
+        // PV_{g-1} (the previous tile's contribution to O) must be waited for
+        // exactly once per tile: the parity wait is only sound when this thread
+        // is never more than one phase behind the barrier.
+        bool o_pending = j > 0;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O holds P_0..P_{j-1} V: wait for PV_{j-1}, then rescale in TMEM
           if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
             ok = false;
             break;
           }
+          o_pending = false;
           tc_fence_after();
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
           const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
-          for (int c0 = 0; c0 < p.kp; c0 += 16) {
+          for (int c = wg; c < nchunk; c += NWG) {
             uint32_t o[16];
-            tmem_ld16(oa + c0, o);
+            tmem_ld16(oa + 16 * c, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st16(oa + c0, o);
+            tmem_st16(oa + 16 * c, o);
           }
           tmem_st_wait();
           l *= f;
@@ -317,29 +358,43 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           m = m_new;
         }
         const float neg_m = -m;
-        float rs = 0.f;
-        uint32_t pk[4][16];
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[NC][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < NC; ++c)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i]), p.scale_log2, neg_m));
-            const float a1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i + 1]), p.scale_log2, neg_m));
-            rs += a0 + a1;
+            const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
+            const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], p.scale_log2, neg_m));
+            rs[i & 3] += a0 + a1;
             pk[c][i] = pack_bf16x2(a0, a1);
           }
-        l += rs;
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        // P over this thread's columns: TMEM columns buf*128 + col0/2 ...
+        const uint32_t pa = tmem_lane_addr(tmem, warp, buf * 128 + col0 / 2);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_st16(sa + 16 * c, pk[c]);
+        for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
         tmem_st_wait();
+        if (o_pending && !mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
         tc_fence_before();
         mbar_arrive(&bar_p_full[buf]);
       }
       if (!ok) break;
-      // epilogue: O / l, lse
+      // epilogue: wait for the last PV, combine the partial row sums, O / l, lse
       const uint32_t glast = it + nk - 1;
       if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
       tc_fence_after();
+      if (NWG > 1) {
+        s_psum[wg][lrow] = l;
+        mbar_arrive(&bar_xsum);
+        if (!mbar_wait(&bar_xsum, tcount & 1, p.ctl, abort)) break;
+        l = 0.f;
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) l += s_psum[w][lrow];
+      }
       const int row = tile.row0 + lrow;
       int orow = (lrow < tile.nrows && row < p.nq) ? (p.row_map ? p.row_map[row] : row) : -1;
       if (orow >= p.nq) orow = -1;
@@ -348,17 +403,26 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       float* optr = p.O + (size_t)orow * p.ldo;
       const float inv = 1.0f / l;
       const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
-      for (int c0 = 0; c0 < p.kp; c0 += 16) {
+      for (int c = wg; c < nchunk; c += NWG) {
         uint32_t o[16];
-        tmem_ld16(oa + c0, o);
+        tmem_ld16(oa + 16 * c, o);
         tmem_ld_wait();
         if (live) {
+          const int c0 = 16 * c;
+          if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(optr + c0 + i) =
+                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+          }
         }
       }
-      if (live) p.lse[orow] = (m + log2f(l)) * kLn2;
+      if (live && wg == 0) p.lse[orow] = (m + log2f(l)) * kLn2;
       it += nk;
     }
   }
@@ -373,9 +437,13 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
 
 // ------------------------------------------------------------------ backward
 // kDV = false: dQ (stored) and dK (atomics).  kDV = true: dV (atomics).
-template <bool kDV>
-__global__ void __launch_bounds__(kThreadsBwd, 1)
+// NCG compute warpgroups split the key columns of S / dP (and the columns of
+// the dK / dV / dQ flushes); every element is independent in the backward.
+template <bool kDV, int NCG>
+__global__ void __launch_bounds__(64 + 128 * NCG, 1)
     tc_bwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr int CW = 128 / NCG;  // key columns per compute thread
+  constexpr int NC = CW / 32;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_qg_full, bar_qg_empty, bar_k_full, bar_k_empty, bar_v_full, bar_v_empty,
       bar_sdp_full, bar_ds_full, bar_dkp_full, bar_dq_full, bar_drain;
@@ -403,7 +471,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     mbar_init(&bar_v_full, 1);
     mbar_init(&bar_v_empty, 1);
     mbar_init(&bar_sdp_full, 1);
-    mbar_init(&bar_ds_full, 128);
+    mbar_init(&bar_ds_full, 128 * NCG);
     mbar_init(&bar_dkp_full, 1);
     mbar_init(&bar_dq_full, 1);
     mbar_init(&bar_drain, 1);
@@ -564,11 +632,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_wait(&bar_drain, 0, p.ctl, &never);
     }
   } else {
-    // ---------------- compute (warps 2..5): one thread per query row for S/dP,
-    // one thread per key row for the dK / dV flush.
+    // ---------------- compute (NCG warpgroups): one thread per query row for
+    // S/dP, one thread per key row for the dK / dV flush.
+    const int wg = (warp - 2) >> 2;
     const int lrow = 32 * (warp & 3) + lane;
+    const int col0 = wg * CW;
     uint32_t it = 0, tcount = 0;
     const int kt_out = kDV ? p.kp : p.d;  // columns of the partial to flush
+    const int nchunk_out = kt_out / 16;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       const RowTile tile = p.tiles[t];
       const int qrow = tile.row0 + lrow;
@@ -576,38 +647,42 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const float lse2 = live_row ? p.lse_in[qrow] * kLog2e : 0.f;
       const float Di = (!kDV && live_row) ? p.Dvec[qrow] : 0.f;
       bool ok = true;
+      KeySeg sg_next = tile.nseg > 0 ? p.segs[tile.seg0] : KeySeg{0, 0};
       for (int j = 0; j < tile.nseg; ++j, ++it) {
-        const KeySeg sg = p.segs[tile.seg0 + j];
+        const KeySeg sg = sg_next;
+        if (j + 1 < tile.nseg) sg_next = p.segs[tile.seg0 + j + 1];
         if (!mbar_wait(&bar_sdp_full, it & 1, p.ctl, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t ta = tmem_lane_addr(tmem, warp, 0);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t s[32], dp[32];
-          tmem_ld32(ta + c_s + 32 * c, s);
-          if (!kDV) tmem_ld32(ta + c_dp + 32 * c, dp);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          uint32_t sv[32], dp[32];
+          tmem_ld32(ta + c_s + col0 + 32 * c, sv);
+          if (!kDV) tmem_ld32(ta + c_dp + col0 + 32 * c, dp);
           tmem_ld_wait();
           uint32_t pk[16];
+          const int cbase = col0 + 32 * c;
+          const bool full = live_row && cbase + 32 <= sg.nkeys;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             float v2[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int col = 32 * c + 2 * i + h;
-              float pr = ex2_approx(fmaf(__uint_as_float(s[2 * i + h]), p.scale_log2, -lse2));
-              if (col >= sg.nkeys || !live_row) pr = 0.f;
+              float pr = ex2_approx(fmaf(__uint_as_float(sv[2 * i + h]), p.scale_log2, -lse2));
+              if (!full && (cbase + 2 * i + h >= sg.nkeys || !live_row)) pr = 0.f;
               v2[h] = kDV ? pr : pr * (__uint_as_float(dp[2 * i + h]) - Di);
             }
             pk[i] = pack_bf16x2(v2[0], v2[1]);
           }
-          // row lrow, keys [32c, 32c+32): chunk c/2, 16-byte units (c&1)*4 + 0..3
-          const uint32_t rowb = sS + (c >> 1) * kChunk + lrow * 128;
+          // row lrow, keys [cbase, cbase+32): 64-key chunk cbase/64, 16-byte
+          // units ((cbase%64)/8) + 0..3, swizzled by the row
+          const uint32_t rowb = sS + (cbase >> 6) * kChunk + lrow * 128;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint32_t unit = ((c & 1) * 4 + u) ^ (lrow & 7);
+            const uint32_t unit = (((cbase & 63) >> 3) + u) ^ (lrow & 7);
             asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(rowb + unit * 16),
                          "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
                          : "memory");
@@ -616,7 +691,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar_ds_full);
-        // flush the partial dK (or dV) of this key tile: thread = key row
+        // flush the partial dK (or dV) of this key tile: thread = key row,
+        // 16-column chunks split among the warpgroups
         if (!mbar_wait(&bar_dkp_full, it & 1, p.ctl, abort)) {
           ok = false;
           break;
@@ -630,7 +706,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         float* dst = kDV ? p.dV + (size_t)okey * p.lddv : p.dK + (size_t)okey * p.lddk;
         const int ncols = kDV ? p.k : p.d;
         const float mul = kDV ? 1.0f : p.scale;
-        for (int c0 = 0; c0 < kt_out; c0 += 16) {
+        for (int cc = wg; cc < nchunk_out; cc += NCG) {
+          const int c0 = 16 * cc;
           uint32_t o[16];
           tmem_ld16(ta + c_dkp + c0, o);
           tmem_ld_wait();
@@ -652,8 +729,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
       }
       if (!ok) break;
+      if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
       if (!kDV) {
-        if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
         tc_fence_after();
         // TMEM loads are warp-collective: every lane loads, live rows store
         int orow = live_row ? (p.row_map ? p.row_map[qrow] : qrow) : -1;
@@ -661,17 +738,21 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (!store_row) orow = 0;
         float* dq = p.dQ + (size_t)orow * p.lddq;
         const uint32_t ta = tmem_lane_addr(tmem, warp, c_dq);
-        for (int c0 = 0; c0 < p.d; c0 += 16) {
+        for (int cc = wg; cc < p.d / 16; cc += NCG) {
           uint32_t o[16];
-          tmem_ld16(ta + c0, o);
+          tmem_ld16(ta + 16 * cc, o);
           tmem_ld_wait();
-          if (store_row) {
+          if (store_row && (p.lddq & 3) == 0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) dq[c0 + i] = __uint_as_float(o[i]) * p.scale;
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(dq + 16 * cc + i) = make_float4(
+                  __uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                  __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
+          } else if (store_row) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dq[16 * cc + i] = __uint_as_float(o[i]) * p.scale;
           }
         }
-      } else {
-        if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
       }
     }
   }
@@ -792,11 +873,13 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
   if (p.vr && !make_map(&tm.vr, a.V, a.nKrows, a.k, a.ldv, p.vr, rem_sw_host(p.vr)))
     return cudaErrorInvalidValue;
   const int smem = 1024 + p.qch * kChunk * 3 + 2 * vtile_bytes(p.vf, p.vr);
-  cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int NWG = kFwdSoftmaxGroups;
+  cudaError_t e =
+      cudaFuncSetAttribute(tc_fwd_kernel<NWG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
   const int grid = std::max(1, std::min(work, num_sms()));
-  tc_fwd_kernel<<<grid, kThreadsFwd, smem, st>>>(tm, p);
+  tc_fwd_kernel<NWG><<<grid, 64 + 128 * NWG, smem, st>>>(tm, p);
   count_launch();
   return cudaGetLastError();
 }
@@ -831,20 +914,20 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
   {
     p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
     const int smem = 1024 + 2 * p.qch * kChunk + 2 * vb + 2 * kChunk;
-    cudaError_t e =
-        cudaFuncSetAttribute(tc_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = tc_bwd_kernel<false, kBwdComputeGroups>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_bwd_kernel<false><<<grid, kThreadsBwd, smem, st>>>(tm, p);
+    kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (dV) {
     p.vec_atomics = (lddv % 4 == 0) && (reinterpret_cast<uintptr_t>(dV) % 16 == 0);
     const int smem = 1024 + 2 * p.qch * kChunk + vb + 2 * kChunk;
-    cudaError_t e =
-        cudaFuncSetAttribute(tc_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = tc_bwd_kernel<true, kBwdComputeGroups>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_bwd_kernel<true><<<grid, kThreadsBwd, smem, st>>>(tm, p);
+    kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

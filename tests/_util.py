@@ -26,14 +26,25 @@ def errors(got, ref):
     return maxabs, relfro
 
 
-def assert_close(got, ref, tol, name=""):
+def assert_close(got, ref, tol, name="", scale_by_ref=False):
+    """max-abs and relative-Frobenius bounds.
+
+    The relative measure is skipped when the exact result is zero to rounding
+    (||ref||_F below 1e-9 per element, e.g. the gradients of a single-key
+    coupling, which vanish identically); max-abs still applies.  With
+    scale_by_ref the max-abs bound is multiplied by max(1, max|ref|): bf16
+    rounding is relative, so stress inputs with outputs far above the
+    workloads' O(1) magnitudes get the same relative allowance."""
     if isinstance(got, torch.Tensor):
         got = got.detach().double().cpu().numpy()
+    ref = np.asarray(ref, dtype=np.float64)
     maxabs, relfro = errors(got, ref)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    assert maxabs <= tol["maxabs"] and relfro <= tol["relfro"], (
-        f"{name}: max-abs {maxabs:.3e} (<= {tol['maxabs']}), rel-Frobenius {relfro:.3e} "
-        f"(<= {tol['relfro']})")
+    bound = tol["maxabs"] * (max(1.0, float(np.abs(ref).max())) if scale_by_ref else 1.0)
+    degenerate = float(np.linalg.norm(ref)) < 1e-9 * np.sqrt(max(ref.size, 1))
+    ok = maxabs <= bound and (degenerate or relfro <= tol["relfro"])
+    assert ok, (f"{name}: max-abs {maxabs:.3e} (<= {bound:.3g}), rel-Frobenius {relfro:.3e} "
+                f"(<= {tol['relfro']}{', skipped: exact result is zero' if degenerate else ''})")
     return maxabs, relfro
 
 

@@ -31,19 +31,20 @@ def _status_ok():
     assert api.ssc_device_status() == 0
 
 
-def _dense_case(Qn, Kn, Vn, dOn, scale, dtype, need_dV=True):
+def _dense_case(Qn, Kn, Vn, dOn, scale, dtype, need_dV=True, scale_by_ref=False):
     tol = TOL_BF16 if dtype == "bf16" else TOL_F32
     (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(Qn, Kn, Vn, dOn, dtype)
     O, lse = api.ssc_dense_coupling_fwd(Q, K, V, scale)
     dQ, dK, dV = api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=need_dV)
     _status_ok()
     ref = oracle.dense_bwd(Q64, K64, V64, dO64, scale)
-    assert_close(O, ref["O"], tol, "O")
-    assert_close(lse, ref["lse"], tol, "lse")
-    assert_close(dQ, ref["dQ"], tol, "dQ")
-    assert_close(dK, ref["dK"], tol, "dK")
+    kw = dict(scale_by_ref=scale_by_ref)
+    assert_close(O, ref["O"], tol, "O", **kw)
+    assert_close(lse, ref["lse"], tol, "lse", **kw)
+    assert_close(dQ, ref["dQ"], tol, "dQ", **kw)
+    assert_close(dK, ref["dK"], tol, "dK", **kw)
     if need_dV:
-        assert_close(dV, ref["dV"], tol, "dV")
+        assert_close(dV, ref["dV"], tol, "dV", **kw)
 
 
 def test_dense_fp32_check_mode_small_workload():
@@ -82,9 +83,10 @@ def test_dense_bf16_unaligned_v_is_repacked():
 
 
 def test_dense_bf16_peaked_softmax_rescaling():
-    # a large scale makes the running max jump often: exercises the O rescale
+    # a large scale makes the running max jump often: exercises the O rescale.
+    # Gradients here reach |dQ| ~ 10, so the max-abs bound scales with max|ref|.
     Qn, Kn, Vn, dOn = synth.random_inputs(256, 1024, 128, 64, seed=9)
-    _dense_case(Qn, Kn, Vn, dOn, 0.6, "bf16")
+    _dense_case(Qn, Kn, Vn, dOn, 0.6, "bf16", scale_by_ref=True)
 
 
 def test_dense_bf16_full_size_sampled():
