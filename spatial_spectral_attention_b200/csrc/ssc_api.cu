@@ -6,7 +6,7 @@
 #include <cmath>
 #include <cstdint>
 
-#include "../../include/ssc.h"
+#include "ssc.h"
 #include "internal.h"
 
 using namespace ssc;
@@ -232,6 +232,7 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex, int* center
   if (n < 1 || P < 1 || P > n || P > 65535 || n > (1 << 24)) return SSC_ERR_INVALID_ARG;
   if (seed_vertex < 0 || seed_vertex >= n) return SSC_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, fps_workspace_bytes(n, P))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   WaitCtl c = make_ctl();
   return cuda_status(launch_fps_patches(pts, n, P, seed_vertex, centers, owner, offsets, members, ws,
                                         static_cast<cudaStream_t>(stream), c));
@@ -252,6 +253,7 @@ int ssc_patch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int l
   if (PN < 1 || PM < 1 || PN > nN || PM > nM || PN > 65535 || PM > 65535) return SSC_ERR_INVALID_ARG;
   if (R < 1 || R > PM) return SSC_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, scores_topk_workspace_bytes(PN, PM, d))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   WaitCtl c = make_ctl();
   return cuda_status(launch_scores_topk(FN, ldn, nN, FM, ldm, nM, d, dtype, offN, memN, PN, offM,
                                         memM, PM, R, topk, scores, ws, c.status,
@@ -272,6 +274,7 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
   if ((rc = check_out(O, ldo, k))) return rc;
   if (!lse) return SSC_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, dense_ws(nullptr, nN, nM, d, k, dtype, nullptr))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DenseWs w;
   dense_ws(ws, nN, nM, d, k, dtype, &w);
@@ -304,6 +307,7 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
   if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
   if (dV && (rc = check_out(dV, lddv, k))) return rc;
   if (!ws_ok(ws, ws_bytes, dense_ws(nullptr, nN, nM, d, k, dtype, nullptr))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WaitCtl ctl = make_ctl();
   DenseWs w;
@@ -388,6 +392,7 @@ int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const v
   if (!lse) return SSC_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
     return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WaitCtl ctl = make_ctl();
   GeoWs w;
@@ -421,6 +426,7 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const v
   if (dV && (rc = check_out(dV, lddv, k))) return rc;
   if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
     return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WaitCtl ctl = make_ctl();
   GeoWs w;
