@@ -1,0 +1,483 @@
+// coupling_tc2.cu -- the dense forward coupling on CTA pairs (2-SM tcgen05 MMAs).
+//
+// Same operation as tc_fwd_kernel ("Spatial-Spectral Coupling as Attention",
+// project page, "Spatial-spectral coupling is attention": O = softmax(s Q K^T) V
+// with Q = F_N, K = F_M, V = Phi_M, plus lse), laid out for the B200's 2-SM
+// tensor-core instructions.  A cluster of two CTAs owns a 256-row query tile;
+// CTA r holds query rows [128 r, 128 r + 128) of it.  For every 128-key tile
+// each CTA loads only half of the shared operands -- 64 key rows of K and half
+// of the (32-padded) V columns -- and the even CTA issues M = 256 MMAs that read
+// both halves:
+//     S = Q K^T    SS, M = 256, N = 128 keys (each CTA: 64 keys of B)
+//     O += P V     TS, P from each CTA's tensor memory, N = kp2 (V padded to a
+//                  multiple of 32; each CTA supplies kp2/2 columns of B)
+// Each CTA's tensor memory receives its own 128 rows of S and O, so the softmax
+// warps of both CTAs run exactly as in the single-CTA kernel.  This halves the
+// bytes every SM streams per key tile (K and V traffic is the limit of the
+// single-CTA forward) and reduces the shared-memory operand reads per MMA.
+//
+// Barrier topology: operand "full" barriers and the P-ready barrier live in the
+// even CTA (the MMA issuer); TMA loads of both CTAs complete on them.  Every
+// "empty"/"ready" signal produced by the MMAs is a commit multicast to both
+// CTAs.  All waits are bounded.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "internal.h"
+
+namespace ssc {
+namespace {
+
+constexpr int kChunk = 128 * 128;     // 128 rows x 64 bf16, 128B-swizzled
+constexpr int kHalfChunk = 64 * 128;  // 64 rows x 64 bf16
+constexpr int kKS = 4;                // K ring depth
+constexpr int kVS = 3;                // V ring depth
+constexpr int kNWG = 2;               // softmax warpgroups per CTA
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct PairMaps {
+  CUtensorMap q;  // {d, nq}, box {64, 128}
+  CUtensorMap k;  // {d, nk}, box {64, 64}: one CTA's half of a key tile
+  CUtensorMap v;  // {k, nk}, box {64, 128}
+};
+
+struct PairParams {
+  int nq, nk, d, k;
+  int kp2;     // V columns padded to a multiple of 32 (MMA N of P V)
+  int qch;     // d / 64
+  int vh;      // V columns supplied by each CTA (kp2 / 2)
+  int vbox;    // 64-column boxes per CTA per V tile
+  int nkt;     // key tiles of 128
+  int ntiles;  // query tiles of 256 rows
+  float scale_log2;
+  float* O;
+  int ldo;
+  float* lse;
+  WaitCtl ctl;
+};
+
+__device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, uint32_t col) {
+  return base + ((uint32_t)(32 * (warp & 3)) << 16) + col;
+}
+
+__device__ __forceinline__ float max32(const float (&x)[32]) {
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = fmaxf(x[i], x[i + 16]);
+#pragma unroll
+  for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return t[0];
+}
+
+template <int NWG>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
+    tc_fwd_pair_kernel(const __grid_constant__ PairMaps tm, const PairParams p) {
+  constexpr int CW = 128 / NWG;
+  constexpr int NC = CW / 32;
+  constexpr int NSM = 128 * NWG;
+  constexpr int kVWarp = 2 + 4 * NWG;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[kKS], bar_k_empty[kKS], bar_v_full[kVS],
+      bar_v_empty[kVS], bar_s_full[2], bar_p_full[2], bar_o_full, bar_drain, bar_xmax, bar_xsum;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ float s_pmax[2][NWG][128];
+  __shared__ float s_psum[NWG][128];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
+  const int qbytes = p.qch * kChunk;
+  const int kbytes = p.qch * kHalfChunk;
+  const int vbytes = p.vbox * kChunk;
+  const uint32_t sQ = sbase;
+  const uint32_t sK0 = sQ + qbytes;
+  const uint32_t sV0 = sK0 + kKS * kbytes;
+  // barriers of the even CTA, as cluster addresses
+  auto lead = [&](uint64_t* b) { return mapa_shared(smem_u32(b), 0); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    for (int i = 0; i < kKS; ++i) {
+      mbar_init(&bar_k_full[i], 1);
+      mbar_init(&bar_k_empty[i], 1);
+    }
+    for (int i = 0; i < kVS; ++i) {
+      mbar_init(&bar_v_full[i], 1);
+      mbar_init(&bar_v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_p_full[i], 2 * (NSM / 32));  // one arrival per softmax warp of both CTAs
+    }
+    mbar_init(&bar_o_full, 1);
+    mbar_init(&bar_drain, 1);
+    mbar_init(&bar_xmax, NSM);
+    mbar_init(&bar_xsum, NSM);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s_tmem, 512);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm.q);
+    tma_prefetch_desc(&tm.k);
+    tma_prefetch_desc(&tm.v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote operation
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+
+  if (warp == 0) {
+    // ---------------- Q and K producer (both CTAs)
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      for (int t = pair; t < p.ntiles && !*abort; t += npairs, ++tcount) {
+        const int row0 = t * 256 + 128 * (int)rank;
+        if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        if (rank == 0) mbar_arrive_expect_tx(&bar_q_full, 2 * qbytes);
+        for (int c = 0; c < p.qch; ++c)
+          tma_load_2d_pair(gptr(sQ) + c * kChunk, &tm.q, 64 * c, row0, lead(&bar_q_full));
+        bool ok = true;
+        for (int j = 0; j < p.nkt; ++j, ++it) {
+          const int st = it % kKS;
+          if (it >= (uint32_t)kKS &&
+              !mbar_wait(&bar_k_empty[st], ((it / kKS) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&bar_k_full[st], 2 * kbytes);
+          for (int c = 0; c < p.qch; ++c)
+            tma_load_2d_pair(gptr(sK0) + st * kbytes + c * kHalfChunk, &tm.k, 64 * c,
+                             j * 128 + 64 * (int)rank, lead(&bar_k_full[st]));
+        }
+        if (!ok) break;
+      }
+      if (*abort) __nanosleep(20000);  // let copies already in flight land
+    }
+  } else if (warp == kVWarp) {
+    // ---------------- V producer (both CTAs): this CTA's kp2/2 columns
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = pair; t < p.ntiles && !*abort; t += npairs) {
+        bool ok = true;
+        for (int j = 0; j < p.nkt; ++j, ++it) {
+          const int st = it % kVS;
+          if (it >= (uint32_t)kVS &&
+              !mbar_wait(&bar_v_empty[st], ((it / kVS) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&bar_v_full[st], 2 * vbytes);
+          for (int b = 0; b < p.vbox; ++b)
+            tma_load_2d_pair(gptr(sV0) + st * vbytes + b * kChunk, &tm.v,
+                             p.vh * (int)rank + 64 * b, j * 128, lead(&bar_v_full[st]));
+        }
+        if (!ok) break;
+      }
+      if (*abort) __nanosleep(20000);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (even CTA only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(256, 128, 0, 0);
+      const uint32_t idesc_pv = make_idesc_bf16(256, p.kp2, 0, 1);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      auto issue_s = [&](uint32_t g) -> bool {
+        const int st = g % kKS;
+        if (!mbar_wait(&bar_k_full[st], (g / kKS) & 1, p.ctl, abort)) return false;
+        tc_fence_after();
+        const uint32_t sk = sK0 + st * kbytes;
+        const uint32_t d_tmem = tmem + (g & 1) * 128;
+        for (int kk = 0; kk < p.d / 16; ++kk) {
+          const uint32_t ch = kk >> 2, w = (kk & 3) * 32;
+          mma_ss_pair(d_tmem, make_sdesc(sQ + ch * kChunk + w, 16, 1024, kSw128),
+                      make_sdesc(sk + ch * kHalfChunk + w, 16, 1024, kSw128), idesc_s, kk > 0);
+        }
+        mma_commit_pair(&bar_s_full[g & 1]);
+        mma_commit_pair(&bar_k_empty[st]);
+        return true;
+      };
+      for (int t = pair; t < p.ntiles && ok; t += npairs, ++tcount) {
+        const int nk = p.nkt;
+        if (!mbar_wait(&bar_q_full, tcount & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < std::min(2, nk) && ok; ++j) ok = issue_s(it + j);
+        for (int j = 0; j < nk && ok; ++j) {
+          const uint32_t g = it + j;
+          const int buf = g & 1, vst = g % kVS;
+          if (!mbar_wait_cluster(&bar_p_full[buf], (g >> 1) & 1, p.ctl, abort) ||
+              !mbar_wait(&bar_v_full[vst], (g / kVS) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sv = sV0 + vst * vbytes;
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_pair(tmem + 256, tmem + buf * 128 + kk * 8,
+                        make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_pair(&bar_v_empty[vst]);
+          mma_commit_pair(&bar_o_full);
+          if (j + 2 < nk) ok = issue_s(g + 2);
+        }
+        mma_commit_pair(&bar_q_empty);
+        it += nk;
+      }
+      mma_commit_pair(&bar_drain);
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue (both CTAs)
+    const int wg = (warp - 2) >> 2;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int col0 = wg * CW;
+    const int nchunk = p.kp2 / 16;
+    uint32_t it = 0, tcount = 0;
+    for (int t = pair; t < p.ntiles; t += npairs, ++tcount) {
+      const int row0 = t * 256 + 128 * (int)rank;
+      const int nk = p.nkt;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nk; ++j) {
+        const uint32_t g = it + j;
+        const int buf = g & 1;
+        const int nkeys = min(128, p.nk - 128 * j);
+        if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float x[NC][32];
+        const uint32_t sa = lane_addr(tmem, warp, buf * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, reinterpret_cast<uint32_t(&)[32]>(x[c]));
+        tmem_ld_wait();
+        if (nkeys < 128) {
+#pragma unroll
+          for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + 32 * c + i >= nkeys) x[c][i] = -INFINITY;
+        }
+        float mx = max32(x[0]);
+#pragma unroll
+        for (int c = 1; c < NC; ++c) mx = fmaxf(mx, max32(x[c]));
+        if (NWG > 1) {
+          s_pmax[g & 1][wg][lrow] = mx;
+          mbar_arrive(&bar_xmax);
+          if (!mbar_wait(&bar_xmax, g & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int w = 0; w < NWG; ++w) mx = fmaxf(mx, s_pmax[g & 1][w][lrow]);
+        }
+        const float m_new = fmaxf(m, mx * p.scale_log2);
+        const bool need = m_new > m + 8.0f;
+        // one wait on O per key tile keeps the parity wait in step
+        bool o_pending = j > 0;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          o_pending = false;
+          tc_fence_after();
+          const float f = need ? ex2_approx(m - m_new) : 1.0f;
+          const uint32_t oa = lane_addr(tmem, warp, 256);
+          for (int c = wg; c < nchunk; c += NWG) {
+            uint32_t o[16];
+            tmem_ld16(oa + 16 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st16(oa + 16 * c, o);
+          }
+          tmem_st_wait();
+          l *= f;
+          if (need) m = m_new;
+        } else if (need) {
+          m = m_new;
+        }
+        const float neg_m = -m;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[NC][16];
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
+            const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], p.scale_log2, neg_m));
+            rs[i & 3] += a0 + a1;
+            pk[c][i] = pack_bf16x2(a0, a1);
+          }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        const uint32_t pa = lane_addr(tmem, warp, buf * 128 + col0 / 2);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
+        tmem_st_wait();
+        if (o_pending && !mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&bar_p_full[buf]);
+          else mbar_arrive_remote(lead(&bar_p_full[buf]));
+        }
+      }
+      if (!ok) break;
+      const uint32_t glast = it + nk - 1;
+      if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      if (NWG > 1) {
+        s_psum[wg][lrow] = l;
+        mbar_arrive(&bar_xsum);
+        if (!mbar_wait(&bar_xsum, tcount & 1, p.ctl, abort)) break;
+        l = 0.f;
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) l += s_psum[w][lrow];
+      }
+      const int row = row0 + lrow;
+      const bool live = row < p.nq;
+      float* optr = p.O + (size_t)(live ? row : 0) * p.ldo;
+      const float inv = 1.0f / l;
+      const uint32_t oa = lane_addr(tmem, warp, 256);
+      for (int c = wg; c < nchunk; c += NWG) {
+        uint32_t o[16];
+        tmem_ld16(oa + 16 * c, o);
+        tmem_ld_wait();
+        if (live) {
+          const int c0 = 16 * c;
+          if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(optr + c0 + i) =
+                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+          }
+        }
+      }
+      if (live && wg == 0) p.lse[row] = (m + log2f(l)) * kLn2;
+      it += nk;
+    }
+  }
+
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer's MMAs or signals may target it
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn2() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool map2(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn2();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_pair_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
+
+cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
+                               const __nv_bfloat16* V, int ldv, int nN, int nM, int d, int k,
+                               float scale, float* O, int ldo, float* lse, cudaStream_t st,
+                               const WaitCtl& ctl) {
+  PairParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.nq = nN;
+  p.nk = nM;
+  p.d = d;
+  p.k = k;
+  p.kp2 = (k + 31) / 32 * 32;
+  p.qch = d / 64;
+  p.vh = p.kp2 / 2;
+  p.vbox = (p.vh + 63) / 64;
+  p.nkt = (nM + 127) / 128;
+  p.ntiles = (nN + 255) / 256;
+  p.scale_log2 = scale * kLog2e;
+  p.O = O;
+  p.ldo = ldo;
+  p.lse = lse;
+  p.ctl = ctl;
+  PairMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (!map2(&tm.q, Q, nN, d, ldq, 64, 128) || !map2(&tm.k, K, nM, d, ldk, 64, 64) ||
+      !map2(&tm.v, V, nM, k, ldv, 64, 128))
+    return cudaErrorInvalidValue;
+  auto kern = tc_fwd_pair_kernel<kNWG>;
+  const int smem = 1024 + p.qch * kChunk + kKS * p.qch * kHalfChunk + kVS * p.vbox * kChunk;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 96 + 128 * kNWG;
+  // pairs that can be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.gridDim = dim3(2 * std::max(1, sms / 2));
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1)
+    nclusters = std::max(1, sms / 2);
+  cudaGetLastError();
+  const int pairs = std::max(1, std::min(p.ntiles, nclusters));
+  cfg.gridDim = dim3(2 * pairs);
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, tm, p);
+}
+
+}  // namespace ssc

@@ -290,6 +290,10 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
   const __nv_bfloat16* Vt;
   int ldvt;
   if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (tc_pair_supported(d, k))
+    return cuda_status(launch_tc_fwd_pair(static_cast<const __nv_bfloat16*>(Q), ldq,
+                                          static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt, nN,
+                                          nM, d, k, scale, O, ldo, lse, st, ctl));
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
            ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), nullptr,
            nullptr};
