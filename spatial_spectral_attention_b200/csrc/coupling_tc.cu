@@ -69,6 +69,7 @@ struct TcParams {
   const KeySeg* segs;
   const int* ntiles_dev;
   int ntiles_host;
+  const int* tile_prefix;  // [ntiles + 1]: units (key segments) before each row tile
   const int* row_map;
   const int* col_map;
   int d, k, kp, qch, vf, vr;
@@ -90,6 +91,7 @@ struct TcParams {
   float* dV;
   int lddv;
   int vec_atomics;
+  int vec_atomics_dq;
   WaitCtl ctl;
 };
 
@@ -471,15 +473,33 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
 
 // ------------------------------------------------------------------ backward
 // kDV = false: dQ (stored) and dK (atomics).  kDV = true: dV (atomics).
-// The backward visits the key tiles of a row tile starting at a CTA-dependent
-// offset: the result does not depend on the order, and CTAs that would walk the
-// keys in lockstep otherwise all reduce into the same rows of dK at once.
-__device__ __forceinline__ int seg_rotation(int nseg) {
-  return nseg > 0 ? (int)((blockIdx.x * 131u) % (unsigned)nseg) : 0;
-}
-__device__ __forceinline__ int rotated(int j, int rot, int nseg) {
-  const int r = j + rot;
-  return r >= nseg ? r - nseg : r;
+// The backward's work is the flat list of (row tile, key segment) units, in
+// row-tile order; CTA c takes units [c U / G, (c + 1) U / G).  Every CTA gets
+// the same amount of work (no tail wave), at the price that a row tile may be
+// shared by two CTAs, which then reduce their dQ contributions atomically.
+struct UnitRange {
+  int t, j, left;  // current tile, first segment in it, units still to do
+};
+// Next run of consecutive segments [jb, je) of one tile t; false when done.
+__device__ __forceinline__ bool next_segment(UnitRange& r, const RowTile* tiles, int ntiles, int& t,
+                                             int& jb, int& je) {
+  while (r.left > 0 && r.t < ntiles) {
+    const int avail = tiles[r.t].nseg - r.j;
+    if (avail <= 0) {
+      ++r.t;
+      r.j = 0;
+      continue;
+    }
+    const int take = min(avail, r.left);
+    t = r.t;
+    jb = r.j;
+    je = r.j + take;
+    r.left -= take;
+    ++r.t;
+    r.j = 0;
+    return true;
+  }
+  return false;
 }
 
 // NCG compute warpgroups split the key columns of S / dP (and the columns of
@@ -494,6 +514,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       bar_sdp_full, bar_ds_full, bar_dkp_full, bar_dq_full, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_range[3];  // first tile, first segment in it, number of units
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base_u = smem_u32(smem_raw);
@@ -522,6 +543,19 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     mbar_init(&bar_drain, 1);
     s_abort = 0;
     fence_barrier_init();
+    // this CTA's share of the (row tile, key segment) units
+    const int U = p.tile_prefix[ntiles];
+    const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+    const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+    int lo = 0, hi = ntiles;  // largest t < ntiles with prefix[t] <= u0
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.tile_prefix[mid] <= u0) lo = mid;
+      else hi = mid;
+    }
+    s_range[0] = lo;
+    s_range[1] = ntiles > 0 ? (int)(u0 - p.tile_prefix[lo]) : 0;
+    s_range[2] = ntiles > 0 ? (int)(u1 - u0) : 0;
   }
   if (warp == 1) {
     tmem_alloc(&s_tmem, 512);
@@ -539,7 +573,9 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       int q_issued = -1, k_last = -1, v_last = -1;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
+      UnitRange ur{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (!*abort && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
         const RowTile tile = p.tiles[t];
         if (tcount > 0 && !mbar_wait(&bar_qg_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         q_issued = (int)tcount;
@@ -550,9 +586,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
           tma_load_2d(gptr(sG) + c * kChunk, &tm.g, 64 * c, tile.row0, &bar_qg_full);
         if (p.vr) tma_load_2d(gptr(sG) + p.vf * kChunk, &tm.gr, 64 * p.vf, tile.row0, &bar_qg_full);
         bool ok = true;
-        const int rot = seg_rotation(tile.nseg);
-        for (int j = 0; j < tile.nseg; ++j, ++it) {
-          const KeySeg sg = p.segs[tile.seg0 + rotated(j, rot, tile.nseg)];
+        for (int j = jb; j < je; ++j, ++it) {
+          const KeySeg sg = p.segs[tile.seg0 + j];
           if (!kDV) {
             if (it >= 1 && !mbar_wait(&bar_v_empty, (it - 1) & 1, p.ctl, abort)) {
               ok = false;
@@ -573,6 +608,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
             tma_load_2d(gptr(sK) + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_k_full);
           k_last = (int)it;
         }
+        ++tcount;
         if (!ok) break;
       }
       if (*abort) {
@@ -595,14 +631,15 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       const uint32_t rrow = (uint32_t)p.vr * 2;
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-        const RowTile tile = p.tiles[t];
+      UnitRange ur{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
         if (!mbar_wait(&bar_qg_full, tcount & 1, p.ctl, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int j = 0; j < tile.nseg && ok; ++j, ++it) {
+        for (int j = jb; j < je && ok; ++j, ++it) {
           if (!kDV) {
             // dP = dO V^T (K = kp)
             if (!mbar_wait(&bar_v_full, it & 1, p.ctl, abort)) {
@@ -648,7 +685,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
               const uint32_t aoff = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + c_dq, make_sdesc(sS + aoff, 16, 1024, kSw128),
                      make_sdesc(sK + kk * 2048, kChunk, 1024, kSw128), idesc_dq,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+                     (j > jb || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bar_k_empty);
             if (p.dk_t) {
@@ -681,6 +718,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         if (!ok) break;
         mma_commit(&bar_dq_full);
         mma_commit(&bar_qg_empty);
+        ++tcount;
       }
       mma_commit(&bar_drain);
       volatile int never = 0;
@@ -695,18 +733,19 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     uint32_t it = 0, tcount = 0;
     const int kt_out = kDV ? p.kp : p.d;  // columns of the partial to flush
     const int nchunk_out = kt_out / 16;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+    UnitRange ur{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    for (; next_segment(ur, p.tiles, ntiles, t, jb, je); ++tcount) {
       const RowTile tile = p.tiles[t];
       const int qrow = tile.row0 + lrow;
       const bool live_row = lrow < tile.nrows && qrow < p.nq;
       const float lse2 = live_row ? p.lse_in[qrow] * kLog2e : 0.f;
       const float Di = (!kDV && live_row) ? p.Dvec[qrow] : 0.f;
       bool ok = true;
-      const int rot = seg_rotation(tile.nseg);
-      KeySeg sg_next = tile.nseg > 0 ? p.segs[tile.seg0 + rot] : KeySeg{0, 0};
-      for (int j = 0; j < tile.nseg; ++j, ++it) {
+      KeySeg sg_next = p.segs[tile.seg0 + jb];
+      for (int j = jb; j < je; ++j, ++it) {
         const KeySeg sg = sg_next;
-        if (j + 1 < tile.nseg) sg_next = p.segs[tile.seg0 + rotated(j + 1, rot, tile.nseg)];
+        if (j + 1 < je) sg_next = p.segs[tile.seg0 + j + 1];
         if (!mbar_wait(&bar_sdp_full, it & 1, p.ctl, abort)) {
           ok = false;
           break;
@@ -810,6 +849,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         // TMEM loads are warp-collective: every lane loads, live rows store
         int orow = live_row ? (p.row_map ? p.row_map[qrow] : qrow) : -1;
         const bool store_row = orow >= 0 && orow < p.nq;
+        const bool whole = jb == 0 && je == tile.nseg;  // all of the row tile's keys done here
         if (!store_row) orow = 0;
         float* dq = p.dQ + (size_t)orow * p.lddq;
         const uint32_t ta = tmem_lane_addr(tmem, warp, c_dq);
@@ -817,13 +857,27 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
           uint32_t o[16];
           tmem_ld16(ta + 16 * cc, o);
           tmem_ld_wait();
-          if (store_row && (p.lddq & 3) == 0) {
+          if (!store_row) continue;
+          if (!whole) {
+            // the row tile's keys are split over several CTAs: reduce into dQ
+            if (p.vec_atomics_dq) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                atomicAdd(reinterpret_cast<float4*>(dq + 16 * cc + i),
+                          make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                      __uint_as_float(o[i + 2]) * p.scale,
+                                      __uint_as_float(o[i + 3]) * p.scale));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) atomicAdd(dq + 16 * cc + i, __uint_as_float(o[i]) * p.scale);
+            }
+          } else if ((p.lddq & 3) == 0) {
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
               *reinterpret_cast<float4*>(dq + 16 * cc + i) = make_float4(
                   __uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
                   __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
-          } else if (store_row) {
+          } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) dq[16 * cc + i] = __uint_as_float(o[i]) * p.scale;
           }
@@ -924,6 +978,7 @@ void fill_common(const TcArgs& a, TcParams& p) {
   p.segs = a.segs;
   p.ntiles_dev = a.ntiles_dev;
   p.ntiles_host = a.ntiles_host;
+  p.tile_prefix = a.tile_prefix;
   p.row_map = a.row_map;
   p.col_map = a.col_map;
   p.d = a.d;
@@ -993,6 +1048,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
   p.dV = dV;
   p.lddv = lddv;
   p.ctl = ctl;
+  p.vec_atomics_dq = (lddq % 4 == 0) && (reinterpret_cast<uintptr_t>(dQ) % 16 == 0);
   TensorMaps tm;
   std::memset(&tm, 0, sizeof(tm));
   if (!make_map(&tm.q, a.Q, a.nQrows, a.d, a.ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1004,8 +1060,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                !make_map(&tm.gr, dOb, a.nQrows, a.k, lddob, p.vr, rem_sw_host(p.vr))))
     return cudaErrorInvalidValue;
   const int vb = vtile_bytes(p.vf, p.vr);
-  const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
-  const int grid = std::max(1, std::min(work, num_sms()));
+  const int grid = num_sms();  // units are split evenly over every SM
   {
     p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
     p.dk_t = 0;  // the transposed flush measured slower on B200; kept for reference

@@ -83,7 +83,9 @@ cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, 
 // Dense schedule: ceil(nN/128) row tiles, all pointing at ceil(nM/128) segments.
 int dense_num_tiles(int nN);
 int dense_num_segs(int nM);
-cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, cudaStream_t st);
+// prefix [ntiles + 1] receives the prefix sums of the tiles' segment counts.
+cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, int* prefix,
+                                  cudaStream_t st);
 // Geo schedule: per target patch ceil(|p|/128) row tiles that share the list of
 // 128-row pieces of the patch's selected source patches.  Writes the counts to
 // counts[0] (tiles) and counts[1] (segments).  Upper bounds for sizing:
@@ -93,7 +95,7 @@ int geo_max_segs(int nM, int PM, int PN, int R);
 // Offsets outside [0, n] or decreasing are clamped and set the bad-index bit.
 cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
                                 const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
-                                int* scratch, unsigned* status, cudaStream_t st);
+                                int* prefix, int* scratch, unsigned* status, cudaStream_t st);
 size_t geo_schedule_scratch_ints(int PN);
 // Transposed selection (for the key-stationary fp32 backward): for every
 // source patch q the ascending list of target patches p with q in topk[p].
@@ -148,6 +150,7 @@ struct TcArgs {
   const KeySeg* segs;
   const int* ntiles_dev;  // nullable
   int ntiles_host;
+  const int* tile_prefix;  // [ntiles + 1] prefix sums of the tiles' segment counts
   const int* row_map;
   const int* col_map;
 };

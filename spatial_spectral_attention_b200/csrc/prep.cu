@@ -124,12 +124,40 @@ __global__ void bwd_prep_kernel(const float* __restrict__ dO, int lddo, const fl
 }
 
 __global__ void dense_schedule_kernel(int nN, int nM, RowTile* __restrict__ tiles,
-                                      KeySeg* __restrict__ segs) {
+                                      KeySeg* __restrict__ segs, int* __restrict__ prefix) {
   const int nt = (nN + kTileRows - 1) / kTileRows, ns = (nM + kTileRows - 1) / kTileRows;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < max(nt, ns); i += gridDim.x * blockDim.x) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= max(nt, ns); i += gridDim.x * blockDim.x) {
     if (i < nt) tiles[i] = RowTile{i * kTileRows, min(kTileRows, nN - i * kTileRows), 0, ns};
     if (i < ns) segs[i] = KeySeg{i * kTileRows, min(kTileRows, nM - i * kTileRows)};
+    if (i <= nt) prefix[i] = i * ns;
   }
+}
+
+// prefix[t] = sum of tiles[0..t).nseg for t <= counts[0] (single block).
+__global__ void __launch_bounds__(1024) tile_prefix_kernel(const RowTile* __restrict__ tiles,
+                                                           const int* __restrict__ counts,
+                                                           int* __restrict__ prefix) {
+  __shared__ int part[1024];
+  const int m = counts[0];
+  const int tid = threadIdx.x;
+  const int per = (m + 1023) / 1024;
+  const int lo = tid * per, hi = min(m, lo + per);
+  int s = 0;
+  for (int i = lo; i < hi; ++i) s += tiles[i].nseg;
+  part[tid] = s;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int x = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += x;
+    __syncthreads();
+  }
+  int r = part[tid] - s;
+  for (int i = lo; i < hi; ++i) {
+    prefix[i] = r;
+    r += tiles[i].nseg;
+  }
+  if (tid == 1023) prefix[m] = part[1023];
 }
 
 // pieces[p] = row tiles of target patch p; nsegs[p] = 128-row pieces of its
@@ -319,9 +347,10 @@ cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, 
 int dense_num_tiles(int nN) { return (nN + kTileRows - 1) / kTileRows; }
 int dense_num_segs(int nM) { return (nM + kTileRows - 1) / kTileRows; }
 
-cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, cudaStream_t st) {
-  const int m = std::max(dense_num_tiles(nN), dense_num_segs(nM));
-  dense_schedule_kernel<<<grid_for(m, 256), 256, 0, st>>>(nN, nM, tiles, segs);
+cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, int* prefix,
+                                  cudaStream_t st) {
+  const int m = std::max(dense_num_tiles(nN), dense_num_segs(nM)) + 1;
+  dense_schedule_kernel<<<grid_for(m, 256), 256, 0, st>>>(nN, nM, tiles, segs, prefix);
   count_launch();
   return cudaGetLastError();
 }
@@ -336,7 +365,7 @@ size_t geo_schedule_scratch_ints(int PN) { return 4 * (size_t)PN + 2; }
 
 cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
                                 const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
-                                int* scratch, unsigned* status, cudaStream_t st) {
+                                int* prefix, int* scratch, unsigned* status, cudaStream_t st) {
   int* pieces = scratch;
   int* nsegs = scratch + PN;
   int* tbase = scratch + 2 * PN;
@@ -352,6 +381,8 @@ cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM
                                                     seg_cap);
   count_launch();
   clamp_counts_kernel<<<1, 1, 0, st>>>(counts, tile_cap, seg_cap);
+  count_launch();
+  tile_prefix_kernel<<<1, 1024, 0, st>>>(tiles, counts, prefix);
   count_launch();
   return cudaGetLastError();
 }

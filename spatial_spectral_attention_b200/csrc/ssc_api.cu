@@ -92,6 +92,7 @@ cudaError_t zero_matrix(float* p, int ld, int rows, int cols, cudaStream_t st) {
 struct DenseWs {
   RowTile* tiles;
   KeySeg* segs;
+  int* prefix;
   __nv_bfloat16* dOb;
   __nv_bfloat16* Vpad;  // V re-packed with a 16-byte aligned row pitch
   float* D;
@@ -102,6 +103,7 @@ size_t dense_ws(void* base, int nN, int nM, int d, int k, int dtype, DenseWs* w)
   DenseWs x;
   x.tiles = c.take<RowTile>(dense_num_tiles(nN));
   x.segs = c.take<KeySeg>(dense_num_segs(nM));
+  x.prefix = c.take<int>(dense_num_tiles(nN) + 1);
   x.dOb = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nN * kp_of(k)) : nullptr;
   x.Vpad = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nM * kp_of(k)) : nullptr;
   x.D = c.take<float>(nN);
@@ -119,6 +121,7 @@ struct GeoWs {
   RowTile* tiles;
   KeySeg* segs;
   int* counts;
+  int* prefix;
   int* sched_scratch;
   int* inv_off;
   int* inv_p;
@@ -143,6 +146,7 @@ size_t geo_ws(void* base, int nN, int nM, int d, int k, int PN, int PM, int R, i
   x.tiles = c.take<RowTile>(geo_max_tiles(nN, PN));
   x.segs = c.take<KeySeg>(geo_max_segs(nM, PM, PN, R));
   x.counts = c.take<int>(2);
+  x.prefix = c.take<int>(geo_max_tiles(nN, PN) + 1);
   x.sched_scratch = c.take<int>(geo_schedule_scratch_ints(PN));
   x.inv_off = c.take<int>(PM + 1);
   x.inv_p = c.take<int>((size_t)PN * R);
@@ -278,7 +282,7 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DenseWs w;
   dense_ws(ws, nN, nM, d, k, dtype, &w);
-  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, st);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, w.prefix, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   if (dtype == SSC_F32) {
     SimtArgs a{static_cast<const float*>(Q), static_cast<const float*>(K),
@@ -295,7 +299,7 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
                                           static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt, nN,
                                           nM, d, k, scale, O, ldo, lse, st, ctl));
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
-           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), nullptr,
+           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
   return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
 }
@@ -316,7 +320,7 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
   WaitCtl ctl = make_ctl();
   DenseWs w;
   dense_ws(ws, nN, nM, d, k, dtype, &w);
-  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, st);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, w.prefix, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   if (dtype == SSC_F32) {
     e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, nullptr, 0, nullptr, 0, w.D,
@@ -335,12 +339,13 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
                       nullptr, ctl.status, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
   const __nv_bfloat16* Vt;
   int ldvt;
   if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
-           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), nullptr,
+           ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
   return cuda_status(launch_tc_bwd(a, w.dOb, kp, lse, w.D, dQ, lddq, dK, lddk, dV, lddv, st, ctl));
 }
@@ -378,7 +383,7 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
       return SSC_ERR_CUDA;
   }
   e = launch_geo_schedule(offN, PN, nN, offM, PM, nM, topk, R, w.tiles, w.segs, w.counts,
-                          w.sched_scratch, ctl.status, st);
+                          w.prefix, w.sched_scratch, ctl.status, st);
   return cuda_status(e);
 }
 
@@ -412,7 +417,7 @@ int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const v
   }
   TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
            static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
-           w.tiles, w.segs, w.counts, 0, memN, memM};
+           w.tiles, w.segs, w.counts, 0, w.prefix, memN, memM};
   return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
 }
 
@@ -460,10 +465,11 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const v
                       w.ldg, nullptr, 0, w.D, w.lsep, ctl.status, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
            static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
-           w.tiles, w.segs, w.counts, 0, memN, memM};
+           w.tiles, w.segs, w.counts, 0, w.prefix, memN, memM};
   return cuda_status(launch_tc_bwd(a, static_cast<const __nv_bfloat16*>(w.dOp), w.ldg, w.lsep, w.D,
                                    dQ, lddq, dK, lddk, dV, lddv, st, ctl));
 }
