@@ -51,90 +51,79 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    """SM clock and clock-event (throttle) reasons, polled through NVML every
+    10 ms on a background thread (read-only queries)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event reason bits
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "sw_power_cap": 0x4,
+    }
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.stop = threading.Event()
+        self.window = (0.0, float("inf"))
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         except Exception:
-            self.proc = None
+            self.nvml = None
         return self
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+    def _run(self):
+        n = self.nvml
+        while not self.stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                try:
+                    r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), sm, r))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def mark(self, t0, t1):
+        """Restrict the summary to samples taken between wall times t0 and t1."""
+        self.window = (t0, t1)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        if self.nvml is not None:
+            self.t.join(timeout=1)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 7:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx.append(float(f[1]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
+        w0, w1 = self.window
+        sel = [s for s in self.samples if w0 <= s[0] <= w1]
+        if not sel:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = sorted({nm for _, _, r in sel for nm, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": float(np.median([s[1] for s in sel])), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(sel)}
 
 
 def dist_setup(ngpus):
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return ws, rank, local
+    from spatial_spectral_attention_b200 import dist
+    return dist.init("nccl")
 
 
 def max_over_ranks(x, ws):
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from spatial_spectral_attention_b200 import dist
+    return dist.max_over_ranks(x, ws, device="cuda")
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from spatial_spectral_attention_b200 import dist
+    dist.barrier(ws)
 
 
 # ---------------------------------------------------------------- our arm
@@ -201,6 +190,7 @@ def run_ours(args, ws, rank, local):
                                  workspace=g["ws"])
         return topk
 
+    clk = ClockSampler(local).__enter__()
     for _ in range(args.warmup):
         dense_step(Q, K, V, dO)
         if geo:
@@ -214,17 +204,20 @@ def run_ours(args, ws, rank, local):
     launches0 = api.ssc_kernel_launches()
     torch.cuda.reset_peak_memory_stats(dev)
     mem0 = torch.cuda.memory_allocated(dev)
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        for s in range(args.steps):
+    torch.cuda.synchronize()
+    w0 = time.time()
+    for s in range(args.steps):
+        flush.zero_()
+        dense_step(Q, K, V, dO, evs[s])
+        if geo:
             flush.zero_()
-            dense_step(Q, K, V, dO, evs[s])
-            if geo:
-                flush.zero_()
-                gev[s][0].record(stream)
-                geo_step()
-                gev[s][1].record(stream)
-        torch.cuda.synchronize()
+            gev[s][0].record(stream)
+            geo_step()
+            gev[s][1].record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    clk.mark(w0, w1)
+    clk.__exit__()
     launches = api.ssc_kernel_launches() - launches0
     peak_gib = (torch.cuda.max_memory_allocated(dev) - mem0 + ws_bytes) / 2**30
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -245,17 +238,25 @@ def run_ours(args, ws, rank, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(ws)
+    parts = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(e2e_steps)]
+    dev_in = {x: torch.empty_like(host[x], device=dev) for x in host}
     e0.record(stream)
-    for _ in range(e2e_steps):
-        Qd, Kd, Vd, dOd = (host[x].to(dev, non_blocking=True) for x in ("Q", "K", "V", "dO"))
-        O, lse, (dQ, dK, _) = dense_step(Qd, Kd, Vd, dOd)
+    for i in range(e2e_steps):
+        for x in ("Q", "K", "V", "dO"):
+            dev_in[x].copy_(host[x], non_blocking=True)
+        parts[i][0].record(stream)
+        O, lse, (dQ, dK, _) = dense_step(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in["dO"])
+        parts[i][1].record(stream)
         out_host["O"].copy_(O, non_blocking=True)
         out_host["lse"].copy_(lse, non_blocking=True)
         out_host["dQ"].copy_(dQ, non_blocking=True)
         out_host["dK"].copy_(dK, non_blocking=True)
+        parts[i][2].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(e2e_steps, 1), ws)
+    e2e_compute = float(np.mean([p[0].elapsed_time(p[1]) for p in parts])) if parts else 0.0
+    e2e_d2h = float(np.mean([p[1].elapsed_time(p[2]) for p in parts])) if parts else 0.0
     h2d = sum(host[x].numel() * host[x].element_size() for x in ("Q", "K", "V", "dO"))
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
 
@@ -297,7 +298,8 @@ def run_ours(args, ws, rank, local):
                      " burst bf16 (MEASURED_PEAKS.json bf16_tflops)", "traffic": None},
         "e2e": {"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h), "compute_ms": round(e2e_compute, 4),
+                "d2h_ms": round(e2e_d2h, 4)},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
@@ -401,9 +403,8 @@ def main():
                                    "sample": f"{rows} of {res['config']['n']} target rows "
                                              f"({dt:.1f} s), extrapolated to all rows"}
         print(json.dumps(res), flush=True)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    from spatial_spectral_attention_b200 import dist
+    dist.finalize(ws)
 
 
 if __name__ == "__main__":
