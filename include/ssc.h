@@ -117,6 +117,26 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex,
                     int* centers, int* owner, int* offsets, int* members,
                     void* ws, size_t ws_bytes, ssc_stream_t stream);
 
+/* The same patches without a workspace argument, for callers that cannot
+ * allocate device memory at all (for instance code embedded in a host program
+ * that owns every device allocation and hands over only input and output
+ * buffers).  The pages have no counterpart of this call; it exists for such
+ * callers only.  Results equal ssc_fps_patches bit for bit.
+ *   Limits: n <= SSC_FPS_NOALLOC_MAX_N, P <= SSC_FPS_NOALLOC_MAX_P; larger
+ *   sizes return SSC_ERR_UNSUPPORTED before any work is enqueued.
+ *   Scratch: a fixed 3 MiB array in the library's own device memory, held by
+ *   every GPU that loads the library until the process exits.  The first
+ *   call on a device looks up the array's device address (with that device
+ *   current); make that first call before capturing any stream into a graph.
+ *   Every call shares the array: calls that overlap on the GPU (different
+ *   streams or host threads) race and must be serialised by the caller; each
+ *   call clears the counters it needs zeroed.  No device allocation is made. */
+#define SSC_FPS_NOALLOC_MAX_N 262144
+#define SSC_FPS_NOALLOC_MAX_P 65535
+int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_vertex,
+                            int* centers, int* owner, int* offsets, int* members,
+                            ssc_stream_t stream);
+
 /* Scratch bytes ssc_patch_scores_topk needs. */
 size_t ssc_patch_scores_topk_workspace_size(int PN, int PM, int d);
 

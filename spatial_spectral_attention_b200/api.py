@@ -93,6 +93,23 @@ def ssc_fps_patches(pts, P, seed_vertex=0):
     return centers, owner, offsets, members
 
 
+def ssc_fps_patches_noalloc(pts, P, seed_vertex=0):
+    """ssc_fps_patches without a workspace: the library's fixed device scratch
+    is used instead (n <= 262144, P <= 65535; concurrent calls must not overlap)."""
+    _cuda(pts)
+    pts = pts.contiguous()
+    n = pts.shape[0]
+    dev = pts.device
+    centers = torch.empty(P, dtype=torch.int32, device=dev)
+    owner = torch.empty(n, dtype=torch.int32, device=dev)
+    offsets = torch.empty(P + 1, dtype=torch.int32, device=dev)
+    members = torch.empty(n, dtype=torch.int32, device=dev)
+    check("ssc_fps_patches_noalloc", lib().ssc_fps_patches_noalloc(
+        _ptr(pts), n, P, seed_vertex, _ptr(centers), _ptr(owner), _ptr(offsets), _ptr(members),
+        _stream()))
+    return centers, owner, offsets, members
+
+
 def ssc_patch_scores_topk(FN, FM, offN, memN, offM, memM, R, return_scores=False):
     """Patch-mean scores and the top-R source patches of every target patch."""
     _cuda(FN, FM, offN, memN, offM, memM)
