@@ -75,7 +75,6 @@ struct TcParams {
   int d, k, kp, qch, vf, vr;
   int nq, nk;        // rows of Q (and of the outputs O, lse, dQ) and of K/V (dK, dV)
   int vstages;       // forward V ring depth
-  int dk_t;          // backward: partial dK computed transposed (TMEM lane = d), d == 128
   float scale_log2;  // scale * log2(e)
   float scale;
   float* O;
@@ -472,6 +471,43 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
 }
 
 // ------------------------------------------------------------------ backward
+// Transpose a 4 x 4 block of float4 held by the 4 lanes of a quad (lane q holds
+// row q, float4 columns 0..3) so that lane q ends with column q of rows 0..3 in
+// v[0..3].  Two butterfly exchanges (lane distance 1, then 2), each moving half
+// of the block; every lane of the warp must take part.
+__device__ __forceinline__ float4 shfl_xor4(float4 a, int m) {
+  return make_float4(__shfl_xor_sync(0xffffffffu, a.x, m), __shfl_xor_sync(0xffffffffu, a.y, m),
+                     __shfl_xor_sync(0xffffffffu, a.z, m), __shfl_xor_sync(0xffffffffu, a.w, m));
+}
+__device__ __forceinline__ void quad_transpose4(float4 (&v)[4], int q) {
+  {
+    // distance 1: column pairs (0,1) and (2,3) swap their off-diagonal entries
+    const bool odd = (q & 1) != 0;
+    const float4 r0 = shfl_xor4(odd ? v[0] : v[1], 1);
+    const float4 r1 = shfl_xor4(odd ? v[2] : v[3], 1);
+    if (odd) {
+      v[0] = r0;
+      v[2] = r1;
+    } else {
+      v[1] = r0;
+      v[3] = r1;
+    }
+  }
+  {
+    // distance 2: 2 x 2 blocks swap across the quad's halves
+    const bool hi = (q & 2) != 0;
+    const float4 r0 = shfl_xor4(hi ? v[0] : v[2], 2);
+    const float4 r1 = shfl_xor4(hi ? v[1] : v[3], 2);
+    if (hi) {
+      v[0] = r0;
+      v[1] = r1;
+    } else {
+      v[2] = r0;
+      v[3] = r1;
+    }
+  }
+}
+
 // kDV = false: dQ (stored) and dK (atomics).  kDV = true: dV (atomics).
 // The backward's work is the flat list of (row tile, key segment) units, in
 // row-tile order; CTA c takes units [c U / G, (c + 1) U / G).  Every CTA gets
@@ -504,9 +540,20 @@ __device__ __forceinline__ bool next_segment(UnitRange& r, const RowTile* tiles,
 
 // NCG compute warpgroups split the key columns of S / dP (and the columns of
 // the dK / dV / dQ flushes); every element is independent in the backward.
-template <bool kDV, int NCG>
+//
+// QCH > 0 fixes the operand shape at compile time (d = 64 QCH; V and dO rows of
+// VF full 64-column chunks plus VR remainder columns), so that every MMA issue
+// loop has a constant trip count and is fully unrolled: a single issuing thread
+// with run-time loop bounds cannot keep the tensor pipe busy at N = 128.
+// QCH = 0 reads the shape from the parameters (any d, k).
+template <bool kDV, int NCG, int QCH, int VF, int VR>
 __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     tc_bwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr bool kFixed = QCH > 0;
+  const int qch = kFixed ? QCH : p.qch;
+  const int vf = kFixed ? VF : p.vf;
+  const int vr = kFixed ? VR : p.vr;
+  const int d16 = kFixed ? 4 * QCH : p.d / 16;
   constexpr int CW = 128 / NCG;  // key columns per compute thread
   constexpr int NC = CW / 32;
   extern __shared__ uint8_t smem_raw[];
@@ -519,8 +566,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base_u = smem_u32(smem_raw);
   const uint32_t sbase = (base_u + 1023u) & ~1023u;
-  const int qbytes = p.qch * kChunk;
-  const int vbytes = vtile_bytes(p.vf, p.vr);
+  const int qbytes = qch * kChunk;
+  const int vbytes = vtile_bytes(vf, vr);
   const uint32_t sQ = sbase;
   const uint32_t sG = sQ + qbytes;           // dO tile
   const uint32_t sK = sG + vbytes;
@@ -580,11 +627,11 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         if (tcount > 0 && !mbar_wait(&bar_qg_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         q_issued = (int)tcount;
         mbar_arrive_expect_tx(&bar_qg_full, qbytes + vbytes);
-        for (int c = 0; c < p.qch; ++c)
+        for (int c = 0; c < qch; ++c)
           tma_load_2d(gptr(sQ) + c * kChunk, &tm.q, 64 * c, tile.row0, &bar_qg_full);
-        for (int c = 0; c < p.vf; ++c)
+        for (int c = 0; c < vf; ++c)
           tma_load_2d(gptr(sG) + c * kChunk, &tm.g, 64 * c, tile.row0, &bar_qg_full);
-        if (p.vr) tma_load_2d(gptr(sG) + p.vf * kChunk, &tm.gr, 64 * p.vf, tile.row0, &bar_qg_full);
+        if (vr) tma_load_2d(gptr(sG) + vf * kChunk, &tm.gr, 64 * vf, tile.row0, &bar_qg_full);
         bool ok = true;
         for (int j = jb; j < je; ++j, ++it) {
           const KeySeg sg = p.segs[tile.seg0 + j];
@@ -594,9 +641,9 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
               break;
             }
             mbar_arrive_expect_tx(&bar_v_full, vbytes);
-            for (int c = 0; c < p.vf; ++c)
+            for (int c = 0; c < vf; ++c)
               tma_load_2d(gptr(sV) + c * kChunk, &tm.v, 64 * c, sg.key0, &bar_v_full);
-            if (p.vr) tma_load_2d(gptr(sV) + p.vf * kChunk, &tm.vr, 64 * p.vf, sg.key0, &bar_v_full);
+            if (vr) tma_load_2d(gptr(sV) + vf * kChunk, &tm.vr, 64 * vf, sg.key0, &bar_v_full);
             v_last = (int)it;
           }
           if (it >= 1 && !mbar_wait(&bar_k_empty, (it - 1) & 1, p.ctl, abort)) {
@@ -604,7 +651,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
             break;
           }
           mbar_arrive_expect_tx(&bar_k_full, qbytes);
-          for (int c = 0; c < p.qch; ++c)
+          for (int c = 0; c < qch; ++c)
             tma_load_2d(gptr(sK) + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_k_full);
           k_last = (int)it;
         }
@@ -624,11 +671,10 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t idesc_dq = make_idesc_bf16(128, p.d, 0, 1);
       const uint32_t idesc_dkp = make_idesc_bf16(128, p.d, 1, 1);
-      const uint32_t idesc_dkt = make_idesc_bf16(128, 128, 1, 1);
-      const uint32_t idesc_dv = make_idesc_bf16(128, 64 * (p.vf > 0 ? p.vf : 1), 1, 1);
-      const uint32_t idesc_dvr = make_idesc_bf16(128, p.vr > 0 ? p.vr : 16, 1, 1);
-      const uint32_t rsw = rem_swizzle(p.vr);
-      const uint32_t rrow = (uint32_t)p.vr * 2;
+      const uint32_t idesc_dv = make_idesc_bf16(128, 64 * (vf > 0 ? vf : 1), 1, 1);
+      const uint32_t idesc_dvr = make_idesc_bf16(128, vr > 0 ? vr : 16, 1, 1);
+      const uint32_t rsw = rem_swizzle(vr);
+      const uint32_t rrow = (uint32_t)vr * 2;
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       UnitRange ur{s_range[0], s_range[1], s_range[2]};
@@ -648,14 +694,17 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
             }
             tc_fence_after();
             int kk = 0;
-            for (int c = 0; c < p.vf; ++c)
+#pragma unroll
+            for (int c = 0; c < vf; ++c)
+#pragma unroll
               for (int u = 0; u < 4; ++u, ++kk) {
                 const uint32_t off = c * kChunk + u * 32;
                 mma_ss(tmem + c_dp, make_sdesc(sG + off, 16, 1024, kSw128),
                        make_sdesc(sV + off, 16, 1024, kSw128), idesc_s, kk > 0);
               }
-            for (int u = 0; u < p.vr / 16; ++u, ++kk) {
-              const uint32_t off = p.vf * kChunk + u * 32;
+#pragma unroll
+            for (int u = 0; u < vr / 16; ++u, ++kk) {
+              const uint32_t off = vf * kChunk + u * 32;
               mma_ss(tmem + c_dp, make_sdesc(sG + off, 16, 8 * rrow, rsw),
                      make_sdesc(sV + off, 16, 8 * rrow, rsw), idesc_s, kk > 0);
             }
@@ -667,7 +716,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
             break;
           }
           tc_fence_after();
-          for (int kk = 0; kk < p.d / 16; ++kk) {
+#pragma unroll
+          for (int kk = 0; kk < d16; ++kk) {
             const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
             mma_ss(tmem + c_s, make_sdesc(sQ + off, 16, 1024, kSw128),
                    make_sdesc(sK + off, 16, 1024, kSw128), idesc_s, kk > 0);
@@ -681,6 +731,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
           tc_fence_after();
           if (!kDV) {
             // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t aoff = (kk >> 2) * kChunk + (kk & 3) * 32;
               mma_ss(tmem + c_dq, make_sdesc(sS + aoff, 16, 1024, kSw128),
@@ -688,28 +739,21 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
                      (j > jb || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bar_k_empty);
-            if (p.dk_t) {
-              // dK^T partial = Q^T dS : A = Q viewed MN-major (M = d), B = dS viewed
-              // MN-major (N = keys); TMEM lane = d, so the flush is coalesced
-              for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + c_dkp, make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128),
-                       make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128), idesc_dkt, kk > 0);
-            } else {
-              // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
-              for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
-                       make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
-            }
+            // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                     make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
           } else {
             mma_commit(&bar_k_empty);
             // dVp = P^T dO : A = P viewed MN-major (M = keys), B = dO MN-major (N = k)
             for (int kk = 0; kk < 8; ++kk) {
-              if (p.vf > 0)
+              if (vf > 0)
                 mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
                        make_sdesc(sG + kk * 2048, kChunk, 1024, kSw128), idesc_dv, kk > 0);
-              if (p.vr > 0)
-                mma_ss(tmem + c_dkp + 64 * p.vf, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
-                       make_sdesc(sG + p.vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+              if (vr > 0)
+                mma_ss(tmem + c_dkp + 64 * vf, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                       make_sdesc(sG + vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
                        idesc_dvr, kk > 0);
             }
           }
@@ -793,52 +837,50 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
           break;
         }
         tc_fence_after();
-        if (!kDV && p.dk_t) {
-          // lane = d column; each warp reduction covers 128 contiguous bytes of one
-          // key row of dK.  Warpgroup wg flushes key columns [64 wg, 64 wg + 64).
-          for (int c0 = wg * (128 / NCG); c0 < (wg + 1) * (128 / NCG); c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(ta + c_dkp + c0, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int kc = c0 + i, krow = sg.key0 + kc;
-              if (kc < sg.nkeys && krow < p.nk) {
-                const int okey = p.col_map ? p.col_map[krow] : krow;
-                if (okey >= 0 && okey < p.nk)
-                  atomicAdd(p.dK + (size_t)okey * p.lddk + lrow, __uint_as_float(o[i]) * p.scale);
-              }
-            }
-          }
-          continue;
-        }
         const int krow = sg.key0 + lrow;
         int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
         if (okey >= p.nk) okey = -1;
         const bool live_key = okey >= 0;
         if (!live_key) okey = 0;
-        float* dst = kDV ? p.dV + (size_t)okey * p.lddv : p.dK + (size_t)okey * p.lddk;
+        const int ldd = kDV ? p.lddv : p.lddk;
+        float* const dbase = kDV ? p.dV : p.dK;
+        float* dst = dbase + (size_t)okey * ldd;
         const int ncols = kDV ? p.k : p.d;
         const float mul = kDV ? 1.0f : p.scale;
+        // Rows of this thread's lane quad (destination offset, liveness): the
+        // vector path below transposes each quad's 4 x 16 values so that one
+        // reduction instruction covers 64 contiguous bytes of each of 8 rows.
+        const int qbase = lane & ~3;
+        int qkey[4];
+        bool qlive[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          qkey[m] = __shfl_sync(0xffffffffu, okey, qbase + m);
+          qlive[m] = __shfl_sync(0xffffffffu, live_key ? 1 : 0, qbase + m) != 0;
+        }
         for (int cc = wg; cc < nchunk_out; cc += NCG) {
           const int c0 = 16 * cc;
           uint32_t o[16];
           tmem_ld16(ta + c_dkp + c0, o);
           tmem_ld_wait();
-          if (live_key) {
-            if (p.vec_atomics && c0 + 16 <= ncols) {
+          if (p.vec_atomics && c0 + 16 <= ncols) {
+            float4 v[4];
 #pragma unroll
-              for (int i = 0; i < 16; i += 4) {
-                float4 v = make_float4(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul,
-                                       __uint_as_float(o[i + 2]) * mul,
-                                       __uint_as_float(o[i + 3]) * mul);
-                atomicAdd(reinterpret_cast<float4*>(dst + c0 + i), v);
-              }
-            } else {
+            for (int c = 0; c < 4; ++c)
+              v[c] = make_float4(__uint_as_float(o[4 * c]) * mul, __uint_as_float(o[4 * c + 1]) * mul,
+                                 __uint_as_float(o[4 * c + 2]) * mul,
+                                 __uint_as_float(o[4 * c + 3]) * mul);
+            quad_transpose4(v, lane & 3);
+            // v[m] = columns [c0 + 4 (lane & 3), +4) of quad row m
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (c0 + i < ncols) atomicAdd(dst + c0 + i, __uint_as_float(o[i]) * mul);
-            }
+            for (int m = 0; m < 4; ++m)
+              if (qlive[m])
+                atomicAdd(reinterpret_cast<float4*>(dbase + (size_t)qkey[m] * ldd + c0 + 4 * (lane & 3)),
+                          v[m]);
+          } else if (live_key) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < ncols) atomicAdd(dst + c0 + i, __uint_as_float(o[i]) * mul);
           }
         }
       }
@@ -853,7 +895,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         if (!store_row) orow = 0;
         float* dq = p.dQ + (size_t)orow * p.lddq;
         const uint32_t ta = tmem_lane_addr(tmem, warp, c_dq);
-        for (int cc = wg; cc < p.d / 16; cc += NCG) {
+        for (int cc = wg; cc < d16; cc += NCG) {
           uint32_t o[16];
           tmem_ld16(ta + 16 * cc, o);
           tmem_ld_wait();
@@ -1061,11 +1103,14 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     return cudaErrorInvalidValue;
   const int vb = vtile_bytes(p.vf, p.vr);
   const int grid = num_sms();  // units are split evenly over every SM
+  const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
   {
     p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
-    p.dk_t = 0;  // the transposed flush measured slower on B200; kept for reference
     const int smem = 1024 + 2 * p.qch * kChunk + 2 * vb + 2 * kChunk;
-    auto kern = tc_bwd_kernel<false, kBwdComputeGroups>;
+    // d = 128 and k in (192, 208] (V rows of 3 chunks + 16 columns) run the
+    // fixed-shape instantiation; every other shape the general one
+    auto kern = fixed ? tc_bwd_kernel<false, kBwdComputeGroups, 2, 3, 16>
+                      : tc_bwd_kernel<false, kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
@@ -1074,9 +1119,9 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
   }
   if (dV) {
     p.vec_atomics = (lddv % 4 == 0) && (reinterpret_cast<uintptr_t>(dV) % 16 == 0);
-    p.dk_t = 0;
     const int smem = 1024 + 2 * p.qch * kChunk + vb + 2 * kChunk;
-    auto kern = tc_bwd_kernel<true, kBwdComputeGroups>;
+    auto kern = fixed ? tc_bwd_kernel<true, kBwdComputeGroups, 2, 3, 16>
+                      : tc_bwd_kernel<true, kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
