@@ -118,9 +118,17 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
 
 // NWG softmax warpgroups split every query row's 128 key columns: thread
 // (wg, lane row) owns columns [wg*CW, (wg+1)*CW) of the S tile, CW = 128/NWG.
-template <int NWG>
+// QCH > 0 fixes the operand shape at compile time (d = 64 QCH; V rows of VF
+// full 64-column chunks plus VR remainder columns) so the MMA issue loops are
+// fully unrolled; QCH = 0 reads the shape from the parameters.
+template <int NWG, int QCH, int VF, int VR>
 __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     tc_fwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr bool kFixed = QCH > 0;
+  const int qch = kFixed ? QCH : p.qch;
+  const int vf = kFixed ? VF : p.vf;
+  const int vr = kFixed ? VR : p.vr;
+  const int d16 = kFixed ? 4 * QCH : p.d / 16;
   constexpr int CW = 128 / NWG;  // S columns per softmax thread
   constexpr int NC = CW / 32;    // 32-column TMEM loads per thread
   constexpr int NSM = 128 * NWG; // softmax threads
@@ -139,8 +147,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   const uint32_t base_u = smem_u32(smem_raw);
   const uint32_t sbase = (base_u + 1023u) & ~1023u;
   auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
-  const int qbytes = p.qch * kChunk;
-  const int vbytes = vtile_bytes(p.vf, p.vr);
+  const int qbytes = qch * kChunk;
+  const int vbytes = vtile_bytes(vf, vr);
   const int VS = p.vstages;  // V ring depth (1 or 2); the K ring has 2 stages
   const uint32_t sQ = sbase;
   const uint32_t sK0 = sQ + qbytes;
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     tma_prefetch_desc(&tm.q);
     tma_prefetch_desc(&tm.k);
     tma_prefetch_desc(&tm.v);
-    if (p.vr) tma_prefetch_desc(&tm.vr);
+    if (vr) tma_prefetch_desc(&tm.vr);
   }
   tc_fence_before();
   __syncthreads();
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         const RowTile tile = p.tiles[t];
         if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         mbar_arrive_expect_tx(&bar_q_full, qbytes);
-        for (int c = 0; c < p.qch; ++c)
+        for (int c = 0; c < qch; ++c)
           tma_load_2d(gptr(sQ) + c * kChunk, &tm.q, 64 * c, tile.row0, &bar_q_full);
         q_issued = (int)tcount;
         bool ok = true;
@@ -204,7 +212,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           }
           mbar_arrive_expect_tx(&bar_k_full[st], qbytes);
           uint8_t* dk = gptr(sK0) + st * qbytes;
-          for (int c = 0; c < p.qch; ++c)
+          for (int c = 0; c < qch; ++c)
             tma_load_2d(dk + c * kChunk, &tm.k, 64 * c, key0, &bar_k_full[st]);
         }
         if (!ok) break;
@@ -235,9 +243,9 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           }
           mbar_arrive_expect_tx(&bar_v_full[st], vbytes);
           uint8_t* dv = gptr(sV0) + st * vbytes;
-          for (int c = 0; c < p.vf; ++c)
+          for (int c = 0; c < vf; ++c)
             tma_load_2d(dv + c * kChunk, &tm.v, 64 * c, key0, &bar_v_full[st]);
-          if (p.vr) tma_load_2d(dv + p.vf * kChunk, &tm.vr, 64 * p.vf, key0, &bar_v_full[st]);
+          if (vr) tma_load_2d(dv + vf * kChunk, &tm.vr, 64 * vf, key0, &bar_v_full[st]);
         }
         if (!ok) break;
       }
@@ -251,11 +259,11 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
-      const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (p.vf > 0 ? p.vf : 1), 0, 1);
-      const uint32_t idesc_pvr = make_idesc_bf16(128, p.vr > 0 ? p.vr : 16, 0, 1);
+      const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (vf > 0 ? vf : 1), 0, 1);
+      const uint32_t idesc_pvr = make_idesc_bf16(128, vr > 0 ? vr : 16, 0, 1);
       const uint32_t o_col = tmem + 256;
-      const uint32_t rsw = rem_swizzle(p.vr);
-      const uint32_t rrow = (uint32_t)p.vr * 2;  // bytes per row of the remainder box
+      const uint32_t rsw = rem_swizzle(vr);
+      const uint32_t rrow = (uint32_t)vr * 2;  // bytes per row of the remainder box
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       auto issue_s = [&](uint32_t g) -> bool {
@@ -264,7 +272,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         tc_fence_after();
         const uint32_t sk = sK0 + st * qbytes;
         const uint32_t d_tmem = tmem + (g & 1) * 128;
-        for (int kk = 0; kk < p.d / 16; ++kk) {
+#pragma unroll
+        for (int kk = 0; kk < d16; ++kk) {
           const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
           mma_ss(d_tmem, make_sdesc(sQ + off, 16, 1024, kSw128), make_sdesc(sk + off, 16, 1024, kSw128),
                  idesc_s, kk > 0);
@@ -293,14 +302,15 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           tc_fence_after();
           const uint32_t sv = sV0 + vst * vbytes;
           const uint32_t a_tmem = tmem + buf * 128;
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            if (p.vf > 0)
+            if (vf > 0)
               mma_ts(o_col, a_tmem + kk * 8, make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128),
                      idesc_pv, acc);
-            if (p.vr > 0)
-              mma_ts(o_col + 64 * p.vf, a_tmem + kk * 8,
-                     make_sdesc(sv + p.vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+            if (vr > 0)
+              mma_ts(o_col + 64 * vf, a_tmem + kk * 8,
+                     make_sdesc(sv + vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
                      idesc_pvr, acc);
           }
           mma_commit(&bar_v_empty[vst]);
@@ -1056,7 +1066,8 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
   if (p.vr && !make_map(&tm.vr, a.V, a.nKrows, a.k, a.ldv, p.vr, rem_sw_host(p.vr)))
     return cudaErrorInvalidValue;
   constexpr int NWG = kFwdSoftmaxGroups;
-  auto kern = tc_fwd_kernel<NWG>;
+  const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
+  auto kern = fixed ? tc_fwd_kernel<NWG, 2, 3, 16> : tc_fwd_kernel<NWG, 0, 0, 0>;
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;

@@ -73,9 +73,13 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return t[0];
 }
 
-template <int NWG>
+// D16 > 0 fixes d = 16 D16 at compile time so the S = Q K^T issue loop is fully
+// unrolled (a run-time trip count slows the single issuing thread); D16 = 0
+// takes d from the parameters.
+template <int NWG, int D16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     tc_fwd_pair_kernel(const __grid_constant__ PairMaps tm, const PairParams p) {
+  const int d16 = D16 > 0 ? D16 : p.d / 16;
   constexpr int CW = 128 / NWG;
   constexpr int NC = CW / 32;
   constexpr int NSM = 128 * NWG;
@@ -203,7 +207,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         tc_fence_after();
         const uint32_t sk = sK0 + st * kbytes;
         const uint32_t d_tmem = tmem + (g & 1) * 128;
-        for (int kk = 0; kk < p.d / 16; ++kk) {
+#pragma unroll
+        for (int kk = 0; kk < d16; ++kk) {
           const uint32_t ch = kk >> 2, w = (kk & 3) * 32;
           mma_ss_pair(d_tmem, make_sdesc(sQ + ch * kChunk + w, 16, 1024, kSw128),
                       make_sdesc(sk + ch * kHalfChunk + w, 16, 1024, kSw128), idesc_s, kk > 0);
@@ -456,7 +461,7 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   if (!map2(&tm.q, Q, nN, d, ldq, 64, 128) || !map2(&tm.k, K, nM, d, ldk, 64, 64) ||
       !map2(&tm.v, V, nM, k, ldv, 64, 128))
     return cudaErrorInvalidValue;
-  auto kern = tc_fwd_pair_kernel<kNWG>;
+  auto kern = d == 128 ? tc_fwd_pair_kernel<kNWG, 8> : tc_fwd_pair_kernel<kNWG, 0>;
   const int smem = 1024 + p.qch * kChunk + kKS * p.qch * kHalfChunk + kVS * p.vbox * kChunk;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
