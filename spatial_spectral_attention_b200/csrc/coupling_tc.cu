@@ -557,7 +557,7 @@ __device__ __forceinline__ bool next_segment(UnitRange& r, const RowTile* tiles,
 // with run-time loop bounds cannot keep the tensor pipe busy at N = 128.
 // QCH = 0 reads the shape from the parameters (any d, k).
 template <bool kDV, int NCG, int QCH, int VF, int VR>
-__global__ void __launch_bounds__(64 + 128 * NCG, 1)
+__global__ void __launch_bounds__(64 + 128 * NCG + 128, 1)
     tc_bwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
   constexpr bool kFixed = QCH > 0;
   const int qch = kFixed ? QCH : p.qch;
@@ -568,7 +568,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
   constexpr int NC = CW / 32;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_qg_full, bar_qg_empty, bar_k_full, bar_k_empty, bar_v_full, bar_v_empty,
-      bar_sdp_full, bar_ds_full, bar_dkp_full, bar_dq_full, bar_drain;
+      bar_sdp_full, bar_ds_full, bar_dkp_full, bar_dkp_empty, bar_dq_full, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_range[3];  // first tile, first segment in it, number of units
@@ -596,6 +596,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     mbar_init(&bar_sdp_full, 1);
     mbar_init(&bar_ds_full, 128 * NCG);
     mbar_init(&bar_dkp_full, 1);
+    mbar_init(&bar_dkp_empty, 128);
     mbar_init(&bar_dq_full, 1);
     mbar_init(&bar_drain, 1);
     s_abort = 0;
@@ -749,6 +750,12 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
                      (j > jb || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bar_k_empty);
+            // the flush warpgroup has read the previous partial out of TMEM
+            if (it >= 1 && !mbar_wait(&bar_dkp_empty, (it - 1) & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -756,6 +763,12 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
                      make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
           } else {
             mma_commit(&bar_k_empty);
+            // the flush warpgroup has read the previous partial out of TMEM
+            if (it >= 1 && !mbar_wait(&bar_dkp_empty, (it - 1) & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             // dVp = P^T dO : A = P viewed MN-major (M = keys), B = dO MN-major (N = k)
             for (int kk = 0; kk < 8; ++kk) {
               if (vf > 0)
@@ -778,15 +791,13 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       volatile int never = 0;
       mbar_wait(&bar_drain, 0, p.ctl, &never);
     }
-  } else {
-    // ---------------- compute (NCG warpgroups): one thread per query row for
-    // S/dP, one thread per key row for the dK / dV flush.
+  } else if (warp < 2 + 4 * NCG) {
+    // ---------------- softmax (NCG warpgroups): one thread per query row; the
+    // warpgroups split the key columns of S / dP.  They also store dQ.
     const int wg = (warp - 2) >> 2;
     const int lrow = 32 * (warp & 3) + lane;
     const int col0 = wg * CW;
     uint32_t it = 0, tcount = 0;
-    const int kt_out = kDV ? p.kp : p.d;  // columns of the partial to flush
-    const int nchunk_out = kt_out / 16;
     UnitRange ur{s_range[0], s_range[1], s_range[2]};
     int t, jb, je;
     for (; next_segment(ur, p.tiles, ntiles, t, jb, je); ++tcount) {
@@ -800,6 +811,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       for (int j = jb; j < je; ++j, ++it) {
         const KeySeg sg = sg_next;
         if (j + 1 < je) sg_next = p.segs[tile.seg0 + j + 1];
+        // S / dP of this key tile; the commit behind it also covers the MMAs of
+        // the previous tile that read the dS tile overwritten below
         if (!mbar_wait(&bar_sdp_full, it & 1, p.ctl, abort)) {
           ok = false;
           break;
@@ -840,59 +853,6 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar_ds_full);
-        // flush the partial dK (or dV) of this key tile: thread = key row,
-        // 16-column chunks split among the warpgroups
-        if (!mbar_wait(&bar_dkp_full, it & 1, p.ctl, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int krow = sg.key0 + lrow;
-        int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
-        if (okey >= p.nk) okey = -1;
-        const bool live_key = okey >= 0;
-        if (!live_key) okey = 0;
-        const int ldd = kDV ? p.lddv : p.lddk;
-        float* const dbase = kDV ? p.dV : p.dK;
-        float* dst = dbase + (size_t)okey * ldd;
-        const int ncols = kDV ? p.k : p.d;
-        const float mul = kDV ? 1.0f : p.scale;
-        // Rows of this thread's lane quad (destination offset, liveness): the
-        // vector path below transposes each quad's 4 x 16 values so that one
-        // reduction instruction covers 64 contiguous bytes of each of 8 rows.
-        const int qbase = lane & ~3;
-        int qkey[4];
-        bool qlive[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          qkey[m] = __shfl_sync(0xffffffffu, okey, qbase + m);
-          qlive[m] = __shfl_sync(0xffffffffu, live_key ? 1 : 0, qbase + m) != 0;
-        }
-        for (int cc = wg; cc < nchunk_out; cc += NCG) {
-          const int c0 = 16 * cc;
-          uint32_t o[16];
-          tmem_ld16(ta + c_dkp + c0, o);
-          tmem_ld_wait();
-          if (p.vec_atomics && c0 + 16 <= ncols) {
-            float4 v[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              v[c] = make_float4(__uint_as_float(o[4 * c]) * mul, __uint_as_float(o[4 * c + 1]) * mul,
-                                 __uint_as_float(o[4 * c + 2]) * mul,
-                                 __uint_as_float(o[4 * c + 3]) * mul);
-            quad_transpose4(v, lane & 3);
-            // v[m] = columns [c0 + 4 (lane & 3), +4) of quad row m
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-              if (qlive[m])
-                atomicAdd(reinterpret_cast<float4*>(dbase + (size_t)qkey[m] * ldd + c0 + 4 * (lane & 3)),
-                          v[m]);
-          } else if (live_key) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (c0 + i < ncols) atomicAdd(dst + c0 + i, __uint_as_float(o[i]) * mul);
-          }
-        }
       }
       if (!ok) break;
       if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
@@ -932,6 +892,89 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) dq[16 * cc + i] = __uint_as_float(o[i]) * p.scale;
+          }
+        }
+      }
+    }
+  } else {
+    // ---------------- flush (one warpgroup): thread = key row of the partial
+    // dK (or dV) in TMEM; reduces it into global memory while the softmax
+    // warpgroups and the tensor cores work on the next key tile.
+    const int lrow = 32 * (warp & 3) + lane;
+    const int kt_out = kDV ? p.kp : p.d;  // columns of the partial
+    const int nchunk_out = kt_out / 16;
+    const int ldd = kDV ? p.lddv : p.lddk;
+    float* const dbase = kDV ? p.dV : p.dK;
+    const int ncols = kDV ? p.k : p.d;
+    const float mul = kDV ? 1.0f : p.scale;
+    const int qbase = lane & ~3;
+    uint32_t it = 0;
+    bool ok = true;
+    UnitRange ur{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+      const RowTile tile = p.tiles[t];
+      for (int j = jb; j < je; ++j, ++it) {
+        const KeySeg sg = p.segs[tile.seg0 + j];
+        const int krow = sg.key0 + lrow;
+        int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
+        if (okey >= p.nk) okey = -1;
+        const bool live_key = okey >= 0;
+        if (!live_key) okey = 0;
+        float* dst = dbase + (size_t)okey * ldd;
+        // Rows of this thread's lane quad (destination row, liveness): the
+        // vector path transposes each quad's 4 x 16 values so that one
+        // reduction instruction covers 64 contiguous bytes of each of 8 rows.
+        int qkey[4];
+        bool qlive[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          qkey[m] = __shfl_sync(0xffffffffu, okey, qbase + m);
+          qlive[m] = __shfl_sync(0xffffffffu, live_key ? 1 : 0, qbase + m) != 0;
+        }
+        if (!mbar_wait(&bar_dkp_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem_lane_addr(tmem, warp, c_dkp);
+        // four 16-column chunks per TMEM round trip; the partial's columns are
+        // released to the MMA issuer as soon as the last load has landed
+        for (int g0 = 0; g0 < nchunk_out; g0 += 4) {
+          uint32_t o[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (g0 + q < nchunk_out) tmem_ld16(ta + 16 * (g0 + q), o[q]);
+          tmem_ld_wait();
+          if (g0 + 4 >= nchunk_out) {
+            tc_fence_before();
+            mbar_arrive(&bar_dkp_empty);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c0 = 16 * (g0 + q);
+            if (g0 + q >= nchunk_out) break;
+            if (p.vec_atomics && c0 + 16 <= ncols) {
+              float4 v[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                v[c] = make_float4(__uint_as_float(o[q][4 * c]) * mul,
+                                   __uint_as_float(o[q][4 * c + 1]) * mul,
+                                   __uint_as_float(o[q][4 * c + 2]) * mul,
+                                   __uint_as_float(o[q][4 * c + 3]) * mul);
+              quad_transpose4(v, lane & 3);
+              // v[m] = columns [c0 + 4 (lane & 3), +4) of quad row m
+#pragma unroll
+              for (int m = 0; m < 4; ++m)
+                if (qlive[m])
+                  atomicAdd(reinterpret_cast<float4*>(dbase + (size_t)qkey[m] * ldd + c0 +
+                                                      4 * (lane & 3)),
+                            v[m]);
+            } else if (live_key) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (c0 + i < ncols) atomicAdd(dst + c0 + i, __uint_as_float(o[q][i]) * mul);
+            }
           }
         }
       }
@@ -1124,7 +1167,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                       : tc_bwd_kernel<false, kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
+    kern<<<grid, 64 + 128 * kBwdComputeGroups + 128, smem, st>>>(tm, p);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1135,7 +1178,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                       : tc_bwd_kernel<true, kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 64 + 128 * kBwdComputeGroups, smem, st>>>(tm, p);
+    kern<<<grid, 64 + 128 * kBwdComputeGroups + 128, smem, st>>>(tm, p);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
