@@ -62,6 +62,7 @@ struct TensorMaps {
   CUtensorMap vr;    // box {vr, 128}, SW32/SW64 (remainder columns of V)
   CUtensorMap g;     // dO: box {64, 128}, SW128
   CUtensorMap gr;    // dO remainder
+  CUtensorMap dk;    // dK fp32 [nk, d]: box {32, 128}, SW128 (TMA reductions of the partials)
 };
 
 struct TcParams {
@@ -89,8 +90,11 @@ struct TcParams {
   int lddk;
   float* dV;
   int lddv;
+  const __nv_bfloat16* dOb;  // bf16 dO rows of kp columns (zero padded), row order of Q
+  int lddob;
   int vec_atomics;
   int vec_atomics_dq;
+  int dk_tma;  // partial dK reduced by TMA through tm.dk (key rows contiguous, no column map)
   WaitCtl ctl;
 };
 
@@ -989,6 +993,525 @@ __global__ void __launch_bounds__(64 + 128 * NCG + 128, 1)
   }
 }
 
+// ------------------------------------------------------------------ backward, dQ and dK
+// Query-stationary backward for dQ and dK (the dV pass keeps tc_bwd_kernel).
+// 128 (2 + NCG) threads in four warpgroups:
+//   WG0   warp 0: TMA producer (Q once per row tile; K_j into a 2-stage ring;
+//         V_j); warp 1: MMA issuer and TMEM owner; warps 2-3 idle.
+//   WG1.. (NCG softmax warpgroups): thread = query row (TMEM lane); the
+//         warpgroups split the key columns.  They write the row tile's dO into
+//         TMEM once and store dQ at the end of the row tile.
+//   last  (flush): thread = key row; reduces every key tile's partial dK into
+//         global memory while the other roles move on.
+// TMEM columns: [0,128) S_j and then dP_j of the same key tile (dP is issued
+// once the softmax has read S, so its MMAs run under the softmax's exp2);
+// [128, 128 + kp/2) dO as bf16 pairs, the A operand of dP; [256, 256 + d) dQ;
+// [384, 384 + d) the partial dK.  Per key tile j:
+//   S_j  = Q K_j^T      (SS)                -> softmax: P = exp2(S s log2e - lse log2e)
+//   dP_j = dO V_j^T     (TS, A = dO)        -> softmax: dS = P (dP - D) -> bf16 smem
+//   dQ  += dS K_j       (SS, K_j MN-major)
+//   dKp  = dS^T Q       (SS, MN-major views) -> flush warpgroup -> dK
+// Shared memory: Q, two K stages, V, dS (no dO tile), which leaves room for
+// the second K stage; a key tile's K load overlaps the previous tile's work.
+template <int NCG, int QCH, int VF, int VR>
+__global__ void __launch_bounds__(128 * (2 + NCG), 1)
+    tc_bwd_dqk_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  static_assert(NCG == 2, "the register split assumes two softmax warpgroups");
+  constexpr bool kFixed = QCH > 0;
+  const int qch = kFixed ? QCH : p.qch;
+  const int vf = kFixed ? VF : p.vf;
+  const int vr = kFixed ? VR : p.vr;
+  const int d16 = kFixed ? 4 * QCH : p.d / 16;
+  constexpr int CW = 128 / NCG;  // key columns per softmax thread
+  constexpr int NC = CW / 32;
+  constexpr int kFlushWarp = 4 + 4 * NCG;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full,
+      bar_v_empty, bar_s_full, bar_s_read, bar_dp_full, bar_ds_full, bar_do_full, bar_dkp_full,
+      bar_dkp_empty, bar_dq_full, bar_drain, bar_stage_full[2], bar_stage_free[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_range[3];  // first tile, first segment in it, number of units
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  const int qbytes = qch * kChunk;
+  const int vbytes = vtile_bytes(vf, vr);
+  const uint32_t sQ = sbase;
+  const uint32_t sK0 = sQ + qbytes;  // K stage s at sK0 + s * qbytes
+  const uint32_t sV = sK0 + 2 * qbytes;
+  const uint32_t sS = sV + vbytes;   // dS tile [q][keys], 2 chunks
+  const uint32_t sStage = sS + 2 * kChunk;  // two 16 KB staging boxes of the dK partial (TMA path)
+  auto gptr = [&](uint32_t s) { return smem_raw + (s - base_u); };
+  const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_k_full[i], 1);
+      mbar_init(&bar_k_empty[i], 1);
+    }
+    mbar_init(&bar_v_full, 1);
+    mbar_init(&bar_v_empty, 1);
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_s_read, 128 * NCG);
+    mbar_init(&bar_dp_full, 1);
+    mbar_init(&bar_ds_full, 128 * NCG);
+    mbar_init(&bar_do_full, 128 * NCG);
+    mbar_init(&bar_dkp_full, 1);
+    mbar_init(&bar_dkp_empty, 128);
+    mbar_init(&bar_dq_full, 1);
+    mbar_init(&bar_drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_stage_full[i], 128);
+      mbar_init(&bar_stage_free[i], 1);
+    }
+    s_abort = 0;
+    fence_barrier_init();
+    // this CTA's share of the (row tile, key segment) units
+    const int U = p.tile_prefix[ntiles];
+    const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+    const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+    int lo = 0, hi = ntiles;  // largest t < ntiles with prefix[t] <= u0
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.tile_prefix[mid] <= u0) lo = mid;
+      else hi = mid;
+    }
+    s_range[0] = lo;
+    s_range[1] = ntiles > 0 ? (int)(u0 - p.tile_prefix[lo]) : 0;
+    s_range[2] = ntiles > 0 ? (int)(u1 - u0) : 0;
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+  const uint32_t c_sp = 0, c_do = 128, c_dq = 256, c_dkp = 384;
+
+  if (warp < 4) {
+    warpgroup_reg_dealloc<80>();
+    if (warp == 0 && lane == 0) {
+      // ---------------- TMA producer
+      uint32_t it = 0, tcount = 0;
+      int q_last = -1, v_last = -1;
+      int k_last[2] = {-1, -1};  // phase index of the last load issued per K stage
+      UnitRange ur{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (!*abort && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+        const RowTile tile = p.tiles[t];
+        if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        mbar_arrive_expect_tx(&bar_q_full, qbytes);
+        for (int c = 0; c < qch; ++c)
+          tma_load_2d(gptr(sQ) + c * kChunk, &tm.q, 64 * c, tile.row0, &bar_q_full);
+        q_last = (int)tcount;
+        bool ok = true;
+        for (int j = jb; j < je; ++j, ++it) {
+          const KeySeg sg = p.segs[tile.seg0 + j];
+          const int st = it & 1;
+          if (it >= 2 && !mbar_wait(&bar_k_empty[st], ((it >> 1) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_k_full[st], qbytes);
+          for (int c = 0; c < qch; ++c)
+            tma_load_2d(gptr(sK0 + st * qbytes) + c * kChunk, &tm.k, 64 * c, sg.key0, &bar_k_full[st]);
+          k_last[st] = (int)(it >> 1);
+          if (it >= 1 && !mbar_wait(&bar_v_empty, (it - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_v_full, vbytes);
+          for (int c = 0; c < vf; ++c)
+            tma_load_2d(gptr(sV) + c * kChunk, &tm.v, 64 * c, sg.key0, &bar_v_full);
+          if (vr) tma_load_2d(gptr(sV) + vf * kChunk, &tm.vr, 64 * vf, sg.key0, &bar_v_full);
+          v_last = (int)it;
+        }
+        ++tcount;
+        if (!ok) break;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        if (q_last >= 0) mbar_wait(&bar_q_full, q_last & 1, p.ctl, &never);
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (k_last[s2] >= 0) mbar_wait(&bar_k_full[s2], k_last[s2] & 1, p.ctl, &never);
+        if (v_last >= 0) mbar_wait(&bar_v_full, v_last & 1, p.ctl, &never);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---------------- MMA issuer
+      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);  // S and dP: N = 128 keys
+      const uint32_t idesc_dq = make_idesc_bf16(128, p.d, 0, 1);
+      const uint32_t idesc_dkp = make_idesc_bf16(128, p.d, 1, 1);
+      const uint32_t rsw = rem_swizzle(vr);
+      const uint32_t rrow = (uint32_t)vr * 2;
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      UnitRange ur{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+        if (!mbar_wait(&bar_q_full, tcount & 1, p.ctl, abort) ||
+            !mbar_wait(&bar_do_full, tcount & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // S = Q K_j^T into the S/dP columns (K stage it & 1)
+        auto issue_s = [&](uint32_t u) -> bool {
+          const uint32_t sK = sK0 + (u & 1) * qbytes;
+          if (!mbar_wait(&bar_k_full[u & 1], (u >> 1) & 1, p.ctl, abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < d16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + c_sp, make_sdesc(sQ + off, 16, 1024, kSw128),
+                   make_sdesc(sK + off, 16, 1024, kSw128), idesc_s, kk > 0);
+          }
+          mma_commit(&bar_s_full);
+          return true;
+        };
+        ok = issue_s(it);
+        // Per key tile the tensor pipe runs dP_j, S_{j+1}, dQ_j, dKp_j: the next
+        // tile's S is computed while the softmax finishes dS_j, and the softmax
+        // works on S_{j+1} while dQ_j and dKp_j run.  dP_{j+1} is committed after
+        // dKp_j, so its barrier also tells the softmax that dS_j has been consumed.
+        for (int j = jb; j < je && ok; ++j, ++it) {
+          const int st = it & 1;
+          const uint32_t sK = sK0 + st * qbytes;
+          // dP = dO V^T into the same columns, once the softmax has read S
+          if (!mbar_wait(&bar_s_read, it & 1, p.ctl, abort) ||
+              !mbar_wait(&bar_v_full, it & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          {
+            int kk = 0;
+#pragma unroll
+            for (int c = 0; c < vf; ++c)
+#pragma unroll
+              for (int u = 0; u < 4; ++u, ++kk)
+                mma_ts(tmem + c_sp, tmem + c_do + 8 * kk,
+                       make_sdesc(sV + c * kChunk + u * 32, 16, 1024, kSw128), idesc_s, kk > 0);
+#pragma unroll
+            for (int u = 0; u < vr / 16; ++u, ++kk)
+              mma_ts(tmem + c_sp, tmem + c_do + 8 * kk,
+                     make_sdesc(sV + vf * kChunk + u * 32, 16, 8 * rrow, rsw), idesc_s, kk > 0);
+          }
+          mma_commit(&bar_v_empty);
+          mma_commit(&bar_dp_full);
+          // dS in shared memory (the softmax has read dP: the columns are free)
+          if (!mbar_wait(&bar_ds_full, it & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (j + 1 < je && !issue_s(it + 1)) {
+            ok = false;
+            break;
+          }
+          // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(tmem + c_dq, make_sdesc(sS + aoff, 16, 1024, kSw128),
+                   make_sdesc(sK + kk * 2048, kChunk, 1024, kSw128), idesc_dq,
+                   (j > jb || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar_k_empty[st]);
+          // the flush warpgroup has read the previous partial out of TMEM
+          if (it >= 1 && !mbar_wait(&bar_dkp_empty, (it - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                   make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
+          mma_commit(&bar_dkp_full);
+        }
+        if (!ok) break;
+        mma_commit(&bar_dq_full);
+        mma_commit(&bar_q_empty);
+        ++tcount;
+      }
+      mma_commit(&bar_drain);
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
+    }
+  } else if (warp < kFlushWarp) {
+    // ---------------- softmax (NCG warpgroups): thread = query row
+    warpgroup_reg_alloc<128>();
+    const int wg = (warp - 4) >> 2;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int col0 = wg * CW;
+    const int kp16 = p.kp / 16;  // 8-column TMEM pieces of the dO row
+    uint32_t it = 0, tcount = 0;
+    UnitRange ur{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    for (; next_segment(ur, p.tiles, ntiles, t, jb, je); ++tcount) {
+      const RowTile tile = p.tiles[t];
+      const int qrow = tile.row0 + lrow;
+      const bool live_row = lrow < tile.nrows && qrow < p.nq;
+      const float lse2 = live_row ? p.lse_in[qrow] * kLog2e : 0.f;
+      const float Di = live_row ? p.Dvec[qrow] : 0.f;
+      // this row tile's dO row into TMEM (the previous row tile's MMAs are
+      // complete: its dQ was waited for below before getting here)
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.dOb + (size_t)(live_row ? qrow : 0) * p.lddob);
+        const uint32_t da = tmem_lane_addr(tmem, warp, c_do);
+        for (int pc = wg; pc < kp16; pc += NCG) {
+          uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+          if (live_row) {
+            a = src[2 * pc];
+            b = src[2 * pc + 1];
+          }
+          const uint32_t r[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          tmem_st8(da + 8 * pc, r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_do_full);
+      }
+      bool ok = true;
+      KeySeg sg_next = p.segs[tile.seg0 + jb];
+      for (int j = jb; j < je; ++j, ++it) {
+        const KeySeg sg = sg_next;
+        if (j + 1 < je) sg_next = p.segs[tile.seg0 + j + 1];
+        if (!mbar_wait(&bar_s_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem_lane_addr(tmem, warp, c_sp + col0);
+        uint32_t sv[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(ta + 32 * c, sv[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_s_read);  // the S columns may now receive dP
+        // P = exp2(S s log2e - lse log2e); keys past the segment and dead rows -> 0
+        float pr[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const int cbase = col0 + 32 * c;
+          const bool full = live_row && cbase + 32 <= sg.nkeys;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float v = ex2_approx(fmaf(__uint_as_float(sv[c][i]), p.scale_log2, -lse2));
+            if (!full && (cbase + i >= sg.nkeys || !live_row)) v = 0.f;
+            pr[c][i] = v;
+          }
+        }
+        // dP of this key tile; its commit also covers the MMAs of the previous
+        // key tile that read the dS tile overwritten below
+        if (!mbar_wait(&bar_dp_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(ta + 32 * c, dp);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(pr[c][2 * i] * (__uint_as_float(dp[2 * i]) - Di),
+                                pr[c][2 * i + 1] * (__uint_as_float(dp[2 * i + 1]) - Di));
+          // row lrow, keys [cbase, cbase+32): 64-key chunk cbase/64, 16-byte
+          // units ((cbase%64)/8) + 0..3, swizzled by the row
+          const int cbase = col0 + 32 * c;
+          const uint32_t rowb = sS + (cbase >> 6) * kChunk + lrow * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t unit = (((cbase & 63) >> 3) + u) ^ (lrow & 7);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(rowb + unit * 16),
+                         "r"(pk[4 * u]), "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar_ds_full);
+      }
+      if (!ok) break;
+      if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      // TMEM loads are warp-collective: every lane loads, live rows store
+      int orow = live_row ? (p.row_map ? p.row_map[qrow] : qrow) : -1;
+      const bool store_row = orow >= 0 && orow < p.nq;
+      const bool whole = jb == 0 && je == tile.nseg;  // all of the row tile's keys done here
+      if (!store_row) orow = 0;
+      float* dq = p.dQ + (size_t)orow * p.lddq;
+      const uint32_t qa = tmem_lane_addr(tmem, warp, c_dq);
+      for (int cc = wg; cc < d16; cc += NCG) {
+        uint32_t o[16];
+        tmem_ld16(qa + 16 * cc, o);
+        tmem_ld_wait();
+        if (!store_row) continue;
+        if (!whole) {
+          // the row tile's keys are split over several CTAs: reduce into dQ
+          if (p.vec_atomics_dq) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              atomicAdd(reinterpret_cast<float4*>(dq + 16 * cc + i),
+                        make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                    __uint_as_float(o[i + 2]) * p.scale,
+                                    __uint_as_float(o[i + 3]) * p.scale));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) atomicAdd(dq + 16 * cc + i, __uint_as_float(o[i]) * p.scale);
+          }
+        } else if ((p.lddq & 3) == 0) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dq + 16 * cc + i) = make_float4(
+                __uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) dq[16 * cc + i] = __uint_as_float(o[i]) * p.scale;
+        }
+      }
+    }
+  } else {
+    // ---------------- flush (one warpgroup): thread = key row of the partial dK
+    warpgroup_reg_alloc<176>();
+    const int lrow = 32 * (warp & 3) + lane;
+    const int qbase = lane & ~3;
+    const bool issuer = lrow == 0;  // issues the TMA reductions
+    uint32_t it = 0, blk = 0;
+    bool ok = true;
+    UnitRange ur{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+      const RowTile tile = p.tiles[t];
+      for (int j = jb; j < je; ++j, ++it) {
+        const KeySeg sg = p.segs[tile.seg0 + j];
+        const int krow = sg.key0 + lrow;
+        int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
+        if (okey >= p.nk) okey = -1;
+        const bool live_key = okey >= 0;
+        if (!live_key) okey = 0;
+        float* dst = p.dK + (size_t)okey * p.lddk;
+        // rows of this thread's lane quad (destination row, liveness): each
+        // quad transposes its 4 x 16 values so that one reduction covers 64
+        // contiguous bytes of each of 8 rows
+        int qkey[4] = {0, 0, 0, 0};
+        bool qlive[4] = {false, false, false, false};
+        if (!p.dk_tma) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            qkey[m] = __shfl_sync(0xffffffffu, okey, qbase + m);
+            qlive[m] = __shfl_sync(0xffffffffu, live_key ? 1 : 0, qbase + m) != 0;
+          }
+        }
+        if (!mbar_wait(&bar_dkp_full, it & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem_lane_addr(tmem, warp, c_dkp);
+        // the whole partial (d <= 128 columns) in one TMEM round trip, then the
+        // columns go back to the MMA issuer before the reductions start
+        uint32_t o[8][16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < d16) tmem_ld16(ta + 16 * q, o[q]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_dkp_empty);
+        if (p.dk_tma) {
+          // 32-column blocks: every thread writes its key row (8 units of 16 B,
+          // unit u at u ^ (row & 7), the tensor map's 128-byte swizzle), then one
+          // thread hands the block to the TMA unit, which adds it into dK
+#pragma unroll
+          for (int bq = 0; bq < 4; ++bq) {
+            if (2 * bq >= d16) break;
+            const int sb = blk & 1;
+            const uint32_t sbuf = sStage + sb * kChunk;
+            if (blk >= 2 && !mbar_wait(&bar_stage_free[sb], ((blk >> 1) - 1) & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const uint32_t* src = &o[2 * bq + (u >> 2)][4 * (u & 3)];
+              asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(
+                               sbuf + lrow * 128 + ((u ^ (lrow & 7)) << 4)),
+                           "r"(__float_as_uint(__uint_as_float(src[0]) * p.scale)),
+                           "r"(__float_as_uint(__uint_as_float(src[1]) * p.scale)),
+                           "r"(__float_as_uint(__uint_as_float(src[2]) * p.scale)),
+                           "r"(__float_as_uint(__uint_as_float(src[3]) * p.scale))
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar_stage_full[sb]);
+            if (issuer) {
+              if (!mbar_wait(&bar_stage_full[sb], (blk >> 1) & 1, p.ctl, abort)) {
+                ok = false;
+                break;
+              }
+              tma_reduce_add_2d(&tm.dk, 32 * bq, sg.key0, gptr(sbuf));
+              bulk_commit_group();
+              if (blk >= 1) {
+                // the previous block has been read out of shared memory
+                bulk_wait_group_read<1>();
+                mbar_arrive(&bar_stage_free[(blk - 1) & 1]);
+              }
+            }
+            ++blk;
+          }
+          continue;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q >= d16) break;
+          const int c0 = 16 * q;
+          if (p.vec_atomics) {
+            float4 v[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              v[c] = make_float4(__uint_as_float(o[q][4 * c]) * p.scale,
+                                 __uint_as_float(o[q][4 * c + 1]) * p.scale,
+                                 __uint_as_float(o[q][4 * c + 2]) * p.scale,
+                                 __uint_as_float(o[q][4 * c + 3]) * p.scale);
+            quad_transpose4(v, lane & 3);
+            // v[m] = columns [c0 + 4 (lane & 3), +4) of quad row m
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+              if (qlive[m])
+                atomicAdd(reinterpret_cast<float4*>(p.dK + (size_t)qkey[m] * p.lddk + c0 + 4 * (lane & 3)),
+                          v[m]);
+          } else if (live_key) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) atomicAdd(dst + c0 + i, __uint_as_float(o[q][i]) * p.scale);
+          }
+        }
+      }
+    }
+    // the reductions still in flight must finish before the CTA exits
+    if (issuer && p.dk_tma) bulk_wait_group_all();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 __global__ void wait_probe_kernel(WaitCtl ctl) {
   __shared__ uint64_t bar;
   __shared__ int s_abort;
@@ -1031,6 +1554,21 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int b
   cuuint32_t box[2] = {(cuuint32_t)box_cols, 128};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 tensor [rows, cols] with leading dimension ld (elements), box
+// {box_cols, 128}; elements outside the tensor are skipped by reductions.
+bool make_map_f32(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_cols,
+                  CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1158,16 +1696,21 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
   const int vb = vtile_bytes(p.vf, p.vr);
   const int grid = num_sms();  // units are split evenly over every SM
   const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
+  p.dOb = dOb;
+  p.lddob = lddob;
   {
+    // dQ and dK: dO lives in TMEM, K is double-buffered, a warpgroup of its own
+    // reduces the dK partials
     p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
-    const int smem = 1024 + 2 * p.qch * kChunk + 2 * vb + 2 * kChunk;
-    // d = 128 and k in (192, 208] (V rows of 3 chunks + 16 columns) run the
-    // fixed-shape instantiation; every other shape the general one
-    auto kern = fixed ? tc_bwd_kernel<false, kBwdComputeGroups, 2, 3, 16>
-                      : tc_bwd_kernel<false, kBwdComputeGroups, 0, 0, 0>;
+    // key rows contiguous in dK (no column map): partials go through TMA reductions
+    p.dk_tma = !a.col_map && p.vec_atomics &&
+               make_map_f32(&tm.dk, dK, a.nKrows, a.d, lddk, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
+    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16>
+                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 64 + 128 * kBwdComputeGroups + 128, smem, st>>>(tm, p);
+    kern<<<grid, 128 * (2 + kBwdComputeGroups), smem, st>>>(tm, p);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
