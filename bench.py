@@ -206,16 +206,24 @@ def run_ours(args, ws, rank, local):
     mem0 = torch.cuda.memory_allocated(dev)
     torch.cuda.synchronize()
     w0 = time.time()
+    # launch durations of the dense step's kernels (CUDA events the library
+    # records on the launching stream; paused around the Geo step)
+    api.ssc_profile_enable(True)
     for s in range(args.steps):
         flush.zero_()
         dense_step(Q, K, V, dO, evs[s])
         if geo:
+            api.ssc_profile_enable(False)
             flush.zero_()
             gev[s][0].record(stream)
             geo_step()
             gev[s][1].record(stream)
+            api.ssc_profile_enable(True, clear=False)
+    api.ssc_profile_enable(False)
     torch.cuda.synchronize()
     w1 = time.time()
+    kbwd_ms, kbwd_n = api.ssc_profile_read(api.PROF_BWD_DQK)
+    kfwd_ms, kfwd_n = api.ssc_profile_read(api.PROF_DENSE_FWD)
     clk.mark(w0, w1)
     clk.__exit__()
     launches = api.ssc_kernel_launches() - launches0
@@ -262,11 +270,14 @@ def run_ours(args, ws, rank, local):
 
     pk = peaks()
     tflops = ws * flops_step / (dense_ms * 1e-3) / 1e12
-    # dominant kernel: the backward (2/3 of the flops); its window also holds the
-    # small prep kernels, so the achieved rate is a slight underestimate
+    # dominant kernel: the dQ/dK backward kernel (2/3 of the flops), its average
+    # launch duration from the events around each launch; flops per launch =
+    # executed flops per (i, j) pair x the n^2 pairs one launch processes
     bwd_flops = float(n) * n * bpp
     bwd_mean = float(np.mean(bwd_ms))
-    achieved = bwd_flops / (bwd_mean * 1e-3) / 1e12
+    kbwd_mean = kbwd_ms / max(kbwd_n, 1)
+    achieved = bwd_flops / (kbwd_mean * 1e-3) / 1e12 if kbwd_n else 0.0
+    achieved_model = float(n) * n * (2 * (2 * d + k) + (2 * k if args.need_dv else 0)) / (kbwd_mean * 1e-3) / 1e12 if kbwd_n else 0.0
     res = {
         "metric": METRIC,
         "value": round(tflops, 2),
@@ -289,17 +300,22 @@ def run_ours(args, ws, rank, local):
         "dense": {"fwd_ms": round(float(np.mean(fwd_ms)), 4),
                   "bwd_ms": round(float(np.mean(bwd_ms)), 4),
                   "fwd_tflops": round(float(n) * n * fpp / (np.mean(fwd_ms) * 1e-3) / 1e12, 2),
-                  "bwd_tflops": round(achieved, 2),
+                  "bwd_tflops": round(bwd_flops / (bwd_mean * 1e-3) / 1e12, 2),
+                  "fwd_kernel_ms": round(kfwd_ms / max(kfwd_n, 1), 4),
+                  "bwd_kernel_ms": round(kbwd_mean, 4),
                   "frac_of_peak": round(tflops / ws / pk["tflops"], 4),
                   "peak_gib": round(peak_gib, 3)},
-        "roofline": {"bound": "tensor", "kernel": "tc_bwd_kernel (dense backward)",
+        "roofline": {"bound": "tensor", "kernel": "tc_bwd_dqk_kernel (dense backward, dQ and dK)",
                      "achieved": round(achieved, 2), "peak": pk["tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / pk["tflops"], 4), "peak_source": pk["source"] +
-                     " burst bf16 (MEASURED_PEAKS.json bf16_tflops)", "traffic": None},
-        "e2e": {"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "compute_ms": round(e2e_compute, 4),
-                "d2h_ms": round(e2e_d2h, 4)},
+                     " burst bf16 (MEASURED_PEAKS.json bf16_tflops)",
+                     "flops_per_launch": bwd_flops, "flop_convention": "executed (S recompute included)",
+                     "achieved_model_flops": round(achieved_model, 2),
+                     "launches_timed": kbwd_n, "traffic": None},
+        "e2e": ({"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
+                 "d2h_bytes_per_step": int(d2h), "compute_ms": round(e2e_compute, 4),
+                 "d2h_ms": round(e2e_d2h, 4)} if e2e_steps > 0 else None),
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }

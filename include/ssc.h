@@ -137,6 +137,24 @@ int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_vertex,
                             int* centers, int* owner, int* offsets, int* members,
                             ssc_stream_t stream);
 
+/* Launch timing (a measurement hook; the pages have no counterpart).
+ * ssc_profile_enable(1) clears the record and starts recording: every later
+ * launch of a tracked coupling kernel is bracketed by two CUDA events on the
+ * stream it is launched on.  ssc_profile_enable(0) stops recording (the
+ * record is kept), ssc_profile_enable(2) resumes it without clearing; other
+ * values are SSC_ERR_INVALID_ARG.  ssc_profile_read waits for the recorded launches of one
+ * kernel to finish and returns their summed device time in milliseconds and
+ * their count.  Host-side event objects only; no device memory is allocated.
+ * Errors: SSC_ERR_INVALID_ARG for a null pointer or an unknown kernel id,
+ * SSC_ERR_CUDA if an event cannot be read. */
+#define SSC_PROF_DENSE_FWD 0 /* dense forward on CTA pairs (tc_fwd_pair_kernel) */
+#define SSC_PROF_FWD 1       /* single-CTA forward (Geo, and dense when pairs are not used) */
+#define SSC_PROF_BWD_DQK 2   /* backward dQ/dK kernel (tc_bwd_dqk_kernel) */
+#define SSC_PROF_BWD_DV 3    /* optional dV pass (tc_bwd_kernel) */
+#define SSC_PROF_KERNELS 4
+int ssc_profile_enable(int on);
+int ssc_profile_read(int kernel, double* total_ms, int* launches);
+
 /* Scratch bytes ssc_patch_scores_topk needs. */
 size_t ssc_patch_scores_topk_workspace_size(int PN, int PM, int d);
 

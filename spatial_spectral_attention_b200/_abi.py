@@ -19,6 +19,8 @@ SIGNATURES = {
     "ssc_status_string": (ctypes.c_char_p, [I]),
     "ssc_version": (I, []),
     "ssc_kernel_launches": (U64, []),
+    "ssc_profile_enable": (I, [I]),
+    "ssc_profile_read": (I, [I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
     "ssc_device_status": (I, [P, I, ctypes.POINTER(I)]),
     "ssc_set_wait_limit_ns": (I, [U64]),
     "ssc_debug_wait_timeout": (I, [U64, P]),

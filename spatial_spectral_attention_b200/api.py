@@ -58,6 +58,23 @@ def ssc_kernel_launches():
     return int(lib().ssc_kernel_launches())
 
 
+PROF_DENSE_FWD, PROF_FWD, PROF_BWD_DQK, PROF_BWD_DV = 0, 1, 2, 3
+
+
+def ssc_profile_enable(on=True, clear=True):
+    """Start (clearing the record unless clear=False) or stop recording the
+    device time of every coupling kernel launch with CUDA events on its stream."""
+    check("ssc_profile_enable", lib().ssc_profile_enable((1 if clear else 2) if on else 0))
+
+
+def ssc_profile_read(kernel):
+    """(summed milliseconds, launches) of one tracked kernel in the record."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int(0)
+    check("ssc_profile_read", lib().ssc_profile_read(int(kernel), ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, n.value
+
+
 def ssc_device_status(clear=True):
     """Synchronises the current stream and returns the device status word as a
     status code (0 ok, 6 a bounded wait ran out, 1 a bad index table entry)."""

@@ -45,6 +45,7 @@
 #include <cstring>
 
 #include "internal.h"
+#include "ssc.h"
 
 namespace ssc {
 namespace {
@@ -1663,7 +1664,9 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
   if (e != cudaSuccess) return e;
   const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
   const int grid = std::max(1, std::min(work, num_sms()));
+  prof_launch_begin(st);
   kern<<<grid, 96 + 128 * NWG, smem, st>>>(tm, p);
+  prof_launch_end(st, SSC_PROF_FWD);
   count_launch();
   return cudaGetLastError();
 }
@@ -1710,7 +1713,9 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                       : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    prof_launch_begin(st);
     kern<<<grid, 128 * (2 + kBwdComputeGroups), smem, st>>>(tm, p);
+    prof_launch_end(st, SSC_PROF_BWD_DQK);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1721,7 +1726,9 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                       : tc_bwd_kernel<true, kBwdComputeGroups, 0, 0, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    prof_launch_begin(st);
     kern<<<grid, 64 + 128 * kBwdComputeGroups + 128, smem, st>>>(tm, p);
+    prof_launch_end(st, SSC_PROF_BWD_DV);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -25,6 +25,7 @@
 #include <cstring>
 
 #include "internal.h"
+#include "ssc.h"
 
 namespace ssc {
 namespace {
@@ -482,7 +483,10 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   const int pairs = std::max(1, std::min(p.ntiles, nclusters));
   cfg.gridDim = dim3(2 * pairs);
   count_launch();
-  return cudaLaunchKernelEx(&cfg, kern, tm, p);
+  prof_launch_begin(st);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tm, p);
+  prof_launch_end(st, SSC_PROF_DENSE_FWD);
+  return le;
 }
 
 }  // namespace ssc

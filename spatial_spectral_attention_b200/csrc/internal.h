@@ -154,6 +154,10 @@ struct TcArgs {
   const int* row_map;
   const int* col_map;
 };
+// Launch timing record (profile.cu): bracket a kernel launch on stream st.
+void prof_launch_begin(cudaStream_t st);
+void prof_launch_end(cudaStream_t st, int kernel);
+
 bool tc_supported(int d, int k);
 cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
                           const WaitCtl& ctl);

@@ -75,3 +75,15 @@ def test_argument_checks_return_before_any_device_work():
     assert L.ssc_fps_patches(P0, 10, 3, 10, P0, P0, P0, P0, ctypes.c_void_p(256), 1 << 20, None) == 1
     assert L.ssc_patch_scores_topk(P0, 128, 100, P0, 128, 100, 128, 0, P0, P0, 10, P0, P0, 10,
                                    11, P0, None, ctypes.c_void_p(256), 1 << 20, None) == 1
+
+
+def test_profile_record_arguments_are_checked_on_the_host():
+    L = _abi.lib()
+    ms, n = ctypes.c_double(-1.0), ctypes.c_int(-1)
+    assert L.ssc_profile_enable(3) == 1  # SSC_ERR_INVALID_ARG
+    assert L.ssc_profile_read(4, ctypes.byref(ms), ctypes.byref(n)) == 1
+    assert L.ssc_profile_read(0, None, ctypes.byref(n)) == 1
+    # an empty record reads as zero launches without touching the device
+    assert L.ssc_profile_enable(1) == 0 and L.ssc_profile_enable(0) == 0
+    assert L.ssc_profile_read(2, ctypes.byref(ms), ctypes.byref(n)) == 0
+    assert n.value == 0 and ms.value == 0.0

@@ -197,3 +197,23 @@ def test_wait_timeout_reports_status_without_fault():
     # the context is still usable
     Qn, Kn, Vn, dOn = synth.random_inputs(130, 140, 64, 16, seed=1)
     _dense_case(Qn, Kn, Vn, dOn, 0.125, "bf16", need_dV=False)
+
+
+def test_profile_record_times_each_coupling_launch():
+    torch.manual_seed(0)
+    n, d, k = 3000, 128, 196
+    Q = torch.randn(n, d).to(torch.bfloat16).cuda()
+    K = torch.randn(n, d).to(torch.bfloat16).cuda()
+    V = torch.randn(n, k).to(torch.bfloat16).cuda()
+    dO = torch.randn(n, k).cuda()
+    api.ssc_profile_enable(True)
+    for _ in range(2):
+        O, lse = api.ssc_dense_coupling_fwd(Q, K, V, 1.0 / math.sqrt(d))
+        api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, 1.0 / math.sqrt(d))
+    api.ssc_profile_enable(False)
+    api.ssc_dense_coupling_fwd(Q, K, V, 1.0 / math.sqrt(d))  # not recorded
+    fwd_ms, fwd_n = api.ssc_profile_read(api.PROF_DENSE_FWD)
+    bwd_ms, bwd_n = api.ssc_profile_read(api.PROF_BWD_DQK)
+    assert (fwd_n, bwd_n) == (2, 2)
+    assert fwd_ms > 0 and bwd_ms > 0
+    assert api.ssc_profile_read(api.PROF_BWD_DV) == (0.0, 0)
