@@ -63,7 +63,7 @@ struct TensorMaps {
   CUtensorMap vr;    // box {vr, 128}, SW32/SW64 (remainder columns of V)
   CUtensorMap g;     // dO: box {64, 128}, SW128
   CUtensorMap gr;    // dO remainder
-  CUtensorMap dk;    // dK fp32 [nk, d]: box {32, 128}, SW128 (TMA reductions of the partials)
+  CUtensorMap dk;    // dK fp32 [nk, d]: box {32, 32}, SW128 (TMA reductions of the partials)
 };
 
 struct TcParams {
@@ -1029,7 +1029,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full,
       bar_v_empty, bar_s_full, bar_s_read, bar_dp_full, bar_ds_full, bar_do_full, bar_dkp_full,
-      bar_dkp_empty, bar_dq_full, bar_drain, bar_stage_full[2], bar_stage_free[2];
+      bar_dkp_empty, bar_dq_full, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_range[3];  // first tile, first segment in it, number of units
@@ -1043,7 +1043,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   const uint32_t sK0 = sQ + qbytes;  // K stage s at sK0 + s * qbytes
   const uint32_t sV = sK0 + 2 * qbytes;
   const uint32_t sS = sV + vbytes;   // dS tile [q][keys], 2 chunks
-  const uint32_t sStage = sS + 2 * kChunk;  // two 16 KB staging boxes of the dK partial (TMA path)
+  const uint32_t sStage = sS + 2 * kChunk;  // 32 KB: two 4 KB staging boxes per flush warp (TMA path)
   auto gptr = [&](uint32_t s) { return smem_raw + (s - base_u); };
   const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
 
@@ -1065,10 +1065,6 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     mbar_init(&bar_dkp_empty, 128);
     mbar_init(&bar_dq_full, 1);
     mbar_init(&bar_drain, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_stage_full[i], 128);
-      mbar_init(&bar_stage_free[i], 1);
-    }
     s_abort = 0;
     fence_barrier_init();
     // this CTA's share of the (row tile, key segment) units
@@ -1390,8 +1386,8 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     warpgroup_reg_alloc<176>();
     const int lrow = 32 * (warp & 3) + lane;
     const int qbase = lane & ~3;
-    const bool issuer = lrow == 0;  // issues the TMA reductions
-    uint32_t it = 0, blk = 0;
+    const uint32_t wstage = sStage + (warp & 3) * 8192;  // this warp's two 4 KB boxes
+    uint32_t it = 0, wblk = 0;
     bool ok = true;
     UnitRange ur{s_range[0], s_range[1], s_range[2]};
     int t, jb, je;
@@ -1433,23 +1429,24 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
         tc_fence_before();
         mbar_arrive(&bar_dkp_empty);
         if (p.dk_tma) {
-          // 32-column blocks: every thread writes its key row (8 units of 16 B,
-          // unit u at u ^ (row & 7), the tensor map's 128-byte swizzle), then one
-          // thread hands the block to the TMA unit, which adds it into dK
+          // Each warp adds its own 32 key rows: 32-column boxes of 32 rows (4 KB),
+          // written into the warp's two staging buffers (unit u of a row at
+          // u ^ (row & 7), the tensor map's 128-byte swizzle) and handed by lane 0
+          // to the TMA unit.  The warp only waits for its own reductions, and the
+          // CTA keeps eight of them in flight.
 #pragma unroll
           for (int bq = 0; bq < 4; ++bq) {
             if (2 * bq >= d16) break;
-            const int sb = blk & 1;
-            const uint32_t sbuf = sStage + sb * kChunk;
-            if (blk >= 2 && !mbar_wait(&bar_stage_free[sb], ((blk >> 1) - 1) & 1, p.ctl, abort)) {
-              ok = false;
-              break;
+            const uint32_t sbuf = wstage + (wblk & 1) * 4096;
+            if (wblk >= 2) {
+              if (lane == 0) bulk_wait_group_read<1>();  // the box written two rounds ago is read
+              __syncwarp();
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const uint32_t* src = &o[2 * bq + (u >> 2)][4 * (u & 3)];
               asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(
-                               sbuf + lrow * 128 + ((u ^ (lrow & 7)) << 4)),
+                               sbuf + lane * 128 + ((u ^ (lane & 7)) << 4)),
                            "r"(__float_as_uint(__uint_as_float(src[0]) * p.scale)),
                            "r"(__float_as_uint(__uint_as_float(src[1]) * p.scale)),
                            "r"(__float_as_uint(__uint_as_float(src[2]) * p.scale)),
@@ -1457,21 +1454,12 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
                            : "memory");
             }
             fence_proxy_async_smem();
-            mbar_arrive(&bar_stage_full[sb]);
-            if (issuer) {
-              if (!mbar_wait(&bar_stage_full[sb], (blk >> 1) & 1, p.ctl, abort)) {
-                ok = false;
-                break;
-              }
-              tma_reduce_add_2d(&tm.dk, 32 * bq, sg.key0, gptr(sbuf));
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_2d(&tm.dk, 32 * bq, sg.key0 + 32 * (warp & 3), gptr(sbuf));
               bulk_commit_group();
-              if (blk >= 1) {
-                // the previous block has been read out of shared memory
-                bulk_wait_group_read<1>();
-                mbar_arrive(&bar_stage_free[(blk - 1) & 1]);
-              }
             }
-            ++blk;
+            ++wblk;
           }
           continue;
         }
@@ -1502,7 +1490,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
       }
     }
     // the reductions still in flight must finish before the CTA exits
-    if (issuer && p.dk_tma) bulk_wait_group_all();
+    if (lane == 0 && p.dk_tma) bulk_wait_group_all();
   }
 
   __syncthreads();
@@ -1560,14 +1548,14 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int b
 }
 
 // 2-D fp32 tensor [rows, cols] with leading dimension ld (elements), box
-// {box_cols, 128}; elements outside the tensor are skipped by reductions.
+// {box_cols, box_rows}; elements outside the tensor are skipped by reductions.
 bool make_map_f32(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_cols,
-                  CUtensorMapSwizzle sw) {
+                  int box_rows, CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, 128};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1707,7 +1695,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
     // key rows contiguous in dK (no column map): partials go through TMA reductions
     p.dk_tma = !a.col_map && p.vec_atomics &&
-               make_map_f32(&tm.dk, dK, a.nKrows, a.d, lddk, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+               make_map_f32(&tm.dk, dK, a.nKrows, a.d, lddk, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
     auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16>
                       : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0>;
