@@ -1029,7 +1029,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full,
       bar_v_empty, bar_s_full, bar_s_read, bar_dp_full, bar_ds_full, bar_do_full, bar_dkp_full,
-      bar_dkp_empty, bar_dq_full, bar_drain;
+      bar_dkp_empty, bar_dq_full, bar_drain, bar_dp_read;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_range[3];  // first tile, first segment in it, number of units
@@ -1060,6 +1060,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     mbar_init(&bar_s_read, 128 * NCG);
     mbar_init(&bar_dp_full, 1);
     mbar_init(&bar_ds_full, 128 * NCG);
+    mbar_init(&bar_dp_read, 128 * NCG);
     mbar_init(&bar_do_full, 128 * NCG);
     mbar_init(&bar_dkp_full, 1);
     mbar_init(&bar_dkp_empty, 128);
@@ -1175,9 +1176,10 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
         };
         ok = issue_s(it);
         // Per key tile the tensor pipe runs dP_j, S_{j+1}, dQ_j, dKp_j: the next
-        // tile's S is computed while the softmax finishes dS_j, and the softmax
-        // works on S_{j+1} while dQ_j and dKp_j run.  dP_{j+1} is committed after
-        // dKp_j, so its barrier also tells the softmax that dS_j has been consumed.
+        // tile's S is issued as soon as the softmax has read dP_j and runs while
+        // it computes dS_j; the softmax then works on S_{j+1} while dQ_j and dKp_j
+        // run.  dP_{j+1} is committed after dKp_j, so its barrier also tells the
+        // softmax that dS_j has been consumed.
         for (int j = jb; j < je && ok; ++j, ++it) {
           const int st = it & 1;
           const uint32_t sK = sK0 + st * qbytes;
@@ -1203,8 +1205,9 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
           }
           mma_commit(&bar_v_empty);
           mma_commit(&bar_dp_full);
-          // dS in shared memory (the softmax has read dP: the columns are free)
-          if (!mbar_wait(&bar_ds_full, it & 1, p.ctl, abort)) {
+          // the softmax has read dP: the next S goes into the columns while it
+          // computes dS
+          if (!mbar_wait(&bar_dp_read, it & 1, p.ctl, abort)) {
             ok = false;
             break;
           }
@@ -1213,6 +1216,12 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
             ok = false;
             break;
           }
+          // dS in shared memory
+          if (!mbar_wait(&bar_ds_full, it & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -1315,16 +1324,19 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
           break;
         }
         tc_fence_after();
+        uint32_t dp[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(ta + 32 * c, dp[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_dp_read);  // the S/dP columns may now receive the next S
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-          uint32_t dp[32];
-          tmem_ld32(ta + 32 * c, dp);
-          tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(pr[c][2 * i] * (__uint_as_float(dp[2 * i]) - Di),
-                                pr[c][2 * i + 1] * (__uint_as_float(dp[2 * i + 1]) - Di));
+            pk[i] = pack_bf16x2(pr[c][2 * i] * (__uint_as_float(dp[c][2 * i]) - Di),
+                                pr[c][2 * i + 1] * (__uint_as_float(dp[c][2 * i + 1]) - Di));
           // row lrow, keys [cbase, cbase+32): 64-key chunk cbase/64, 16-byte
           // units ((cbase%64)/8) + 0..3, swizzled by the row
           const int cbase = col0 + 32 * c;

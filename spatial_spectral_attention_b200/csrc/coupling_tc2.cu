@@ -34,7 +34,7 @@ constexpr int kChunk = 128 * 128;     // 128 rows x 64 bf16, 128B-swizzled
 constexpr int kHalfChunk = 64 * 128;  // 64 rows x 64 bf16
 constexpr int kKS = 4;                // K ring depth
 constexpr int kVS = 3;                // V ring depth
-constexpr int kNWG = 2;               // softmax warpgroups per CTA
+constexpr int kNWG = 1;               // softmax warpgroups per CTA (each thread owns a whole row)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
