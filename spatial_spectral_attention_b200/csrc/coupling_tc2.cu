@@ -35,6 +35,7 @@ constexpr int kHalfChunk = 64 * 128;  // 64 rows x 64 bf16
 constexpr int kKS = 4;                // K ring depth
 constexpr int kVS = 3;                // V ring depth
 constexpr int kNWG = 1;               // softmax warpgroups per CTA (each thread owns a whole row)
+constexpr int kMaxPairs = 80;         // CTA pairs the partial-result workspace is sized for
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -52,12 +53,36 @@ struct PairParams {
   int vbox;    // 64-column boxes per CTA per V tile
   int nkt;     // key tiles of 128
   int ntiles;  // query tiles of 256 rows
+  long long units;  // ntiles * nkt (query tile, key tile) units, split evenly over the pairs
   float scale_log2;
   float* O;
   int ldo;
   float* lse;
+  float* part;  // partial results of query tiles split between pairs: 2 slots per pair
   WaitCtl ctl;
 };
+
+// Floats of one partial-result slot: unnormalised O [256][kp2], then the running
+// max (log2 units) and sum of every row.
+__host__ __device__ inline size_t part_slot_floats(int kp2) { return (size_t)256 * kp2 + 512; }
+
+// The (query tile, key tile) units are numbered tile-major and pair c owns
+// [c U / P, (c + 1) U / P); a run of consecutive units of one query tile is a
+// segment [jb, je) of its key tiles.
+__host__ __device__ inline long long pair_first_unit(int c, long long U, int npairs) {
+  return (long long)c * U / npairs;
+}
+struct PairRange {
+  long long u, u1;
+};
+__device__ __forceinline__ bool pair_next(PairRange& r, int nkt, int& t, int& jb, int& je) {
+  if (r.u >= r.u1) return false;
+  t = (int)(r.u / nkt);
+  jb = (int)(r.u - (long long)t * nkt);
+  je = (int)min((long long)nkt, jb + (r.u1 - r.u));
+  r.u += je - jb;
+  return true;
+}
 
 __device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, uint32_t col) {
   return base + ((uint32_t)(32 * (warp & 3)) << 16) + col;
@@ -145,19 +170,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort = &s_abort;
+  const long long u_first = pair_first_unit(pair, p.units, npairs);
+  const long long u_end = pair_first_unit(pair + 1, p.units, npairs);
 
   if (warp == 0) {
     // ---------------- Q and K producer (both CTAs)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
-      for (int t = pair; t < p.ntiles && !*abort; t += npairs, ++tcount) {
+      PairRange rr{u_first, u_end};
+      int t, jb, je;
+      for (; !*abort && pair_next(rr, p.nkt, t, jb, je); ++tcount) {
         const int row0 = t * 256 + 128 * (int)rank;
         if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         if (rank == 0) mbar_arrive_expect_tx(&bar_q_full, 2 * qbytes);
         for (int c = 0; c < p.qch; ++c)
           tma_load_2d_pair(gptr(sQ) + c * kChunk, &tm.q, 64 * c, row0, lead(&bar_q_full));
         bool ok = true;
-        for (int j = 0; j < p.nkt; ++j, ++it) {
+        for (int j = jb; j < je; ++j, ++it) {
           const int st = it % kKS;
           if (it >= (uint32_t)kKS &&
               !mbar_wait(&bar_k_empty[st], ((it / kKS) - 1) & 1, p.ctl, abort)) {
@@ -177,9 +206,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     // ---------------- V producer (both CTAs): this CTA's kp2/2 columns
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = pair; t < p.ntiles && !*abort; t += npairs) {
+      PairRange rr{u_first, u_end};
+      int t, jb, je;
+      while (!*abort && pair_next(rr, p.nkt, t, jb, je)) {
         bool ok = true;
-        for (int j = 0; j < p.nkt; ++j, ++it) {
+        for (int j = jb; j < je; ++j, ++it) {
           const int st = it % kVS;
           if (it >= (uint32_t)kVS &&
               !mbar_wait(&bar_v_empty[st], ((it / kVS) - 1) & 1, p.ctl, abort)) {
@@ -218,8 +249,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         mma_commit_pair(&bar_k_empty[st]);
         return true;
       };
-      for (int t = pair; t < p.ntiles && ok; t += npairs, ++tcount) {
-        const int nk = p.nkt;
+      PairRange rr{u_first, u_end};
+      int t, jb, je;
+      for (; ok && pair_next(rr, p.nkt, t, jb, je); ++tcount) {
+        const int nk = je - jb;
         if (!mbar_wait(&bar_q_full, tcount & 1, p.ctl, abort)) {
           ok = false;
           break;
@@ -258,15 +291,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     const int col0 = wg * CW;
     const int nchunk = p.kp2 / 16;
     uint32_t it = 0, tcount = 0;
-    for (int t = pair; t < p.ntiles; t += npairs, ++tcount) {
+    PairRange rr{u_first, u_end};
+    int t, jb, je;
+    for (; pair_next(rr, p.nkt, t, jb, je); ++tcount) {
       const int row0 = t * 256 + 128 * (int)rank;
-      const int nk = p.nkt;
+      const int nk = je - jb;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nk; ++j) {
-        const uint32_t g = it + j;
+      for (int jj = 0; jj < nk; ++jj) {
+        const uint32_t g = it + jj;
         const int buf = g & 1;
-        const int nkeys = min(128, p.nk - 128 * j);
+        const int nkeys = min(128, p.nk - 128 * (jb + jj));
         if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort)) {
           ok = false;
           break;
@@ -300,8 +335,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         const float m_new = fmaxf(m, mx * p.scale_log2);
         const bool need = m_new > m + 8.0f;
         // one wait on O per key tile keeps the parity wait in step
-        bool o_pending = j > 0;
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
+        bool o_pending = jj > 0;
+        if (jj > 0 && __any_sync(0xffffffffu, need)) {
           if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
             ok = false;
             break;
@@ -366,29 +401,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
       }
       const int row = row0 + lrow;
       const bool live = row < p.nq;
-      float* optr = p.O + (size_t)(live ? row : 0) * p.ldo;
-      const float inv = 1.0f / l;
       const uint32_t oa = lane_addr(tmem, warp, 256);
-      for (int c = wg; c < nchunk; c += NWG) {
-        uint32_t o[16];
-        tmem_ld16(oa + 16 * c, o);
-        tmem_ld_wait();
-        if (live) {
-          const int c0 = 16 * c;
-          if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
+      if (jb == 0 && je == p.nkt) {
+        // every key tile of this query tile was processed here: O / l and lse
+        float* optr = p.O + (size_t)(live ? row : 0) * p.ldo;
+        const float inv = 1.0f / l;
+        for (int c = wg; c < nchunk; c += NWG) {
+          uint32_t o[16];
+          tmem_ld16(oa + 16 * c, o);
+          tmem_ld_wait();
+          if (live) {
+            const int c0 = 16 * c;
+            if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(optr + c0 + i) =
-                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-          } else {
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(optr + c0 + i) =
+                    make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+              for (int i = 0; i < 16; ++i)
+                if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+            }
           }
         }
+        if (live && wg == 0) p.lse[row] = (m + log2f(l)) * kLn2;
+      } else {
+        // the query tile's key tiles are split between pairs: the unnormalised
+        // O, the running max and the sum go to this pair's slot for the merge
+        // (slot 0: the first query tile of the pair's range, 1: the last)
+        const int slot = 2 * pair + ((long long)t == u_first / p.nkt ? 0 : 1);
+        float* ps = p.part + (size_t)slot * part_slot_floats(p.kp2);
+        const int prow = 128 * (int)rank + lrow;
+        float* po = ps + (size_t)prow * p.kp2;
+        for (int c = wg; c < nchunk; c += NWG) {
+          uint32_t o[16];
+          tmem_ld16(oa + 16 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(po + 16 * c + i) =
+                make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
+                            __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
+        }
+        if (wg == 0) {
+          ps[(size_t)256 * p.kp2 + prow] = m;
+          ps[(size_t)256 * p.kp2 + 256 + prow] = l;
+        }
       }
-      if (live && wg == 0) p.lse[row] = (m + log2f(l)) * kLn2;
       it += nk;
     }
   }
@@ -400,6 +460,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
+}
+
+// Merges the pieces of every query tile whose key tiles were split between
+// pairs (the per-pair results are exact softmax-weighted sums over their key
+// tiles, relative to their own running max m_q, log2 units):
+//   m = max_q m_q,  l = sum_q l_q 2^(m_q - m),  O = sum_q O_q 2^(m_q - m) / l,
+//   lse = (m + log2 l) ln 2.
+// Block c looks at the boundary between pair c and pair c + 1; the first
+// boundary inside a query tile merges that tile, one thread per row.
+__global__ void __launch_bounds__(256) pair_merge_kernel(const PairParams p, int npairs) {
+  const int c = blockIdx.x;
+  const long long U = p.units;
+  const long long b = pair_first_unit(c + 1, U, npairs);
+  if (b >= U || b % p.nkt == 0) return;  // the boundary is not inside a query tile
+  const int t = (int)(b / p.nkt);
+  const long long t0 = (long long)t * p.nkt, t1 = t0 + p.nkt;
+  if (pair_first_unit(c, U, npairs) > t0) return;  // an earlier boundary lies in this tile
+  const int row = threadIdx.x;
+  const int grow = t * 256 + row;
+  if (grow >= p.nq) return;
+  int q0 = c;  // the pair holding the tile's first unit
+  while (q0 > 0 && pair_first_unit(q0, U, npairs) > t0) --q0;
+  const size_t slot_f = part_slot_floats(p.kp2);
+  auto piece = [&](int q) -> const float* {
+    const int slot = 2 * q + (pair_first_unit(q, U, npairs) / p.nkt == t ? 0 : 1);
+    return p.part + (size_t)slot * slot_f;
+  };
+  float m = -INFINITY;
+  for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q)
+    m = fmaxf(m, piece(q)[(size_t)256 * p.kp2 + row]);
+  float l = 0.f;
+  for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q) {
+    const float* ps = piece(q);
+    l += ps[(size_t)256 * p.kp2 + 256 + row] * exp2f(ps[(size_t)256 * p.kp2 + row] - m);
+  }
+  const float inv = 1.0f / l;
+  float* optr = p.O + (size_t)grow * p.ldo;
+  for (int c0 = 0; c0 < p.k; c0 += 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q) {
+      const float* ps = piece(q);
+      const float w = exp2f(ps[(size_t)256 * p.kp2 + row] - m) * inv;
+      const float4 o = *reinterpret_cast<const float4*>(ps + (size_t)row * p.kp2 + c0);
+      acc.x = fmaf(o.x, w, acc.x);
+      acc.y = fmaf(o.y, w, acc.y);
+      acc.z = fmaf(o.z, w, acc.z);
+      acc.w = fmaf(o.w, w, acc.w);
+    }
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    for (int i = 0; i < 4 && c0 + i < p.k; ++i) optr[c0 + i] = v[i];
+  }
+  p.lse[grow] = (m + log2f(l)) * kLn2;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -436,10 +548,14 @@ bool map2(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_c
 
 bool tc_pair_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
 
+size_t tc_pair_part_floats(int k) {
+  return 2 * (size_t)kMaxPairs * part_slot_floats((k + 31) / 32 * 32);
+}
+
 cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* V, int ldv, int nN, int nM, int d, int k,
-                               float scale, float* O, int ldo, float* lse, cudaStream_t st,
-                               const WaitCtl& ctl) {
+                               float scale, float* O, int ldo, float* lse, float* part,
+                               cudaStream_t st, const WaitCtl& ctl) {
   PairParams p;
   std::memset(&p, 0, sizeof(p));
   p.nq = nN;
@@ -452,11 +568,14 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   p.vbox = (p.vh + 63) / 64;
   p.nkt = (nM + 127) / 128;
   p.ntiles = (nN + 255) / 256;
+  p.units = (long long)p.ntiles * p.nkt;
   p.scale_log2 = scale * kLog2e;
   p.O = O;
   p.ldo = ldo;
   p.lse = lse;
+  p.part = part;
   p.ctl = ctl;
+  if (!part) return cudaErrorInvalidValue;
   PairMaps tm;
   std::memset(&tm, 0, sizeof(tm));
   if (!map2(&tm.q, Q, nN, d, ldq, 64, 128) || !map2(&tm.k, K, nM, d, ldk, 64, 64) ||
@@ -480,13 +599,18 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1)
     nclusters = std::max(1, sms / 2);
   cudaGetLastError();
-  const int pairs = std::max(1, std::min(p.ntiles, nclusters));
+  // every resident pair gets an equal share of the units (at least one)
+  const int pairs = (int)std::max<long long>(
+      1, std::min<long long>(p.units, std::min(nclusters, kMaxPairs)));
   cfg.gridDim = dim3(2 * pairs);
   count_launch();
   prof_launch_begin(st);
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tm, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tm, p);
   prof_launch_end(st, SSC_PROF_DENSE_FWD);
-  return le;
+  if (e != cudaSuccess || pairs == 1) return e;
+  pair_merge_kernel<<<pairs - 1, 256, 0, st>>>(p, pairs);
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace ssc

@@ -170,10 +170,13 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
 // ------------------------------------------------------------ coupling_tc2.cu (bf16, CTA pairs)
 // Dense forward on clusters of two CTAs issuing 2-SM MMAs (query tiles of 256).
 bool tc_pair_supported(int d, int k);
+// Partial-result workspace (floats) of the dense pair forward: query tiles whose
+// key tiles are split between CTA pairs are merged from it.
+size_t tc_pair_part_floats(int k);
 cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* V, int ldv, int nN, int nM, int d, int k,
-                               float scale, float* O, int ldo, float* lse, cudaStream_t st,
-                               const WaitCtl& ctl);
+                               float scale, float* O, int ldo, float* lse, float* part,
+                               cudaStream_t st, const WaitCtl& ctl);
 
 // Test hook: a kernel that waits on a barrier nothing arrives on.
 cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl);

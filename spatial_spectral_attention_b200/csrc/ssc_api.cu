@@ -96,9 +96,9 @@ struct DenseWs {
   __nv_bfloat16* dOb;
   __nv_bfloat16* Vpad;  // V re-packed with a 16-byte aligned row pitch
   float* D;
+  float* part;  // split query tiles of the pair forward (partial O, max, sum)
 };
 size_t dense_ws(void* base, int nN, int nM, int d, int k, int dtype, DenseWs* w) {
-  (void)d;
   Carve c(base);
   DenseWs x;
   x.tiles = c.take<RowTile>(dense_num_tiles(nN));
@@ -107,6 +107,7 @@ size_t dense_ws(void* base, int nN, int nM, int d, int k, int dtype, DenseWs* w)
   x.dOb = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nN * kp_of(k)) : nullptr;
   x.Vpad = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)nM * kp_of(k)) : nullptr;
   x.D = c.take<float>(nN);
+  x.part = dtype == SSC_BF16 && tc_pair_supported(d, k) ? c.take<float>(tc_pair_part_floats(k)) : nullptr;
   if (w) *w = x;
   return c.used + 256;
 }
@@ -297,7 +298,7 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
   if (tc_pair_supported(d, k))
     return cuda_status(launch_tc_fwd_pair(static_cast<const __nv_bfloat16*>(Q), ldq,
                                           static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt, nN,
-                                          nM, d, k, scale, O, ldo, lse, st, ctl));
+                                          nM, d, k, scale, O, ldo, lse, w.part, st, ctl));
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
            ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
