@@ -53,6 +53,7 @@ struct PairParams {
   int vbox;    // 64-column boxes per CTA per V tile
   int nkt;     // key tiles of 128
   int ntiles;  // query tiles of 256 rows
+  int sum_col;  // V column holding ones (the row sum comes out of P V), or -1
   long long units;  // ntiles * nkt (query tile, key tile) units, split evenly over the pairs
   float scale_log2;
   float* O;
@@ -88,21 +89,36 @@ __device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, uint32_t 
   return base + ((uint32_t)(32 * (warp & 3)) << 16) + col;
 }
 
-__device__ __forceinline__ float max32(const float (&x)[32]) {
-  float t[16];
+// Maximum of N values with the three-input max of sm_100 (N / 2 instructions
+// instead of N - 1), as a tree.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+template <int N>
+__device__ __forceinline__ float max_tree3(const float (&v)[N]) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(v[0], v[1]);
+  } else {
+    constexpr int M = (N + 2) / 3;
+    float w[M];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = fmaxf(x[i], x[i + 16]);
-#pragma unroll
-  for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  return t[0];
+    for (int i = 0; i < N / 3; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    if constexpr (N % 3 == 1) w[N / 3] = v[N - 1];
+    if constexpr (N % 3 == 2) w[N / 3] = fmaxf(v[N - 2], v[N - 1]);
+    return max_tree3<M>(w);
+  }
 }
 
 // D16 > 0 fixes d = 16 D16 at compile time so the S = Q K^T issue loop is fully
 // unrolled (a run-time trip count slows the single issuing thread); D16 = 0
-// takes d from the parameters.
-template <int NWG, int D16>
+// takes d from the parameters.  kSumCol: V carries a column of ones at
+// p.sum_col, so O's column sum_col is the softmax row sum (of the bf16 P that
+// the MMA multiplies) and the softmax threads do not add it up.
+template <int NWG, int D16, bool kSumCol>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     tc_fwd_pair_kernel(const __grid_constant__ PairMaps tm, const PairParams p) {
   const int d16 = D16 > 0 ? D16 : p.d / 16;
@@ -319,9 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
             for (int i = 0; i < 32; ++i)
               if (col0 + 32 * c + i >= nkeys) x[c][i] = -INFINITY;
         }
-        float mx = max32(x[0]);
-#pragma unroll
-        for (int c = 1; c < NC; ++c) mx = fmaxf(mx, max32(x[c]));
+        float mx = max_tree3<NC * 32>(reinterpret_cast<const float(&)[NC * 32]>(x));
         if (NWG > 1) {
           s_pmax[g & 1][wg][lrow] = mx;
           mbar_arrive(&bar_xmax);
@@ -368,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
           for (int i = 0; i < 16; ++i) {
             const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
             const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], p.scale_log2, neg_m));
-            rs[i & 3] += a0 + a1;
+            if (!kSumCol) rs[i & 3] += a0 + a1;
             pk[c][i] = pack_bf16x2(a0, a1);
           }
         l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
@@ -391,7 +405,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
       const uint32_t glast = it + nk - 1;
       if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
       tc_fence_after();
-      if (NWG > 1) {
+      if (kSumCol) {
+        // the row sum is O's column sum_col (this thread's TMEM lane)
+        const uint32_t lv = tmem_ld1(lane_addr(tmem, warp, 256 + p.sum_col));
+        tmem_ld_wait();
+        l = __uint_as_float(lv);
+      } else if (NWG > 1) {
         s_psum[wg][lrow] = l;
         mbar_arrive(&bar_xsum);
         if (!mbar_wait(&bar_xsum, tcount & 1, p.ctl, abort)) break;
@@ -555,7 +574,7 @@ size_t tc_pair_part_floats(int k) {
 cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* V, int ldv, int nN, int nM, int d, int k,
                                float scale, float* O, int ldo, float* lse, float* part,
-                               cudaStream_t st, const WaitCtl& ctl) {
+                               int sum_col, cudaStream_t st, const WaitCtl& ctl) {
   PairParams p;
   std::memset(&p, 0, sizeof(p));
   p.nq = nN;
@@ -574,14 +593,17 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   p.ldo = ldo;
   p.lse = lse;
   p.part = part;
+  p.sum_col = sum_col;
   p.ctl = ctl;
   if (!part) return cudaErrorInvalidValue;
   PairMaps tm;
   std::memset(&tm, 0, sizeof(tm));
   if (!map2(&tm.q, Q, nN, d, ldq, 64, 128) || !map2(&tm.k, K, nM, d, ldk, 64, 64) ||
-      !map2(&tm.v, V, nM, k, ldv, 64, 128))
+      !map2(&tm.v, V, nM, sum_col >= 0 ? k + 1 : k, ldv, 64, 128))
     return cudaErrorInvalidValue;
-  auto kern = d == 128 ? tc_fwd_pair_kernel<kNWG, 8> : tc_fwd_pair_kernel<kNWG, 0>;
+  if (sum_col >= 0 && (sum_col != k || k + 1 > p.kp2)) return cudaErrorInvalidValue;
+  auto kern = d == 128 ? (sum_col >= 0 ? tc_fwd_pair_kernel<kNWG, 8, true> : tc_fwd_pair_kernel<kNWG, 8, false>)
+                       : (sum_col >= 0 ? tc_fwd_pair_kernel<kNWG, 0, true> : tc_fwd_pair_kernel<kNWG, 0, false>);
   const int smem = 1024 + p.qch * kChunk + kKS * p.qch * kHalfChunk + kVS * p.vbox * kChunk;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

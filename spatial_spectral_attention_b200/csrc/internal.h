@@ -64,9 +64,10 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
 // bf16 or fp32 per in_f32), zero-filled up to out_ld.
 // A map entry outside [0, src_rows) yields a zero row and sets the
 // bad-index bit of the status word.
+// ones_col >= 0: that padding column of every output row is set to one.
 cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const int* map, int rows,
                                     int src_rows, int cols, __nv_bfloat16* out, int out_ld,
-                                    unsigned* status, cudaStream_t st);
+                                    unsigned* status, cudaStream_t st, int ones_col = -1);
 // fp32 variant (check mode).
 cudaError_t launch_gather_rows_f32(const float* in, int in_ld, const int* map, int rows,
                                    int src_rows, int cols, float* out, int out_ld, unsigned* status,
@@ -171,12 +172,14 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
 // Dense forward on clusters of two CTAs issuing 2-SM MMAs (query tiles of 256).
 bool tc_pair_supported(int d, int k);
 // Partial-result workspace (floats) of the dense pair forward: query tiles whose
-// key tiles are split between CTA pairs are merged from it.
+// key tiles are split between CTA pairs are merged from it.  sum_col >= 0: V
+// holds ones in that column (V is read with k + 1 columns), so the softmax row
+// sum comes out of the P V product; -1: the softmax threads add it up.
 size_t tc_pair_part_floats(int k);
 cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* V, int ldv, int nN, int nM, int d, int k,
                                float scale, float* O, int ldo, float* lse, float* part,
-                               cudaStream_t st, const WaitCtl& ctl);
+                               int sum_col, cudaStream_t st, const WaitCtl& ctl);
 
 // Test hook: a kernel that waits on a barrier nothing arrives on.
 cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl);

@@ -36,10 +36,13 @@ __device__ __forceinline__ int checked_src(const int* map, int r, int src_rows, 
   return src;
 }
 
+// Padding columns [cols, out_ld) are zero, except column ones_col (when >= 0),
+// which is set to one: a column of ones in V makes the P V product carry the
+// softmax row sum.
 __global__ void gather_bf16_from_bf16(const __nv_bfloat16* __restrict__ in, int in_ld,
                                       const int* __restrict__ map, int rows, int src_rows, int cols,
                                       __nv_bfloat16* __restrict__ out, int out_ld, int vec_ok,
-                                      unsigned* status) {
+                                      int ones_col, unsigned* status) {
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
@@ -55,9 +58,10 @@ __global__ void gather_bf16_from_bf16(const __nv_bfloat16* __restrict__ in, int 
       for (int v = lane; v < nvec; v += 32)
         reinterpret_cast<uint4*>(o)[v] = __ldg(reinterpret_cast<const uint4*>(a) + v);
       for (int c = (nvec << 3) + lane; c < out_ld; c += 32)
-        o[c] = c < cols ? a[c] : __float2bfloat16(0.f);
+        o[c] = c < cols ? a[c] : __float2bfloat16(c == ones_col ? 1.f : 0.f);
     } else {
-      for (int c = lane; c < out_ld; c += 32) o[c] = c < cols ? a[c] : __float2bfloat16(0.f);
+      for (int c = lane; c < out_ld; c += 32)
+        o[c] = c < cols ? a[c] : __float2bfloat16(c == ones_col ? 1.f : 0.f);
     }
   }
 }
@@ -305,7 +309,7 @@ int grid_for(long work, int per_block) {
 
 cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const int* map, int rows,
                                     int src_rows, int cols, __nv_bfloat16* out, int out_ld,
-                                    unsigned* status, cudaStream_t st) {
+                                    unsigned* status, cudaStream_t st, int ones_col) {
   if (rows <= 0) return cudaSuccess;
   const int g = grid_for(rows, 8);
   if (in_f32) {
@@ -317,7 +321,8 @@ cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const
                        (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
                        (reinterpret_cast<uintptr_t>(out) % 16 == 0);
     gather_bf16_from_bf16<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), in_ld, map,
-                                             rows, src_rows, cols, out, out_ld, vec_ok, status);
+                                             rows, src_rows, cols, out, out_ld, vec_ok, ones_col,
+                                             status);
     count_launch();
   }
   return cudaGetLastError();

@@ -162,16 +162,22 @@ bool ws_ok(void* ws, size_t have, size_t need) {
 
 // The bf16 V operand as the tensor-core kernels read it: in place when its
 // rows are 16-byte aligned, else re-packed into the workspace.
+// V for the tensor-core kernels: used in place when its rows are 16-byte
+// aligned, else re-packed into the workspace with a pitch of kp.  With
+// ones_col = k (possible when k is not a multiple of 16, so the pitch has a
+// padding column) V is always re-packed and that column is set to one.
 cudaError_t dense_v(const void* V, int ldv, int nM, int k, const DenseWs& w,
-                    const __nv_bfloat16** Vout, int* ldout, cudaStream_t st, unsigned* status) {
-  if (ldv % 8 == 0 && aligned16(V)) {
+                    const __nv_bfloat16** Vout, int* ldout, cudaStream_t st, unsigned* status,
+                    int ones_col = -1) {
+  if (ones_col < 0 && ldv % 8 == 0 && aligned16(V)) {
     *Vout = static_cast<const __nv_bfloat16*>(V);
     *ldout = ldv;
     return cudaSuccess;
   }
   *Vout = w.Vpad;
   *ldout = (int)kp_of(k);
-  return launch_gather_rows_bf16(V, ldv, 0, nullptr, nM, nM, k, w.Vpad, (int)kp_of(k), status, st);
+  return launch_gather_rows_bf16(V, ldv, 0, nullptr, nM, nM, k, w.Vpad, (int)kp_of(k), status, st,
+                                 ones_col);
 }
 
 }  // namespace
@@ -294,11 +300,16 @@ int ssc_dense_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const
   WaitCtl ctl = make_ctl();
   const __nv_bfloat16* Vt;
   int ldvt;
-  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
-  if (tc_pair_supported(d, k))
+  // the pair forward takes the softmax row sum from a column of ones in V when
+  // the V pitch has a padding column
+  const bool pair = tc_pair_supported(d, k);
+  const int sum_col = pair && k % 16 != 0 ? k : -1;
+  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status, sum_col)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  if (pair)
     return cuda_status(launch_tc_fwd_pair(static_cast<const __nv_bfloat16*>(Q), ldq,
                                           static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt, nN,
-                                          nM, d, k, scale, O, ldo, lse, w.part, st, ctl));
+                                          nM, d, k, scale, O, ldo, lse, w.part, sum_col, st, ctl));
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
            ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
