@@ -1673,7 +1673,7 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
 
 cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,
                           const float* D, float* dQ, int lddq, float* dK, int lddk, float* dV,
-                          int lddv, cudaStream_t st, const WaitCtl& ctl) {
+                          int lddv, cudaStream_t st, const WaitCtl& ctl, float* dK_ord) {
   TcParams p;
   fill_common(a, p);
   p.lse_in = lse;
@@ -1704,10 +1704,16 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
   {
     // dQ and dK: dO lives in TMEM, K is double-buffered, a warpgroup of its own
     // reduces the dK partials
-    p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
+    if (dK_ord) {
+      // dK in the key order of K: contiguous rows, no column map
+      p.col_map = nullptr;
+      p.dK = dK_ord;
+      p.lddk = a.d;
+    }
+    p.vec_atomics = (p.lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(p.dK) % 16 == 0);
     // key rows contiguous in dK (no column map): partials go through TMA reductions
-    p.dk_tma = !a.col_map && p.vec_atomics &&
-               make_map_f32(&tm.dk, dK, a.nKrows, a.d, lddk, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    p.dk_tma = !p.col_map && p.vec_atomics &&
+               make_map_f32(&tm.dk, p.dK, a.nKrows, a.d, p.lddk, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
     auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16>
                       : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0>;
@@ -1720,6 +1726,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (dV) {
+    p.col_map = a.col_map;  // dV rows are scattered through the column map
     p.vec_atomics = (lddv % 4 == 0) && (reinterpret_cast<uintptr_t>(dV) % 16 == 0);
     const int smem = 1024 + 2 * p.qch * kChunk + vb + 2 * kChunk;
     auto kern = fixed ? tc_bwd_kernel<true, kBwdComputeGroups, 2, 3, 16>

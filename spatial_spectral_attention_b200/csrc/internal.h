@@ -164,9 +164,17 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
                           const WaitCtl& ctl);
 // dQ written (scaled), dK accumulated with atomics (caller zeroes it).
 // dOb: bf16 [nQrows, lddob] (k padded with zeros), lse/D in row order.
+// dK_ord (optional): dK is reduced into this [a.nKrows, d] buffer in the key
+// order of a.K (no column map, contiguous rows) instead of into dK; the caller
+// scatters it.  The dV pass still uses a.col_map.
 cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,
                           const float* D, float* dQ, int lddq, float* dK, int lddk, float* dV,
-                          int lddv, cudaStream_t st, const WaitCtl& ctl);
+                          int lddv, cudaStream_t st, const WaitCtl& ctl, float* dK_ord = nullptr);
+// out[map[r]] = in[r] for r < rows (map entries outside [0, dst_rows) are dropped
+// and set the bad-index bit).
+cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, int rows,
+                                    int dst_rows, int cols, float* out, int out_ld,
+                                    unsigned* status, cudaStream_t st);
 
 // ------------------------------------------------------------ coupling_tc2.cu (bf16, CTA pairs)
 // Dense forward on clusters of two CTAs issuing 2-SM MMAs (query tiles of 256).

@@ -27,13 +27,19 @@ __device__ __forceinline__ double load_elem(const void* F, size_t i) {
   else return (double)__bfloat162float(static_cast<const __nv_bfloat16*>(F)[i]);
 }
 
-// One block per patch, one thread per descriptor channel.
+// One block per patch, one thread per descriptor channel; the member indices
+// are staged in shared memory and each thread issues the loads of kPoolBatch
+// members before adding them, in member order (the fixed summation order keeps
+// the result bit-exact; only the loads run ahead).
 // Offsets are clamped into [0, n] and member indices outside [0, n) skipped;
 // either sets the bad-index bit of the status word.
+constexpr int kPoolStage = 1024;  // member indices staged per round
+constexpr int kPoolBatch = 16;    // loads in flight per thread
 template <bool F32>
 __global__ void pool_kernel(const void* __restrict__ F, int ld, int n, int d,
                             const int* __restrict__ off, const int* __restrict__ mem,
                             double* __restrict__ mu, unsigned* status) {
+  __shared__ int s_mem[kPoolStage];
   const int p = blockIdx.x;
   int b = off[p], e = off[p + 1];
   if (b < 0 || e <= b || e > n) {
@@ -41,17 +47,35 @@ __global__ void pool_kernel(const void* __restrict__ F, int ld, int n, int d,
     b = min(max(b, 0), n);
     e = min(max(e, b), n);
   }
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+  // one pass over the members per group of blockDim.x channels
+  for (int c0 = 0; c0 < d; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
     double s = 0.0;
-    for (int r = b; r < e; ++r) {
-      const int v = mem[r];
-      if (v < 0 || v >= n) {
-        atomicOr(status, kStatusBadIndex);
-        continue;
+    for (int r0 = b; r0 < e; r0 += kPoolStage) {
+      const int nr = min(kPoolStage, e - r0);
+      __syncthreads();
+      for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+        const int v = mem[r0 + i];
+        if (v < 0 || v >= n) atomicOr(status, kStatusBadIndex);
+        s_mem[i] = v;
       }
-      s = __dadd_rn(s, load_elem<F32>(F, (size_t)v * ld + c));
+      __syncthreads();
+      if (c >= d) continue;
+      for (int i0 = 0; i0 < nr; i0 += kPoolBatch) {
+        double x[kPoolBatch];
+#pragma unroll
+        for (int u = 0; u < kPoolBatch; ++u) {
+          const int v = i0 + u < nr ? s_mem[i0 + u] : -1;
+          x[u] = (v >= 0 && v < n) ? load_elem<F32>(F, (size_t)v * ld + c) : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < kPoolBatch; ++u) {
+          const int v = i0 + u < nr ? s_mem[i0 + u] : -1;
+          if (v >= 0 && v < n) s = __dadd_rn(s, x[u]);
+        }
+      }
     }
-    mu[(size_t)p * d + c] = __ddiv_rn(s, (double)max(e - b, 1));
+    if (c < d) mu[(size_t)p * d + c] = __ddiv_rn(s, (double)max(e - b, 1));
   }
 }
 

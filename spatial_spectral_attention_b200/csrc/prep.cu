@@ -53,11 +53,17 @@ __global__ void gather_bf16_from_bf16(const __nv_bfloat16* __restrict__ in, int 
       continue;
     }
     const __nv_bfloat16* a = in + (size_t)src * in_ld;
-    if (vec_ok) {
-      const int nvec = cols >> 3;  // full 8-element chunks
+    if (vec_ok == 2) {
+      const int nvec = cols >> 3;  // full 8-element (16-byte) chunks
       for (int v = lane; v < nvec; v += 32)
         reinterpret_cast<uint4*>(o)[v] = __ldg(reinterpret_cast<const uint4*>(a) + v);
       for (int c = (nvec << 3) + lane; c < out_ld; c += 32)
+        o[c] = c < cols ? a[c] : __float2bfloat16(c == ones_col ? 1.f : 0.f);
+    } else if (vec_ok == 1) {
+      const int nvec = cols >> 2;  // full 4-element (8-byte) chunks
+      for (int v = lane; v < nvec; v += 32)
+        reinterpret_cast<uint2*>(o)[v] = __ldg(reinterpret_cast<const uint2*>(a) + v);
+      for (int c = (nvec << 2) + lane; c < out_ld; c += 32)
         o[c] = c < cols ? a[c] : __float2bfloat16(c == ones_col ? 1.f : 0.f);
     } else {
       for (int c = lane; c < out_ld; c += 32)
@@ -317,14 +323,49 @@ cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const
                                             src_rows, cols, out, out_ld, status);
     count_launch();
   } else {
-    const int vec_ok = (in_ld % 8 == 0) && (out_ld % 8 == 0) &&
-                       (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
-                       (reinterpret_cast<uintptr_t>(out) % 16 == 0);
+    // 2: rows 16-byte aligned on both sides, 1: 8-byte aligned, 0: element copies
+    const uintptr_t ia = reinterpret_cast<uintptr_t>(in), oa = reinterpret_cast<uintptr_t>(out);
+    const int vec_ok = (in_ld % 8 == 0 && out_ld % 8 == 0 && ia % 16 == 0 && oa % 16 == 0)
+                           ? 2
+                           : (in_ld % 4 == 0 && out_ld % 4 == 0 && ia % 8 == 0 && oa % 8 == 0) ? 1 : 0;
     gather_bf16_from_bf16<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), in_ld, map,
                                              rows, src_rows, cols, out, out_ld, vec_ok, ones_col,
                                              status);
     count_launch();
   }
+  return cudaGetLastError();
+}
+
+__global__ void scatter_rows_f32_kernel(const float* __restrict__ in, int in_ld,
+                                        const int* __restrict__ map, int rows, int dst_rows,
+                                        int cols, float* __restrict__ out, int out_ld, int vec_ok,
+                                        unsigned* status) {
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int dst = checked_src(map, r, dst_rows, status);
+    if (dst < 0) continue;
+    const float* a = in + (size_t)r * in_ld;
+    float* o = out + (size_t)dst * out_ld;
+    if (vec_ok) {
+      for (int v = lane; v < (cols >> 2); v += 32)
+        reinterpret_cast<float4*>(o)[v] = __ldg(reinterpret_cast<const float4*>(a) + v);
+      for (int c = ((cols >> 2) << 2) + lane; c < cols; c += 32) o[c] = a[c];
+    } else {
+      for (int c = lane; c < cols; c += 32) o[c] = a[c];
+    }
+  }
+}
+
+cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, int rows,
+                                    int dst_rows, int cols, float* out, int out_ld,
+                                    unsigned* status, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int vec_ok = in_ld % 4 == 0 && out_ld % 4 == 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  scatter_rows_f32_kernel<<<grid_for(rows, 8), 256, 0, st>>>(in, in_ld, map, rows, dst_rows, cols,
+                                                             out, out_ld, vec_ok, status);
+  count_launch();
   return cudaGetLastError();
 }
 

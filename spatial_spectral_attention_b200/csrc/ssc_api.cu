@@ -119,6 +119,7 @@ struct GeoWs {
   void* dOp;
   float* D;
   float* lsep;
+  float* dKg;  // dK in the patch-major key order (bf16 path), scattered to vertex order after
   RowTile* tiles;
   KeySeg* segs;
   int* counts;
@@ -144,6 +145,7 @@ size_t geo_ws(void* base, int nN, int nM, int d, int k, int PN, int PM, int R, i
   x.dOp = c.take<uint8_t>((size_t)nN * x.ldg * es);
   x.D = c.take<float>(nN);
   x.lsep = c.take<float>(nN);
+  x.dKg = dtype == SSC_BF16 ? c.take<float>((size_t)nM * d) : nullptr;
   x.tiles = c.take<RowTile>(geo_max_tiles(nN, PN));
   x.segs = c.take<KeySeg>(geo_max_segs(nM, PM, PN, R));
   x.counts = c.take<int>(2);
@@ -476,14 +478,22 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const v
   e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, static_cast<__nv_bfloat16*>(w.dOp),
                       w.ldg, nullptr, 0, w.D, w.lsep, ctl.status, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
+  // dK is reduced in the patch-major key order (contiguous key rows, so TMA
+  // reductions apply) and scattered to vertex order afterwards: memM lists
+  // every source vertex once, so the scatter writes each row of dK once
+  // (dK itself is zeroed too, so that rows of vertices missing from inconsistent
+  // tables read as zero rather than as stale memory)
+  if ((e = zero_matrix(w.dKg, d, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
            static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
            w.tiles, w.segs, w.counts, 0, w.prefix, memN, memM};
-  return cuda_status(launch_tc_bwd(a, static_cast<const __nv_bfloat16*>(w.dOp), w.ldg, w.lsep, w.D,
-                                   dQ, lddq, dK, lddk, dV, lddv, st, ctl));
+  if ((e = launch_tc_bwd(a, static_cast<const __nv_bfloat16*>(w.dOp), w.ldg, w.lsep, w.D, dQ, lddq,
+                         dK, lddk, dV, lddv, st, ctl, w.dKg)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  return cuda_status(launch_scatter_rows_f32(w.dKg, d, memM, nM, nM, d, dK, lddk, ctl.status, st));
 }
 
 }  // extern "C"

@@ -69,7 +69,10 @@ def test_dense_bf16_workload_ragged():
 
 @pytest.mark.parametrize("nN,nM,d,k", [(1, 1, 128, 196), (129, 300, 64, 25), (513, 77, 128, 16),
                                        (256, 1000, 128, 256), (200, 200, 64, 100),
-                                       (130, 260, 128, 32), (384, 129, 128, 196)])
+                                       (130, 260, 128, 32), (384, 129, 128, 196),
+                                       # one query tile over 157 key tiles: the dense forward
+                                       # splits it between every CTA pair and merges ~74 pieces
+                                       (200, 20000, 128, 196)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_dense_shapes(nN, nM, d, k, dtype):
     Qn, Kn, Vn, dOn = synth.random_inputs(nN, nM, d, k, seed=nN * 7 + nM, q_scale=0.5)
