@@ -23,6 +23,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "internal.h"
 #include "ssc.h"
@@ -486,8 +488,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
 // tiles, relative to their own running max m_q, log2 units):
 //   m = max_q m_q,  l = sum_q l_q 2^(m_q - m),  O = sum_q O_q 2^(m_q - m) / l,
 //   lse = (m + log2 l) ln 2.
-// Block c looks at the boundary between pair c and pair c + 1; the first
-// boundary inside a query tile merges that tile, one thread per row.
+// Block (c, y) looks at the boundary between pair c and pair c + 1; the first
+// boundary inside a query tile merges that tile.  The block covers 32 of the
+// tile's 256 rows; eight threads share a row, each taking every eighth float4
+// of it, so the loads of a row are contiguous.
+constexpr int kMergeRows = 32;
 __global__ void __launch_bounds__(256) pair_merge_kernel(const PairParams p, int npairs) {
   const int c = blockIdx.x;
   const long long U = p.units;
@@ -496,7 +501,8 @@ __global__ void __launch_bounds__(256) pair_merge_kernel(const PairParams p, int
   const int t = (int)(b / p.nkt);
   const long long t0 = (long long)t * p.nkt, t1 = t0 + p.nkt;
   if (pair_first_unit(c, U, npairs) > t0) return;  // an earlier boundary lies in this tile
-  const int row = threadIdx.x;
+  const int row = blockIdx.y * kMergeRows + (threadIdx.x >> 3);
+  const int part = threadIdx.x & 7;
   const int grow = t * 256 + row;
   if (grow >= p.nq) return;
   int q0 = c;  // the pair holding the tile's first unit
@@ -506,31 +512,49 @@ __global__ void __launch_bounds__(256) pair_merge_kernel(const PairParams p, int
     const int slot = 2 * q + (pair_first_unit(q, U, npairs) / p.nkt == t ? 0 : 1);
     return p.part + (size_t)slot * slot_f;
   };
+  const size_t stat = (size_t)256 * p.kp2;  // row maxima, then row sums
   float m = -INFINITY;
   for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q)
-    m = fmaxf(m, piece(q)[(size_t)256 * p.kp2 + row]);
+    m = fmaxf(m, piece(q)[stat + row]);
   float l = 0.f;
   for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q) {
     const float* ps = piece(q);
-    l += ps[(size_t)256 * p.kp2 + 256 + row] * exp2f(ps[(size_t)256 * p.kp2 + row] - m);
+    l += ps[stat + 256 + row] * exp2f(ps[stat + row] - m);
   }
   const float inv = 1.0f / l;
   float* optr = p.O + (size_t)grow * p.ldo;
-  for (int c0 = 0; c0 < p.k; c0 += 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q) {
-      const float* ps = piece(q);
-      const float w = exp2f(ps[(size_t)256 * p.kp2 + row] - m) * inv;
-      const float4 o = *reinterpret_cast<const float4*>(ps + (size_t)row * p.kp2 + c0);
-      acc.x = fmaf(o.x, w, acc.x);
-      acc.y = fmaf(o.y, w, acc.y);
-      acc.z = fmaf(o.z, w, acc.z);
-      acc.w = fmaf(o.w, w, acc.w);
+  constexpr int kMaxF4 = 8;  // kp2 <= 256: at most 8 float4 per thread
+  float4 acc[kMaxF4];
+#pragma unroll
+  for (int i = 0; i < kMaxF4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q = q0; q < npairs && pair_first_unit(q, U, npairs) < t1; ++q) {
+    const float* ps = piece(q);
+    const float w = exp2f(ps[stat + row] - m) * inv;
+    const float4* src = reinterpret_cast<const float4*>(ps + (size_t)row * p.kp2);
+#pragma unroll
+    for (int i = 0; i < kMaxF4; ++i) {
+      const int f4 = part + 8 * i;
+      if (4 * f4 < p.k) {
+        const float4 o = src[f4];
+        acc[i].x = fmaf(o.x, w, acc[i].x);
+        acc[i].y = fmaf(o.y, w, acc[i].y);
+        acc[i].z = fmaf(o.z, w, acc[i].z);
+        acc[i].w = fmaf(o.w, w, acc[i].w);
+      }
     }
-    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-    for (int i = 0; i < 4 && c0 + i < p.k; ++i) optr[c0 + i] = v[i];
   }
-  p.lse[grow] = (m + log2f(l)) * kLn2;
+#pragma unroll
+  for (int i = 0; i < kMaxF4; ++i) {
+    const int c0 = 4 * (part + 8 * i);
+    if (c0 >= p.k) continue;
+    if (c0 + 4 <= p.k && (p.ldo & 3) == 0) {
+      *reinterpret_cast<float4*>(optr + c0) = acc[i];
+    } else {
+      const float v[4] = {acc[i].x, acc[i].y, acc[i].z, acc[i].w};
+      for (int j = 0; j < 4 && c0 + j < p.k; ++j) optr[c0 + j] = v[j];
+    }
+  }
+  if (part == 0) p.lse[grow] = (m + log2f(l)) * kLn2;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -566,6 +590,32 @@ bool map2(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_c
 }  // namespace
 
 bool tc_pair_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
+
+// CTA pairs of one kernel configuration that can be resident at once, per
+// device (the occupancy query costs host time that would leave the GPU idle
+// between the launches of a call, so its answer is kept).
+int resident_pairs(int dev, const void* kern, cudaLaunchConfig_t cfg) {
+  struct Entry {
+    int dev;
+    const void* kern;
+    size_t smem;
+    int pairs;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : cache)
+    if (e.dev == dev && e.kern == kern && e.smem == cfg.dynamicSmemBytes) return e.pairs;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cfg.gridDim = dim3(2 * std::max(1, sms / 2));
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1)
+    nclusters = std::max(1, sms / 2);
+  cudaGetLastError();
+  cache.push_back({dev, kern, cfg.dynamicSmemBytes, nclusters});
+  return nclusters;
+}
 
 size_t tc_pair_part_floats(int k) {
   return 2 * (size_t)kMaxPairs * part_slot_floats((k + 31) / 32 * 32);
@@ -607,20 +657,14 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   const int smem = 1024 + p.qch * kChunk + kKS * p.qch * kHalfChunk + kVS * p.vbox * kChunk;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int threads = 96 + 128 * kNWG;
-  // pairs that can be resident at once
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cfg.gridDim = dim3(2 * std::max(1, sms / 2));
-  int nclusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1)
-    nclusters = std::max(1, sms / 2);
-  cudaGetLastError();
+  const int nclusters = resident_pairs(dev, reinterpret_cast<const void*>(kern), cfg);
   // every resident pair gets an equal share of the units (at least one)
   const int pairs = (int)std::max<long long>(
       1, std::min<long long>(p.units, std::min(nclusters, kMaxPairs)));
@@ -630,7 +674,7 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   e = cudaLaunchKernelEx(&cfg, kern, tm, p);
   prof_launch_end(st, SSC_PROF_DENSE_FWD);
   if (e != cudaSuccess || pairs == 1) return e;
-  pair_merge_kernel<<<pairs - 1, 256, 0, st>>>(p, pairs);
+  pair_merge_kernel<<<dim3(pairs - 1, 256 / kMergeRows), 256, 0, st>>>(p, pairs);
   count_launch();
   return cudaGetLastError();
 }
