@@ -126,6 +126,55 @@ def barrier(ws):
     dist.barrier(ws)
 
 
+GEO_SWEEP_N = (20000, 40000, 60000, 100000, 160000)
+
+
+def run_geo_sweep(api, synth, torch, dev, need_dv, fpp, bpp):
+    """Geo step (scores/top-R + fwd + bwd) against n with P = n/125 and R = 8:
+    ms per step and peak device memory per size (160k is the warped,
+    non-isometric pair).  Each size: patch tables once, 2 warm-up and 3 timed
+    steps, L2 flushed before each timed step."""
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    bf = lambda a: torch.tensor(a).to(torch.bfloat16).to(dev)
+    out = []
+    for n in GEO_SWEEP_N:
+        gp = synth.make_workload("geo_160k_warped" if n == 160000 else "geo_60k", n=n)
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev) - flush.numel()
+        Q, K, V, dO = bf(gp.F_N), bf(gp.F_M), bf(gp.Phi_M), torch.tensor(gp.dO).to(dev)
+        _, _, offN, memN = api.ssc_fps_patches(torch.tensor(gp.pts_N).to(dev), gp.P)
+        _, _, offM, memM = api.ssc_fps_patches(torch.tensor(gp.pts_M).to(dev), gp.P)
+        gws = torch.empty(api.lib().ssc_geo_coupling_workspace_size(n, n, gp.d, gp.k, gp.P, gp.P, gp.R, 0),
+                          dtype=torch.uint8, device=dev)
+
+        def step():
+            topk = api.ssc_patch_scores_topk(Q, K, offN, memN, offM, memM, gp.R)
+            O, lse = api.ssc_geo_coupling_fwd(Q, K, V, gp.scale, offN, memN, offM, memM, topk,
+                                              workspace=gws)
+            api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, gp.scale, offN, memN, offM, memM, topk,
+                                     need_dV=need_dv, workspace=gws)
+
+        for _ in range(2):
+            step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+        for e in evs:
+            flush.zero_()
+            e[0].record(stream)
+            step()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        peak = (torch.cuda.max_memory_allocated(dev) - flush.numel() - base) / 2**30
+        U = float(np.mean(np.diff(offM.cpu().numpy()))) * gp.R
+        out.append({"n": n, "P": gp.P, "ms_per_step": round(ms, 4),
+                    "tflops": round(float(n) * U * (fpp + bpp) / (ms * 1e-3) / 1e12, 2),
+                    "peak_gib": round(peak, 3)})
+        del Q, K, V, dO, offN, memN, offM, memM, gws
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ws, rank, local):
     import torch
@@ -235,36 +284,64 @@ def run_ours(args, ws, rank, local):
     geo_ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in gev])), ws) if geo else None
     barrier(ws)
 
-    # ---- end to end through the public API with host buffers
-    if not args.e2e:
-        e2e_steps = 0
+    # ---- end to end through the public API with host buffers (pinned).  Every step
+    # copies its inputs up and its results down inside the timed region; the copies
+    # run on two copy streams and overlap the compute: a step's Q, K, V go up into
+    # one of two device buffer sets while the previous step computes, its dO goes
+    # up during its forward, O and lse come down during its backward and dQ, dK
+    # after it.  The time runs from the first upload to the last download.
     out_host = dict(O=torch.empty((n, k), dtype=torch.float32).pin_memory(),
                     lse=torch.empty(n, dtype=torch.float32).pin_memory(),
                     dQ=torch.empty((n, d), dtype=torch.float32).pin_memory(),
                     dK=torch.empty((n, d), dtype=torch.float32).pin_memory())
-    e2e_steps = max(2, min(args.steps, 5)) if args.e2e else 0
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 8)) if args.e2e else 0
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nbuf = 2
+    dev_in = [{x: torch.empty_like(host[x], device=dev) for x in host} for _ in range(nbuf)]
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev(), ev()
+    ev_qkv, ev_do = [ev() for _ in range(nbuf)], [ev() for _ in range(nbuf)]
+    ev_done = [ev() for _ in range(nbuf)]
+    parts = [[ev() for _ in range(3)] for _ in range(e2e_steps)]
     torch.cuda.synchronize()
     barrier(ws)
-    parts = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(e2e_steps)]
-    dev_in = {x: torch.empty_like(host[x], device=dev) for x in host}
-    e0.record(stream)
+    e0.record(up)
     for i in range(e2e_steps):
-        for x in ("Q", "K", "V", "dO"):
-            dev_in[x].copy_(host[x], non_blocking=True)
+        bi = i % nbuf
+        buf = dev_in[bi]
+        with torch.cuda.stream(up):
+            if i >= nbuf:
+                up.wait_event(ev_done[bi])  # step i - 2 is done with these buffers
+            for x in ("Q", "K", "V"):
+                buf[x].copy_(host[x], non_blocking=True)
+            ev_qkv[bi].record(up)
+            buf["dO"].copy_(host["dO"], non_blocking=True)
+            ev_do[bi].record(up)
+        stream.wait_event(ev_qkv[bi])
         parts[i][0].record(stream)
-        O, lse, (dQ, dK, _) = dense_step(dev_in["Q"], dev_in["K"], dev_in["V"], dev_in["dO"])
+        O, lse = api.ssc_dense_coupling_fwd(buf["Q"], buf["K"], buf["V"], scale, workspace=wsb)
         parts[i][1].record(stream)
-        out_host["O"].copy_(O, non_blocking=True)
-        out_host["lse"].copy_(lse, non_blocking=True)
-        out_host["dQ"].copy_(dQ, non_blocking=True)
-        out_host["dK"].copy_(dK, non_blocking=True)
+        with torch.cuda.stream(down):
+            down.wait_event(parts[i][1])
+            O.record_stream(down)
+            lse.record_stream(down)
+            out_host["O"].copy_(O, non_blocking=True)
+            out_host["lse"].copy_(lse, non_blocking=True)
+        stream.wait_event(ev_do[bi])
+        dQ, dK, _ = api.ssc_dense_coupling_bwd(buf["Q"], buf["K"], buf["V"], O, lse, buf["dO"],
+                                               scale, need_dV=args.need_dv, workspace=wsb)
         parts[i][2].record(stream)
-    e1.record(stream)
+        ev_done[bi].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(parts[i][2])
+            dQ.record_stream(down)
+            dK.record_stream(down)
+            out_host["dQ"].copy_(dQ, non_blocking=True)
+            out_host["dK"].copy_(dK, non_blocking=True)
+    e1.record(down)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(e2e_steps, 1), ws)
-    e2e_compute = float(np.mean([p[0].elapsed_time(p[1]) for p in parts])) if parts else 0.0
-    e2e_d2h = float(np.mean([p[1].elapsed_time(p[2]) for p in parts])) if parts else 0.0
+    e2e_compute = float(np.mean([p[0].elapsed_time(p[2]) for p in parts])) if parts else 0.0
     h2d = sum(host[x].numel() * host[x].element_size() for x in ("Q", "K", "V", "dO"))
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
 
@@ -314,11 +391,19 @@ def run_ours(args, ws, rank, local):
                      "launches_timed": kbwd_n, "traffic": None},
         "e2e": ({"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                  "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-                 "d2h_bytes_per_step": int(d2h), "compute_ms": round(e2e_compute, 4),
-                 "d2h_ms": round(e2e_d2h, 4)} if e2e_steps > 0 else None),
+                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+                 "compute_ms_per_step": round(e2e_compute, 4),
+                 "overlap": "uploads and downloads on two copy streams overlap the compute; "
+                            "two input buffer sets; time from the first upload to the last "
+                            "download"} if e2e_steps > 0 else None),
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
+    if args.geo_sweep and rank == 0:
+        res["geo_sweep"] = {"note": "Geo step vs n, P = n/125, R = 8 (160k: warped pair); "
+                                    "peak_gib = peak device memory of the size's inputs, "
+                                    "tables, workspace and outputs",
+                            "sizes": run_geo_sweep(api, synth, torch, dev, args.need_dv, fpp, bpp)}
     if geo:
         U = float(np.mean(np.diff(geo["offM"].cpu().numpy()))) * gpair.R
         gflops = float(gpair.n) * U * (fpp + bpp)
@@ -337,14 +422,21 @@ def oracle_sample(pair, budget_s, need_dv):
     bf = lambda a: torch.tensor(a).to(torch.bfloat16).double().numpy()
     Q, K, V = bf(pair.F_N), bf(pair.F_M), bf(pair.Phi_M)
     dO = bf(pair.dO)
-    rows = 16
-    while True:
+    def run(r):
         t0 = time.perf_counter()
-        oracle.dense_bwd(Q[:rows], K, V, dO[:rows], pair.scale)
-        dt = time.perf_counter() - t0
-        if dt > budget_s / 4 or rows >= pair.n:
-            break
+        oracle.dense_bwd(Q[:r], K, V, dO[:r], pair.scale)
+        return time.perf_counter() - t0
+
+    # grow the sample until a run takes an eighth of the budget, then one run
+    # sized to fill the budget (about budget_s of host work in that last run)
+    rows = 16
+    dt = run(rows)
+    while dt < budget_s / 8 and rows < pair.n:
         rows = min(pair.n, rows * 4)
+        dt = run(rows)
+    if rows < pair.n:
+        rows = max(rows, min(pair.n, int(rows * budget_s / dt)))
+        dt = run(rows)
     full_s = dt * pair.n / rows
     fpp, bpp = pair_flops(pair.d, pair.k, need_dv)
     tflops = float(pair.n) * pair.n * (fpp + bpp) / full_s / 1e12
@@ -397,6 +489,8 @@ def main():
     ap.add_argument("--workload", default="dense_60k")
     ap.add_argument("--n", type=int, default=None, help="resize the workload (profiling runs)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-geo-sweep", dest="geo_sweep", action="store_false",
+                    help="skip the Geo step sweep over n = 20k..160k")
     ap.add_argument("--need-dv", action="store_true")
     ap.add_argument("--no-geo", dest="with_geo", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
