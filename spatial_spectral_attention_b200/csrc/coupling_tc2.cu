@@ -36,7 +36,7 @@ constexpr int kChunk = 128 * 128;     // 128 rows x 64 bf16, 128B-swizzled
 constexpr int kHalfChunk = 64 * 128;  // 64 rows x 64 bf16
 constexpr int kKS = 4;                // K ring depth
 constexpr int kVS = 3;                // V ring depth
-constexpr int kNWG = 1;               // softmax warpgroups per CTA (each thread owns a whole row)
+constexpr int kNWG = 2;               // softmax warpgroups per CTA (a thread pair owns a row)
 constexpr int kMaxPairs = 80;         // CTA pairs the partial-result workspace is sized for
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -87,10 +87,6 @@ __device__ __forceinline__ bool pair_next(PairRange& r, int nkt, int& t, int& jb
   return true;
 }
 
-__device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, uint32_t col) {
-  return base + ((uint32_t)(32 * (warp & 3)) << 16) + col;
-}
-
 // Maximum of N values with the three-input max of sm_100 (N / 2 instructions
 // instead of N - 1), as a tree.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -124,17 +120,13 @@ template <int NWG, int D16, bool kSumCol>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     tc_fwd_pair_kernel(const __grid_constant__ PairMaps tm, const PairParams p) {
   const int d16 = D16 > 0 ? D16 : p.d / 16;
-  constexpr int CW = 128 / NWG;
-  constexpr int NC = CW / 32;
   constexpr int NSM = 128 * NWG;
   constexpr int kVWarp = 2 + 4 * NWG;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[kKS], bar_k_empty[kKS], bar_v_full[kVS],
-      bar_v_empty[kVS], bar_s_full[2], bar_p_full[2], bar_o_full, bar_drain, bar_xmax, bar_xsum;
+      bar_v_empty[kVS], bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ float s_pmax[2][NWG][128];
-  __shared__ float s_psum[NWG][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -166,10 +158,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
       mbar_init(&bar_s_full[i], 1);
       mbar_init(&bar_p_full[i], 2 * (NSM / 32));  // one arrival per softmax warp of both CTAs
     }
-    mbar_init(&bar_o_full, 1);
+    mbar_init(&bar_o_full[0], 1);
+    mbar_init(&bar_o_full[1], 1);
     mbar_init(&bar_drain, 1);
-    mbar_init(&bar_xmax, NSM);
-    mbar_init(&bar_xsum, NSM);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -292,7 +283,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
                         make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128), idesc_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit_pair(&bar_v_empty[vst]);
-          mma_commit_pair(&bar_o_full);
+          mma_commit_pair(&bar_o_full[g & 1]);
           if (j + 2 < nk) ok = issue_s(g + 2);
         }
         mma_commit_pair(&bar_q_empty);
@@ -304,10 +295,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
     }
   } else {
     // ---------------- softmax / correction / epilogue (both CTAs)
+    // Two warpgroups share every 32-lane TMEM quarter: warpgroup w takes lanes
+    // [16 w, 16 w + 16) of each quarter (.16x32bx2 accesses) and the two halves of
+    // a warp split each of those rows' 128 columns, thread half h holding S
+    // columns [64 h, 64 h + 64).  A row's max then takes one shuffle and no
+    // exchange between warpgroups, and every SMSP runs two softmax warps.  O is
+    // handled in 32-column chunks, half h taking the 16 columns at 32 c + 16 h.
+    static_assert(NWG == 2, "the softmax layout below is for two warpgroups");
     const int wg = (warp - 2) >> 2;
-    const int lrow = 32 * (warp & 3) + lane;
-    const int col0 = wg * CW;
-    const int nchunk = p.kp2 / 16;
+    const int half = lane >> 4;
+    const int lrow = 32 * (warp & 3) + 16 * wg + (lane & 15);  // TMEM lane = query row in the CTA
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3) + 16 * wg) << 16);
+    const int nchunk2 = p.kp2 / 32;
     uint32_t it = 0, tcount = 0;
     PairRange rr{u_first, u_end};
     int t, jb, je;
@@ -316,6 +315,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
       const int nk = je - jb;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
+      int o_done = 0;  // P V of this segment's key tiles [0, o_done) waited for
+      auto wait_pv = [&](int t2) {
+        const uint32_t g2 = it + t2;
+        return mbar_wait(&bar_o_full[g2 & 1], (g2 >> 1) & 1, p.ctl, abort);
+      };
       for (int jj = 0; jj < nk; ++jj) {
         const uint32_t g = it + jj;
         const int buf = g & 1;
@@ -325,49 +329,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
           break;
         }
         tc_fence_after();
-        float x[NC][32];
-        const uint32_t sa = lane_addr(tmem, warp, buf * 128 + col0);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, reinterpret_cast<uint32_t(&)[32]>(x[c]));
+        float x[64];  // S columns 64 half + i
+        tmem_ld16x2_32<64>(tl + buf * 128, reinterpret_cast<uint32_t(&)[32]>(x[0]));
+        tmem_ld16x2_32<64>(tl + buf * 128 + 32, reinterpret_cast<uint32_t(&)[32]>(x[32]));
         tmem_ld_wait();
         if (nkeys < 128) {
 #pragma unroll
-          for (int c = 0; c < NC; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + 32 * c + i >= nkeys) x[c][i] = -INFINITY;
+          for (int i = 0; i < 64; ++i)
+            if (64 * half + i >= nkeys) x[i] = -INFINITY;
         }
-        float mx = max_tree3<NC * 32>(reinterpret_cast<const float(&)[NC * 32]>(x));
-        if (NWG > 1) {
-          s_pmax[g & 1][wg][lrow] = mx;
-          mbar_arrive(&bar_xmax);
-          if (!mbar_wait(&bar_xmax, g & 1, p.ctl, abort)) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int w = 0; w < NWG; ++w) mx = fmaxf(mx, s_pmax[g & 1][w][lrow]);
-        }
+        float mx = max_tree3<64>(x);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m, mx * p.scale_log2);
         const bool need = m_new > m + 8.0f;
-        // one wait on O per key tile keeps the parity wait in step
-        bool o_pending = jj > 0;
+        // O-complete waits.  The P V of key tile g commits to bar_o_full[g & 1];
+        // a parity wait for it is exact while the P V two tiles later cannot have
+        // completed yet, which holds for every P V before the current tile's
+        // (that one needs this thread's P first).  Each P V is waited for once,
+        // in order: normally two tiles behind, where it never blocks; rescaling O
+        // needs the previous tile's P V complete first.
         if (jj > 0 && __any_sync(0xffffffffu, need)) {
-          if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+          bool waited = true;
+          for (; o_done < jj; ++o_done)
+            if (!wait_pv(o_done)) {
+              waited = false;
+              break;
+            }
+          if (!waited) {
             ok = false;
             break;
           }
-          o_pending = false;
           tc_fence_after();
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
-          const uint32_t oa = lane_addr(tmem, warp, 256);
-          for (int c = wg; c < nchunk; c += NWG) {
+          for (int c = 0; c < nchunk2; ++c) {
             uint32_t o[16];
-            tmem_ld16(oa + 16 * c, o);
+            tmem_ld16x2_16<16>(tl + 256 + 32 * c, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st16(oa + 16 * c, o);
+            tmem_st16x2_16<16>(tl + 256 + 32 * c, o);
           }
           tmem_st_wait();
           l *= f;
@@ -377,24 +377,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         }
         const float neg_m = -m;
         float rs[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[NC][16];
+        uint32_t pk[2][16];  // P as bf16 pairs: words [32 half, 32 half + 32) of the row
 #pragma unroll
-        for (int c = 0; c < NC; ++c)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
-            const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], p.scale_log2, neg_m));
-            if (!kSumCol) rs[i & 3] += a0 + a1;
-            pk[c][i] = pack_bf16x2(a0, a1);
-          }
+        for (int i = 0; i < 32; ++i) {
+          const float a0 = ex2_approx(fmaf(x[2 * i], p.scale_log2, neg_m));
+          const float a1 = ex2_approx(fmaf(x[2 * i + 1], p.scale_log2, neg_m));
+          if (!kSumCol) rs[i & 3] += a0 + a1;
+          pk[i >> 4][i & 15] = pack_bf16x2(a0, a1);
+        }
         l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        const uint32_t pa = lane_addr(tmem, warp, buf * 128 + col0 / 2);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
+        tmem_st16x2_16<32>(tl + buf * 128, pk[0]);
+        tmem_st16x2_16<32>(tl + buf * 128 + 16, pk[1]);
         tmem_st_wait();
-        if (o_pending && !mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
-          ok = false;
-          break;
+        if (o_done + 2 <= jj) {
+          // the P V of two key tiles back
+          if (!wait_pv(o_done)) {
+            ok = false;
+            break;
+          }
+          ++o_done;
         }
         tc_fence_before();
         __syncwarp();
@@ -404,35 +405,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         }
       }
       if (!ok) break;
-      const uint32_t glast = it + nk - 1;
-      if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
+      // the remaining P V of the segment, in order, end with the last one
+      for (; o_done < nk; ++o_done)
+        if (!wait_pv(o_done)) {
+          ok = false;
+          break;
+        }
+      if (!ok) break;
       tc_fence_after();
       if (kSumCol) {
-        // the row sum is O's column sum_col (this thread's TMEM lane)
-        const uint32_t lv = tmem_ld1(lane_addr(tmem, warp, 256 + p.sum_col));
+        // the row sum is O's column sum_col: read at split 1 from column
+        // sum_col - 1 (half 0) and sum_col (half 1), which keeps the access
+        // inside TMEM for every k, and taken from half 1
+        const uint32_t lv = tmem_ld16x2_1<1>(tl + 256 + p.sum_col - 1);
         tmem_ld_wait();
-        l = __uint_as_float(lv);
-      } else if (NWG > 1) {
-        s_psum[wg][lrow] = l;
-        mbar_arrive(&bar_xsum);
-        if (!mbar_wait(&bar_xsum, tcount & 1, p.ctl, abort)) break;
-        l = 0.f;
-#pragma unroll
-        for (int w = 0; w < NWG; ++w) l += s_psum[w][lrow];
+        l = __shfl_sync(0xffffffffu, __uint_as_float(lv), (lane & 15) + 16);
+      } else {
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
       }
       const int row = row0 + lrow;
       const bool live = row < p.nq;
-      const uint32_t oa = lane_addr(tmem, warp, 256);
       if (jb == 0 && je == p.nkt) {
         // every key tile of this query tile was processed here: O / l and lse
         float* optr = p.O + (size_t)(live ? row : 0) * p.ldo;
         const float inv = 1.0f / l;
-        for (int c = wg; c < nchunk; c += NWG) {
+        for (int c = 0; c < nchunk2; ++c) {
           uint32_t o[16];
-          tmem_ld16(oa + 16 * c, o);
+          tmem_ld16x2_16<16>(tl + 256 + 32 * c, o);
           tmem_ld_wait();
           if (live) {
-            const int c0 = 16 * c;
+            const int c0 = 32 * c + 16 * half;
             if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
 #pragma unroll
               for (int i = 0; i < 16; i += 4)
@@ -446,7 +448,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
             }
           }
         }
-        if (live && wg == 0) p.lse[row] = (m + log2f(l)) * kLn2;
+        if (live && half == 0) p.lse[row] = (m + log2f(l)) * kLn2;
       } else {
         // the query tile's key tiles are split between pairs: the unnormalised
         // O, the running max and the sum go to this pair's slot for the merge
@@ -455,17 +457,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(96 + 128 * NWG, 1)
         float* ps = p.part + (size_t)slot * part_slot_floats(p.kp2);
         const int prow = 128 * (int)rank + lrow;
         float* po = ps + (size_t)prow * p.kp2;
-        for (int c = wg; c < nchunk; c += NWG) {
+        for (int c = 0; c < nchunk2; ++c) {
           uint32_t o[16];
-          tmem_ld16(oa + 16 * c, o);
+          tmem_ld16x2_16<16>(tl + 256 + 32 * c, o);
           tmem_ld_wait();
+          const int c0 = 32 * c + 16 * half;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(po + 16 * c + i) =
+            *reinterpret_cast<float4*>(po + c0 + i) =
                 make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
                             __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
         }
-        if (wg == 0) {
+        if (half == 0) {
           ps[(size_t)256 * p.kp2 + prow] = m;
           ps[(size_t)256 * p.kp2 + 256 + prow] = l;
         }
