@@ -34,7 +34,7 @@ __device__ __forceinline__ double load_elem(const void* F, size_t i) {
 // Offsets are clamped into [0, n] and member indices outside [0, n) skipped;
 // either sets the bad-index bit of the status word.
 constexpr int kPoolStage = 1024;  // member indices staged per round
-constexpr int kPoolBatch = 16;    // loads in flight per thread
+constexpr int kPoolBatch = 32;    // loads in flight per thread
 template <bool F32>
 __global__ void pool_kernel(const void* __restrict__ F, int ld, int n, int d,
                             const int* __restrict__ off, const int* __restrict__ mem,

@@ -10,6 +10,8 @@
 // vector accesses, one warp per row.
 #include <algorithm>
 
+#include <type_traits>
+
 #include "internal.h"
 
 namespace ssc {
@@ -72,6 +74,46 @@ __global__ void gather_bf16_from_bf16(const __nv_bfloat16* __restrict__ in, int 
   }
 }
 
+// One thread per VEC-element piece of an output row (VEC = 8: 16-byte pieces,
+// 4: 8-byte pieces); every piece is an independent, aligned copy, so the whole
+// matrix moves with full coalescing and no per-row dependency chain.  Padding
+// columns [cols, out_ld) are zero except ones_col (when >= 0), which is one.
+template <int VEC>
+__global__ void gather_bf16_pieces(const __nv_bfloat16* __restrict__ in, int in_ld,
+                                   const int* __restrict__ map, int rows, int src_rows, int cols,
+                                   __nv_bfloat16* __restrict__ out, int out_ld, int ones_col,
+                                   unsigned* status) {
+  using Vec = typename std::conditional<VEC == 8, uint4, uint2>::type;
+  const int pieces = out_ld / VEC;
+  const long long total = (long long)rows * pieces;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / pieces);
+    const int c0 = (int)(i - (long long)r * pieces) * VEC;
+    const int src = checked_src(map, r, src_rows, status);
+    Vec* o = reinterpret_cast<Vec*>(out + (size_t)r * out_ld + c0);
+    if (src >= 0 && c0 + VEC <= cols) {
+      *o = __ldg(reinterpret_cast<const Vec*>(in + (size_t)src * in_ld + c0));
+    } else {
+      uint32_t w[VEC / 2];  // bf16 pairs, element 2q in the low half of word q
+#pragma unroll
+      for (int q = 0; q < VEC / 2; ++q) {
+        uint32_t h[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c0 + 2 * q + e;
+          const __nv_bfloat16 b = (src >= 0 && c < cols) ? in[(size_t)src * in_ld + c]
+                                                         : __float2bfloat16(c == ones_col ? 1.f : 0.f);
+          h[e] = __bfloat16_as_ushort(b);
+        }
+        w[q] = h[0] | (h[1] << 16);
+      }
+      if constexpr (VEC == 8) *o = make_uint4(w[0], w[1], w[2], w[3]);
+      else *o = make_uint2(w[0], w[1]);
+    }
+  }
+}
+
 __global__ void gather_bf16_from_f32(const float* __restrict__ in, int in_ld,
                                      const int* __restrict__ map, int rows, int src_rows, int cols,
                                      __nv_bfloat16* __restrict__ out, int out_ld, unsigned* status) {
@@ -103,7 +145,7 @@ __global__ void bwd_prep_kernel(const float* __restrict__ dO, int lddo, const fl
                                 int ldo, const float* __restrict__ lse, const int* __restrict__ map,
                                 int rows, int src_rows, int k, __nv_bfloat16* __restrict__ dOb,
                                 int ldb, float* __restrict__ dOf, int ldf, float* __restrict__ D,
-                                float* __restrict__ lse_out, unsigned* status) {
+                                float* __restrict__ lse_out, int vec4, unsigned* status) {
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
@@ -112,7 +154,27 @@ __global__ void bwd_prep_kernel(const float* __restrict__ dO, int lddo, const fl
     const float* g = dO + (size_t)src * lddo;
     const float* o = O + (size_t)src * ldo;
     float acc = 0.f;
-    for (int c = lane; c < k; c += 32) {
+    if (vec4) {
+      // 4 columns per lane and step: 16-byte loads of dO and O, 8-byte bf16 stores
+      for (int c4 = lane; c4 < (k >> 2); c4 += 32) {
+        float4 v = src0 < 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
+                            : __ldg(reinterpret_cast<const float4*>(g) + c4);
+        const float4 ov = __ldg(reinterpret_cast<const float4*>(o) + c4);
+        if (dOb) {
+          const __nv_bfloat162 b01 = __floats2bfloat162_rn(v.x, v.y);
+          const __nv_bfloat162 b23 = __floats2bfloat162_rn(v.z, v.w);
+          reinterpret_cast<uint2*>(dOb + (size_t)r * ldb)[c4] =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b01), *reinterpret_cast<const uint32_t*>(&b23));
+          v = make_float4(__low2float(b01), __high2float(b01), __low2float(b23), __high2float(b23));
+        }
+        if (dOf) reinterpret_cast<float4*>(dOf + (size_t)r * ldf)[c4] = v;
+        acc = fmaf(v.x, ov.x, acc);
+        acc = fmaf(v.y, ov.y, acc);
+        acc = fmaf(v.z, ov.z, acc);
+        acc = fmaf(v.w, ov.w, acc);
+      }
+    }
+    for (int c = (vec4 ? (k & ~3) : 0) + lane; c < k; c += 32) {
       float v = src0 < 0 ? 0.f : g[c];
       if (dOb) {
         __nv_bfloat16 b = __float2bfloat16(v);
@@ -328,6 +390,19 @@ cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const
     const int vec_ok = (in_ld % 8 == 0 && out_ld % 8 == 0 && ia % 16 == 0 && oa % 16 == 0)
                            ? 2
                            : (in_ld % 4 == 0 && out_ld % 4 == 0 && ia % 8 == 0 && oa % 8 == 0) ? 1 : 0;
+    if (vec_ok) {
+      const long long total = (long long)rows * (out_ld / (vec_ok == 2 ? 8 : 4));
+      const int gb = (int)std::max<long long>(1, std::min<long long>((total + 255) / 256, 148LL * 16));
+      const auto* ib = static_cast<const __nv_bfloat16*>(in);
+      if (vec_ok == 2)
+        gather_bf16_pieces<8><<<gb, 256, 0, st>>>(ib, in_ld, map, rows, src_rows, cols, out, out_ld,
+                                                  ones_col, status);
+      else
+        gather_bf16_pieces<4><<<gb, 256, 0, st>>>(ib, in_ld, map, rows, src_rows, cols, out, out_ld,
+                                                  ones_col, status);
+      count_launch();
+      return cudaGetLastError();
+    }
     gather_bf16_from_bf16<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), in_ld, map,
                                              rows, src_rows, cols, out, out_ld, vec_ok, ones_col,
                                              status);
@@ -384,8 +459,13 @@ cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, 
                             int ldb, float* dOf, int ldf, float* D, float* lse_out,
                             unsigned* status, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  // 16-byte row pieces of dO and O (and 8-byte bf16 / 16-byte fp32 output pieces)
+  const auto a16 = [](const void* q) { return reinterpret_cast<uintptr_t>(q) % 16 == 0; };
+  const int vec4 = lddo % 4 == 0 && ldo % 4 == 0 && a16(dO) && a16(O) &&
+                   (!dOb || (ldb % 4 == 0 && reinterpret_cast<uintptr_t>(dOb) % 8 == 0)) &&
+                   (!dOf || (ldf % 4 == 0 && a16(dOf)));
   bwd_prep_kernel<<<grid_for(rows, 8), 256, 0, st>>>(dO, lddo, O, ldo, lse, map, rows, src_rows, k,
-                                                      dOb, ldb, dOf, ldf, D, lse_out, status);
+                                                      dOb, ldb, dOf, ldf, D, lse_out, vec4, status);
   count_launch();
   return cudaGetLastError();
 }
