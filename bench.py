@@ -345,6 +345,30 @@ def run_ours(args, ws, rank, local):
     h2d = sum(host[x].numel() * host[x].element_size() for x in ("Q", "K", "V", "dO"))
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
 
+    # ---- the backward with dV as well (the dV pass after the dQ/dK kernel),
+    # timed after the main region on the same resident inputs, L2 flushed
+    with_dv = None
+    if not args.need_dv:
+        _, bpp_dv = pair_flops(d, k, True)
+        O1, lse1 = api.ssc_dense_coupling_fwd(Q, K, V, scale, workspace=wsb)
+        dv_steps = max(2, min(args.steps, 5))
+        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(dv_steps)]
+        for s in range(dv_steps):
+            flush.zero_()
+            dev_ev[s][0].record(stream)
+            api.ssc_dense_coupling_bwd(Q, K, V, O1, lse1, dO, scale, need_dV=True, workspace=wsb)
+            dev_ev[s][1].record(stream)
+        torch.cuda.synchronize()
+        bwd_dv_ms = max_over_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in dev_ev])), ws)
+        step_dv_ms = float(np.mean(fwd_ms)) + bwd_dv_ms
+        with_dv = {"bwd_ms": round(bwd_dv_ms, 4), "step_ms": round(step_dv_ms, 4),
+                   "tflops": round(float(n) * n * (fpp + bpp_dv) / (step_dv_ms * 1e-3) / 1e12, 2),
+                   "bwd_tflops": round(float(n) * n * bpp_dv / (bwd_dv_ms * 1e-3) / 1e12, 2),
+                   "flops_per_step": float(n) * n * (fpp + bpp_dv), "steps": dv_steps,
+                   "note": "need_dV = 1: dQ/dK kernel + dV pass; step = forward (main region) "
+                           "+ this backward"}
+        barrier(ws)
+
     pk = peaks()
     tflops = ws * flops_step / (dense_ms * 1e-3) / 1e12
     # dominant kernel: the dQ/dK backward kernel (2/3 of the flops), its average
@@ -381,7 +405,8 @@ def run_ours(args, ws, rank, local):
                   "fwd_kernel_ms": round(kfwd_ms / max(kfwd_n, 1), 4),
                   "bwd_kernel_ms": round(kbwd_mean, 4),
                   "frac_of_peak": round(tflops / ws / pk["tflops"], 4),
-                  "peak_gib": round(peak_gib, 3)},
+                  "peak_gib": round(peak_gib, 3),
+                  "with_dV": with_dv},
         "roofline": {"bound": "tensor", "kernel": "tc_bwd_dqk_kernel (dense backward, dQ and dK)",
                      "achieved": round(achieved, 2), "peak": pk["tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / pk["tflops"], 4), "peak_source": pk["source"] +
