@@ -1513,6 +1513,352 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   }
 }
 
+// ------------------------------------------------------------------ backward, dV (dense)
+// Key-stationary dV = P^T dO for the dense coupling: a CTA holds one key tile
+// K_j (128 keys) and streams the query row tiles i past it,
+//   S^T = K_j Q_i^T                (SS, both K-major)   -> TMEM [0,128) / [128,256)
+//   P^T = exp2(S^T s log2e - lse_i log2e)  per column i (the softmax of row i is
+//         already normalised by its lse: no running max, no row sum)
+//   dV_j += P^T dO_i               (TS: P^T from TMEM, dO_i MN-major) -> TMEM [256, 256 + kp)
+// so dV accumulates on chip and leaves once per key tile; no partial dV per
+// (row tile, key tile) goes through L2 reductions.  Units (key tile, row tile)
+// are numbered key-tile-major and split evenly over the CTAs; a key tile whose
+// row tiles two CTAs share is added into dV atomically by both.
+// Warps: 0 producer (K_j once per key tile; Q_i into a 2-stage ring), 1 MMA
+// issuer and TMEM owner, 2..2+4 NWG-1 the P^T warpgroups (thread = key row,
+// the warpgroups split the 128 query columns and nothing orders them against
+// each other, so each packs its bf16 P^T over its own S columns only),
+// 2+4 NWG the dO producer, whose
+// 32 lanes also stage lse_i log2e of the tile's rows in shared memory (+inf
+// past the last row, which zeroes those columns of P^T).
+struct DvRange {
+  int t, j, left;  // key tile, first row tile in it, units still to do
+};
+__device__ __forceinline__ bool dv_next(DvRange& r, int nkt, int nrt, int& t, int& jb, int& je) {
+  if (r.left <= 0 || r.t >= nkt) return false;
+  const int take = min(nrt - r.j, r.left);
+  t = r.t;
+  jb = r.j;
+  je = r.j + take;
+  r.left -= take;
+  ++r.t;
+  r.j = 0;
+  return true;
+}
+
+template <int NWG, int QCH, int VF, int VR>
+__global__ void __launch_bounds__(96 + 128 * NWG, 1)
+    tc_dv_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr bool kFixed = QCH > 0;
+  const int qch = kFixed ? QCH : p.qch;
+  const int vf = kFixed ? VF : p.vf;
+  const int vr = kFixed ? VR : p.vr;
+  const int d16 = kFixed ? 4 * QCH : p.d / 16;
+  constexpr int CW = 128 / NWG;  // query columns per P^T thread
+  constexpr int NC = CW / 32;
+  constexpr int NSM = 128 * NWG;
+  constexpr int kGWarp = 2 + 4 * NWG;  // dO producer
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_k_full, bar_k_empty, bar_q_full[2], bar_q_empty[2], bar_g_full[2],
+      bar_g_empty[2], bar_l_full[2], bar_s_full[2], bar_p_full[2], bar_dv_full, bar_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ __align__(16) float s_lse2[2][128];  // lse_i log2e of the stage's rows
+  __shared__ int s_range[3];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
+  const int qbytes = qch * kChunk;
+  const int gbytes = vtile_bytes(vf, vr);
+  const uint32_t sK = sbase;             // the stationary key tile
+  const uint32_t sQ0 = sK + qbytes;      // Q stage s at sQ0 + s * qbytes
+  const uint32_t sG0 = sQ0 + 2 * qbytes; // dO stage s at sG0 + s * gbytes
+  const int nkt = (p.nk + 127) / 128, nrt = (p.nq + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_k_full, 1);
+    mbar_init(&bar_k_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_q_full[i], 1);
+      mbar_init(&bar_q_empty[i], 1);
+      mbar_init(&bar_g_full[i], 1);
+      mbar_init(&bar_g_empty[i], 1);
+      mbar_init(&bar_l_full[i], 32);
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_p_full[i], NSM);
+    }
+    mbar_init(&bar_dv_full, 1);
+    mbar_init(&bar_drain, 1);
+    s_abort = 0;
+    fence_barrier_init();
+    const long long U = (long long)nkt * nrt;
+    const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+    const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+    s_range[0] = nrt > 0 ? (int)(u0 / nrt) : 0;
+    s_range[1] = nrt > 0 ? (int)(u0 % nrt) : 0;
+    s_range[2] = (int)(u1 - u0);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm.q);
+    tma_prefetch_desc(&tm.k);
+    tma_prefetch_desc(&tm.g);
+    if (vr) tma_prefetch_desc(&tm.gr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+
+  if (warp == 0) {
+    // ---------------- producer: K_j once per key tile, Q_i into a 2-stage ring
+    if (lane == 0) {
+      uint32_t g = 0, tcount = 0;
+      int k_issued = -1;
+      bool ok = true;
+      DvRange r{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && !*abort && dv_next(r, nkt, nrt, t, jb, je)) {
+        if (tcount > 0 && !mbar_wait(&bar_k_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        mbar_arrive_expect_tx(&bar_k_full, qbytes);
+        for (int c = 0; c < qch; ++c)
+          tma_load_2d(gptr(sK) + c * kChunk, &tm.k, 64 * c, 128 * t, &bar_k_full);
+        k_issued = (int)tcount;
+        for (int j = jb; j < je; ++j, ++g) {
+          const int st = g & 1;
+          if (g >= 2 && !mbar_wait(&bar_q_empty[st], ((g >> 1) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_q_full[st], qbytes);
+          for (int c = 0; c < qch; ++c)
+            tma_load_2d(gptr(sQ0 + st * qbytes) + c * kChunk, &tm.q, 64 * c, 128 * j, &bar_q_full[st]);
+        }
+        ++tcount;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        if (k_issued >= 0) mbar_wait(&bar_k_full, k_issued & 1, p.ctl, &never);
+        for (uint32_t h = g >= 2 ? g - 2 : 0; h < g; ++h)
+          mbar_wait(&bar_q_full[h & 1], (h >> 1) & 1, p.ctl, &never);
+      }
+    }
+  } else if (warp == kGWarp) {
+    // ---------------- producer: dO_i into a 2-stage ring (lane 0) and the
+    // stage's lse_i log2e (all lanes)
+    uint32_t g = 0;
+    bool ok = true;
+    DvRange r{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && !*abort && dv_next(r, nkt, nrt, t, jb, je)) {
+      for (int j = jb; j < je; ++j, ++g) {
+        const int st = g & 1;
+        if (g >= 2 && !mbar_wait(&bar_g_empty[st], ((g >> 1) - 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_g_full[st], gbytes);
+          uint8_t* dg = gptr(sG0 + st * gbytes);
+          for (int c = 0; c < vf; ++c)
+            tma_load_2d(dg + c * kChunk, &tm.g, 64 * c, 128 * j, &bar_g_full[st]);
+          if (vr) tma_load_2d(dg + vf * kChunk, &tm.gr, 64 * vf, 128 * j, &bar_g_full[st]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = 128 * j + 32 * q + lane;
+          s_lse2[st][32 * q + lane] = row < p.nq ? p.lse_in[row] * kLog2e : INFINITY;
+        }
+        mbar_arrive(&bar_l_full[st]);
+      }
+    }
+    if (*abort && lane == 0) {
+      volatile int never = 0;
+      for (uint32_t h = g >= 2 ? g - 2 : 0; h < g; ++h)
+        mbar_wait(&bar_g_full[h & 1], (h >> 1) & 1, p.ctl, &never);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (vf > 0 ? vf : 1), 0, 1);
+      const uint32_t idesc_pvr = make_idesc_bf16(128, vr > 0 ? vr : 16, 0, 1);
+      const uint32_t dv_col = tmem + 256;
+      const uint32_t rsw = rem_swizzle(vr);
+      const uint32_t rrow = (uint32_t)vr * 2;  // bytes per row of the remainder box
+      uint32_t g0 = 0, tcount = 0;
+      bool ok = true;
+      // S^T_g = K_j Q_g^T into S buffer g & 1 (Q stage g & 1)
+      auto issue_s = [&](uint32_t g) -> bool {
+        const int st = g & 1;
+        if (!mbar_wait(&bar_q_full[st], (g >> 1) & 1, p.ctl, abort)) return false;
+        tc_fence_after();
+        const uint32_t sq = sQ0 + st * qbytes;
+        const uint32_t d_tmem = tmem + st * 128;
+#pragma unroll
+        for (int kk = 0; kk < d16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+          mma_ss(d_tmem, make_sdesc(sK + off, 16, 1024, kSw128), make_sdesc(sq + off, 16, 1024, kSw128),
+                 idesc_s, kk > 0);
+        }
+        mma_commit(&bar_s_full[st]);
+        mma_commit(&bar_q_empty[st]);
+        return true;
+      };
+      DvRange r{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && dv_next(r, nkt, nrt, t, jb, je)) {
+        const int nu = je - jb;
+        if (!mbar_wait(&bar_k_full, tcount & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < min(2, nu) && ok; ++j) ok = issue_s(g0 + j);
+        for (int j = 0; j < nu && ok; ++j) {
+          const uint32_t g = g0 + j;
+          const int buf = g & 1;
+          if (!mbar_wait(&bar_p_full[buf], (g >> 1) & 1, p.ctl, abort) ||
+              !mbar_wait(&bar_g_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // dV += P^T dO_g : A = P^T (bf16 pairs, each warpgroup's CW query
+          // columns packed at the start of its own CW S columns), B = dO_g MN-major
+          const uint32_t sg = sG0 + buf * gbytes;
+          const uint32_t a_tmem = tmem + buf * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t pcol = 8 * kk + ((16 * kk) / CW) * (CW / 2);
+            if (vf > 0)
+              mma_ts(dv_col, a_tmem + pcol, make_sdesc(sg + kk * 2048, kChunk, 1024, kSw128),
+                     idesc_pv, acc);
+            if (vr > 0)
+              mma_ts(dv_col + 64 * vf, a_tmem + pcol,
+                     make_sdesc(sg + vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+                     idesc_pvr, acc);
+          }
+          mma_commit(&bar_g_empty[buf]);
+          if (j + 2 < nu) ok = issue_s(g + 2);
+        }
+        if (!ok) break;
+        mma_commit(&bar_k_empty);
+        mma_commit(&bar_dv_full);
+        g0 += nu;
+        ++tcount;
+      }
+      // drain: wait until every tensor-core op issued here has completed
+      mma_commit(&bar_drain);
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
+    }
+  } else if (warp >= 2 && warp < kGWarp) {
+    // ---------------- P^T (NWG warpgroups): thread = key row (TMEM lane); the
+    // warpgroups split the 128 query columns; epilogue dV per key tile
+    const int wg = (warp - 2) >> 2;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int col0 = wg * CW;
+    const int nchunk = p.kp / 16;
+    uint32_t g0 = 0, tcount = 0;
+    bool ok = true;
+    DvRange r{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && dv_next(r, nkt, nrt, t, jb, je)) {
+      const int nu = je - jb;
+      for (int j = 0; j < nu; ++j) {
+        const uint32_t g = g0 + j;
+        const int buf = g & 1;
+        if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort) ||
+            !mbar_wait(&bar_l_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t x[NC][32];
+        const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, x[c]);
+        tmem_ld_wait();
+        // P^T = exp2(S^T s log2e - lse_i log2e); columns past the last query row
+        // carry lse = +inf and give 0
+        const float4* l4 = reinterpret_cast<const float4*>(&s_lse2[buf][col0]);
+        uint32_t pk[NC][16];
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 lv = l4[8 * c + q];
+            const float a0 = ex2_approx(fmaf(__uint_as_float(x[c][4 * q]), p.scale_log2, -lv.x));
+            const float a1 = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 1]), p.scale_log2, -lv.y));
+            const float a2 = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 2]), p.scale_log2, -lv.z));
+            const float a3 = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 3]), p.scale_log2, -lv.w));
+            pk[c][2 * q] = pack_bf16x2(a0, a1);
+            pk[c][2 * q + 1] = pack_bf16x2(a2, a3);
+          }
+        // packed into the first half of this warpgroup's own S columns (already
+        // read by this thread): the other warpgroup may still be reading its S
+        const uint32_t pa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[buf]);
+      }
+      if (!ok) break;
+      // epilogue: the key tile's dV rows; a key tile shared with another CTA is
+      // added atomically (dV is zeroed by the caller)
+      if (!mbar_wait(&bar_dv_full, tcount & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      const int key = 128 * t + lrow;
+      const bool live = key < p.nk;
+      const bool whole = jb == 0 && je == nrt;
+      float* dst = p.dV + (size_t)(live ? key : 0) * p.lddv;
+      const uint32_t da = tmem_lane_addr(tmem, warp, 256);
+      for (int c = wg; c < nchunk; c += NWG) {
+        uint32_t o[16];
+        tmem_ld16(da + 16 * c, o);
+        tmem_ld_wait();
+        if (!live) continue;
+        const int c0 = 16 * c;
+        if (c0 + 16 <= p.k && p.vec_atomics) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 v = make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
+                                         __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
+            if (whole) *reinterpret_cast<float4*>(dst + c0 + i) = v;
+            else atomicAdd(reinterpret_cast<float4*>(dst + c0 + i), v);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < p.k) {
+              if (whole) dst[c0 + i] = __uint_as_float(o[i]);
+              else atomicAdd(dst + c0 + i, __uint_as_float(o[i]));
+            }
+        }
+      }
+      g0 += nu;
+      ++tcount;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 __global__ void wait_probe_kernel(WaitCtl ctl) {
   __shared__ uint64_t bar;
   __shared__ int s_abort;
@@ -1740,6 +2086,52 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_tc_dv_dense(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
+                               const __nv_bfloat16* dOb, int lddob, const float* lse, int nN,
+                               int nM, int d, int k, float scale, float* dV, int lddv,
+                               cudaStream_t st, const WaitCtl& ctl) {
+  TcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.Q = Q;
+  a.K = K;
+  a.ldq = ldq;
+  a.ldk = ldk;
+  a.nQrows = nN;
+  a.nKrows = nM;
+  a.d = d;
+  a.k = k;
+  a.scale = scale;
+  TcParams p;
+  fill_common(a, p);
+  p.lse_in = lse;
+  p.dV = dV;
+  p.lddv = lddv;
+  p.ctl = ctl;
+  p.vec_atomics = (lddv % 4 == 0) && (reinterpret_cast<uintptr_t>(dV) % 16 == 0);
+  TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (!make_map(&tm.q, Q, nN, d, ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.k, K, nM, d, ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.g, dOb, nN, k, lddob, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (p.vr && !make_map(&tm.gr, dOb, nN, k, lddob, p.vr, rem_sw_host(p.vr))) return cudaErrorInvalidValue;
+  const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
+  auto kern = fixed ? tc_dv_kernel<2, 2, 3, 16> : tc_dv_kernel<2, 0, 0, 0>;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  // K tile, two Q stages, two dO stages (at most 230,400 bytes for d = 128, k = 256)
+  const int smem = 1024 + 3 * p.qch * kChunk + 2 * vtile_bytes(p.vf, p.vr);
+  if (smem + (int)fa.sharedSizeBytes > smem_optin()) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  prof_launch_begin(st);
+  kern<<<num_sms(), 96 + 128 * 2, smem, st>>>(tm, p);
+  prof_launch_end(st, SSC_PROF_BWD_DV);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl) {

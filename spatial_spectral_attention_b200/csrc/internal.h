@@ -170,6 +170,13 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
 cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,
                           const float* D, float* dQ, int lddq, float* dK, int lddk, float* dV,
                           int lddv, cudaStream_t st, const WaitCtl& ctl, float* dK_ord = nullptr);
+// Dense dV = P^T dO on tensor cores, key-stationary (dV accumulated per key tile
+// on chip; no partial-dV reductions).  dOb: bf16 dO rows of kp columns, zero
+// padded; lse in row order; dV zeroed by the caller.
+cudaError_t launch_tc_dv_dense(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
+                               const __nv_bfloat16* dOb, int lddob, const float* lse, int nN,
+                               int nM, int d, int k, float scale, float* dV, int lddv,
+                               cudaStream_t st, const WaitCtl& ctl);
 // out[map[r]] = in[r] for r < rows (map entries outside [0, dst_rows) are dropped
 // and set the bad-index bit).
 cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, int rows,

@@ -361,7 +361,14 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
            ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
-  return cuda_status(launch_tc_bwd(a, w.dOb, kp, lse, w.D, dQ, lddq, dK, lddk, dV, lddv, st, ctl));
+  // dQ and dK query-stationary; dV key-stationary in a kernel of its own
+  if ((e = launch_tc_bwd(a, w.dOb, kp, lse, w.D, dQ, lddq, dK, lddk, nullptr, 0, st, ctl)) !=
+      cudaSuccess)
+    return SSC_ERR_CUDA;
+  if (!dV) return SSC_OK;
+  return cuda_status(launch_tc_dv_dense(static_cast<const __nv_bfloat16*>(Q), ldq,
+                                        static_cast<const __nv_bfloat16*>(K), ldk, w.dOb, kp, lse, nN,
+                                        nM, d, k, scale, dV, lddv, st, ctl));
 }
 
 // ------------------------------------------------------------ geo

@@ -72,7 +72,10 @@ def test_dense_bf16_workload_ragged():
                                        (130, 260, 128, 32), (384, 129, 128, 196),
                                        # one query tile over 157 key tiles: the dense forward
                                        # splits it between every CTA pair and merges ~74 pieces
-                                       (200, 20000, 128, 196)])
+                                       (200, 20000, 128, 196),
+                                       # two row tiles over 313 key tiles: every CTA of the
+                                       # key-stationary dV pass runs through several key tiles
+                                       (256, 40000, 128, 196)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_dense_shapes(nN, nM, d, k, dtype):
     Qn, Kn, Vn, dOn = synth.random_inputs(nN, nM, d, k, seed=nN * 7 + nM, q_scale=0.5)
