@@ -41,6 +41,34 @@ def pair_flops(d, k, need_dv):
     return fwd, bwd
 
 
+# DRAM traffic of tc_bwd_dqk_kernel on the dense 60k workload, from one ncu
+# capture of this bench's own launch (dram__bytes_read.sum + dram__bytes_write.sum,
+# a 1-pass metric set; summary in profiles/tc_bwd_dqk_kernel_dense60k_dram.md).
+# It stands only while the kernel's source text is the one that was captured.
+DQK_TRAFFIC = {"kernel_sha256_16": "187ae6fa33bfecf9", "n": 60000, "d": 128, "k": 196,
+               "read_bytes": 209.80e6, "write_bytes": 67.15e6}
+
+
+def dqk_kernel_hash():
+    import hashlib
+    path = os.path.join(ROOT, "spatial_spectral_attention_b200", "csrc", "coupling_tc.cu")
+    try:
+        s = open(path).read()
+        i = s.index("template <int NCG, int QCH, int VF, int VR>\n__global__ void "
+                    "__launch_bounds__(128 * (2 + NCG), 1)\n    tc_bwd_dqk_kernel(")
+        j = s.index("\n}\n", i) + 3
+    except (OSError, ValueError):
+        return None
+    return hashlib.sha256(s[i:j].encode()).hexdigest()[:16]
+
+
+def dqk_traffic(n, d, k):
+    t = DQK_TRAFFIC
+    if (n, d, k) != (t["n"], t["d"], t["k"]) or dqk_kernel_hash() != t["kernel_sha256_16"]:
+        return None
+    return t["read_bytes"] + t["write_bytes"]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -413,7 +441,8 @@ def run_ours(args, ws, rank, local):
                      " burst bf16 (MEASURED_PEAKS.json bf16_tflops)",
                      "flops_per_launch": bwd_flops, "flop_convention": "executed (S recompute included)",
                      "achieved_model_flops": round(achieved_model, 2),
-                     "launches_timed": kbwd_n, "traffic": None},
+                     "launches_timed": kbwd_n, "traffic": dqk_traffic(n, d, k),
+                     "traffic_unit": "bytes per launch (DRAM read + write, ncu)"},
         "e2e": ({"value": round(ws * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                  "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
                  "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
