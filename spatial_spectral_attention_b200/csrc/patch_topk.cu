@@ -79,16 +79,108 @@ __global__ void pool_kernel(const void* __restrict__ F, int ld, int n, int d,
   }
 }
 
+// Row-staged pooling (rows of d * esize bytes, a multiple of 16, 16-byte
+// aligned): the block copies the patch's member rows into shared memory with
+// cp.async (16-byte pieces, kPoolRows rows per buffer, two buffers), so every
+// load of a chunk is in flight at once; each thread then adds its channels
+// over the staged rows strictly in member order (bit-identical to pool_kernel).
+constexpr int kPoolRows = 64;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(128) pool_rows_kernel(const void* __restrict__ F, int ld, int n,
+                                                        int d, const int* __restrict__ off,
+                                                        const int* __restrict__ mem,
+                                                        double* __restrict__ mu, unsigned* status) {
+  constexpr int kEsz = F32 ? 4 : 2;
+  extern __shared__ __align__(16) uint8_t s_rows[];  // [2][kPoolRows][d * kEsz]
+  __shared__ int s_mem[kPoolStage];
+  const int p = blockIdx.x;
+  int b = off[p], e = off[p + 1];
+  if (b < 0 || e <= b || e > n) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusBadIndex);
+    b = min(max(b, 0), n);
+    e = min(max(e, b), n);
+  }
+  const int rowb = d * kEsz;
+  const int pieces = rowb / 16;
+  const uint8_t* Fb = static_cast<const uint8_t*>(F);
+  const uint32_t sbase = smem_u32(s_rows);
+  const int c0 = threadIdx.x, c1 = threadIdx.x + 128;  // this thread's channels (d <= 256)
+  double s0 = 0.0, s1 = 0.0;
+  for (int r0 = b; r0 < e; r0 += kPoolStage) {
+    const int nr = min(kPoolStage, e - r0);
+    __syncthreads();  // the previous pass is done with s_mem and the row buffers
+    for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+      int v = mem[r0 + i];
+      if (v < 0 || v >= n) {
+        atomicOr(status, kStatusBadIndex);
+        v = -1;
+      }
+      s_mem[i] = v;
+    }
+    __syncthreads();
+    const int nch = (nr + kPoolRows - 1) / kPoolRows;
+    auto issue = [&](int k) {
+      const uint32_t buf = sbase + (uint32_t)((k & 1) * kPoolRows * rowb);
+      const int rows = min(kPoolRows, nr - k * kPoolRows);
+      for (int i = threadIdx.x; i < rows * pieces; i += blockDim.x) {
+        const int r = i / pieces, pc = i - r * pieces;
+        const int v = s_mem[k * kPoolRows + r];
+        if (v >= 0) cp_async16(buf + r * rowb + pc * 16, Fb + ((size_t)v * ld * kEsz + pc * 16));
+      }
+      cp_async_commit();
+    };
+    issue(0);
+    for (int k = 0; k < nch; ++k) {
+      if (k + 1 < nch) {
+        issue(k + 1);
+        cp_async_wait<1>();  // chunk k has landed (this thread's copies)
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();  // ... and every thread's
+      const uint8_t* buf = s_rows + (k & 1) * kPoolRows * rowb;
+      const int rows = min(kPoolRows, nr - k * kPoolRows);
+      for (int r = 0; r < rows; ++r) {
+        if (s_mem[k * kPoolRows + r] < 0) continue;
+        const uint8_t* row = buf + r * rowb;
+        if constexpr (F32) {
+          if (c0 < d) s0 = __dadd_rn(s0, (double)reinterpret_cast<const float*>(row)[c0]);
+          if (c1 < d) s1 = __dadd_rn(s1, (double)reinterpret_cast<const float*>(row)[c1]);
+        } else {
+          if (c0 < d)
+            s0 = __dadd_rn(s0, (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c0]));
+          if (c1 < d)
+            s1 = __dadd_rn(s1, (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c1]));
+        }
+      }
+      __syncthreads();  // buffer k & 1 is refilled by issue(k + 2)
+    }
+  }
+  const double cnt = (double)max(e - b, 1);
+  if (c0 < d) mu[(size_t)p * d + c0] = __ddiv_rn(s0, cnt);
+  if (c1 < d) mu[(size_t)p * d + c1] = __ddiv_rn(s1, cnt);
+}
+
 constexpr int kST = 32;  // score tile (target x source patches)
-constexpr int kSC = 16;  // channels staged per step
+constexpr int kSC = 128;  // channels staged per step (one load phase for d <= 128)
 
 // scores[p, q] for a 32 x 32 tile per block; each thread owns 4 outputs and
 // sums its products strictly in channel order.
 __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ muN, int PN,
                                                      const double* __restrict__ muM, int PM, int d,
                                                      double* __restrict__ sc) {
-  __shared__ double a[kST][kSC + 1];
-  __shared__ double b[kST][kSC + 1];
+  extern __shared__ double s_ab[];  // a[kST][kSC + 1], then b[kST][kSC + 1]
+  double(*a)[kSC + 1] = reinterpret_cast<double(*)[kSC + 1]>(s_ab);
+  double(*b)[kSC + 1] = reinterpret_cast<double(*)[kSC + 1]>(s_ab + kST * (kSC + 1));
   const int p0 = blockIdx.y * kST, q0 = blockIdx.x * kST;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of threads
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
@@ -190,19 +282,38 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   double* sc_ws = c.take<double>((size_t)PN * PM);
   double* sc = scores ? scores : sc_ws;
   const int pt = d >= 128 ? 128 : 64;
-  if (dtype == 1) {
-    pool_kernel<true><<<PN, pt, 0, st>>>(FN, ldn, nN, d, offN, memN, muN, status);
+  const int esz = dtype == 1 ? 4 : 2;
+  // rows staged through shared memory when they are whole 16-byte pieces
+  auto staged = [&](const void* F, int ld) {
+    return d <= 256 && (d * esz) % 16 == 0 && ((size_t)ld * esz) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(F) % 16 == 0;
+  };
+  const int rows_smem = 2 * kPoolRows * d * esz;
+  auto pool = [&](const void* F, int ld, int n, int P, const int* off, const int* mem, double* mu) {
+    cudaError_t e;
+    if (staged(F, ld)) {
+      auto kern = dtype == 1 ? pool_rows_kernel<true> : pool_rows_kernel<false>;
+      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem)) !=
+          cudaSuccess)
+        return e;
+      kern<<<P, 128, rows_smem, st>>>(F, ld, n, d, off, mem, mu, status);
+    } else if (dtype == 1) {
+      pool_kernel<true><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
+    } else {
+      pool_kernel<false><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
+    }
     count_launch();
-    pool_kernel<true><<<PM, pt, 0, st>>>(FM, ldm, nM, d, offM, memM, muM, status);
-    count_launch();
-  } else {
-    pool_kernel<false><<<PN, pt, 0, st>>>(FN, ldn, nN, d, offN, memN, muN, status);
-    count_launch();
-    pool_kernel<false><<<PM, pt, 0, st>>>(FM, ldm, nM, d, offM, memM, muM, status);
-    count_launch();
-  }
+    return cudaGetLastError();
+  };
+  cudaError_t pe;
+  if ((pe = pool(FN, ldn, nN, PN, offN, memN, muN)) != cudaSuccess) return pe;
+  if ((pe = pool(FM, ldm, nM, PM, offM, memM, muM)) != cudaSuccess) return pe;
   dim3 grid((PM + kST - 1) / kST, (PN + kST - 1) / kST);
-  scores_kernel<<<grid, 256, 0, st>>>(muN, PN, muM, PM, d, sc);
+  const int sc_smem = 2 * kST * (kSC + 1) * (int)sizeof(double);
+  if ((pe = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sc_smem)) != cudaSuccess)
+    return pe;
+  scores_kernel<<<grid, 256, sc_smem, st>>>(muN, PN, muM, PM, d, sc);
   count_launch();
   topk_kernel<<<PN, 256, 0, st>>>(sc, PM, R, topk);
   count_launch();
