@@ -182,7 +182,7 @@ def run_geo_sweep(api, synth, torch, dev, need_dv, fpp, bpp):
             O, lse = api.ssc_geo_coupling_fwd(Q, K, V, gp.scale, offN, memN, offM, memM, topk,
                                               workspace=gws)
             api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, gp.scale, offN, memN, offM, memM, topk,
-                                     need_dV=need_dv, workspace=gws)
+                                     need_dV=need_dv, workspace=gws, reuse_forward=True)
 
         for _ in range(2):
             step()
@@ -264,7 +264,7 @@ def run_ours(args, ws, rank, local):
                                           g["memN"], g["offM"], g["memM"], topk, workspace=g["ws"])
         api.ssc_geo_coupling_bwd(g["Q"], g["K"], g["V"], O, lse, g["dO"], gpair.scale, g["offN"],
                                  g["memN"], g["offM"], g["memM"], topk, need_dV=args.need_dv,
-                                 workspace=g["ws"])
+                                 workspace=g["ws"], reuse_forward=True)
         return topk
 
     clk = ClockSampler(local).__enter__()
@@ -464,7 +464,7 @@ def run_ours(args, ws, rank, local):
         res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_ms, 4),
                       "tflops": round(gflops / (geo_ms * 1e-3) / 1e12, 2),
                       "support_per_row": round(U, 1), "fps_ms_per_shape": round(geo["fps_ms"], 3),
-                      "note": "step = scores/top-R + fwd + bwd; FPS per shape, outside the step"}
+                      "note": "step = scores/top-R + fwd + bwd (the backward reuses the forward's patch-major operands and schedule from the workspace); FPS per shape, outside the step"}
     return res
 
 

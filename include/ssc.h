@@ -238,6 +238,28 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
                          float* dV, int lddv,
                          void* ws, size_t ws_bytes, ssc_stream_t stream);
 
+/* ssc_geo_coupling_bwd without rebuilding what ssc_geo_coupling_fwd left in  */
+/* the workspace: the patch-major copies of Q, K and V and the tile schedule  */
+/* (the saved state a training step keeps from its forward; the pages have   */
+/* no counterpart).  Same arguments and results as ssc_geo_coupling_bwd.     */
+/* Contract (not checked): ws is the workspace of a completed or earlier-     */
+/* enqueued ssc_geo_coupling_fwd call on the same stream with the same Q, K,  */
+/* V, sizes, dtype and patch tables, and nothing wrote to ws or to those      */
+/* inputs in between; otherwise the results are those of the stale copies.   */
+/* The backward itself overwrites only the workspace's backward buffers, so   */
+/* it can be called again on the same forward state.                         */
+int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk,
+                               const void* V, int ldv, int nN, int nM, int d, int k,
+                               float scale, int dtype,
+                               const int* offN, const int* memN, int PN,
+                               const int* offM, const int* memM, int PM,
+                               const int* topk, int R,
+                               const float* O, int ldo, const float* lse,
+                               const float* dO, int lddo,
+                               float* dQ, int lddq, float* dK, int lddk,
+                               float* dV, int lddv,
+                               void* ws, size_t ws_bytes, ssc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

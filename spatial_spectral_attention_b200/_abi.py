@@ -39,6 +39,9 @@ SIGNATURES = {
     "ssc_geo_coupling_bwd": (I, [P, I, P, I, P, I, I, I, I, I, F, I,
                                  P, P, I, P, P, I, P, I, P, I, P, P, I,
                                  P, I, P, I, P, I, P, Z, P]),
+    "ssc_geo_coupling_bwd_reuse": (I, [P, I, P, I, P, I, I, I, I, I, F, I,
+                                       P, P, I, P, P, I, P, I, P, I, P, P, I,
+                                       P, I, P, I, P, I, P, Z, P]),
 }
 
 _lib = None

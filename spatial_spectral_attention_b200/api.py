@@ -212,8 +212,13 @@ def ssc_geo_coupling_fwd(Q, K, V, scale, offN, memN, offM, memM, topk, workspace
 
 
 def ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, scale, offN, memN, offM, memM, topk,
-                         need_dV=False, workspace=None):
-    """Geo-FlashAttention backward: (dQ, dK, dV or None) in vertex order."""
+                         need_dV=False, workspace=None, reuse_forward=False):
+    """Geo-FlashAttention backward: (dQ, dK, dV or None) in vertex order.
+
+    reuse_forward=True calls ssc_geo_coupling_bwd_reuse: the patch-major
+    operands and the tile schedule are taken from `workspace`, which must be the
+    workspace the matching ssc_geo_coupling_fwd call used (same inputs and
+    tables, not written since)."""
     ldq, ldk, ldv, dt = _qkv(Q, K, V)
     PN, PM, R = _patches(offN, memN, offM, memM, topk)
     _cuda(O, lse, dO)
@@ -225,8 +230,14 @@ def ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, scale, offN, memN, offM, memM, top
     dV = torch.empty((nM, k), dtype=torch.float32, device=dev) if need_dV else None
     O, dO, lse, topk = O.contiguous(), dO.contiguous(), lse.contiguous(), topk.contiguous()
     nb = lib().ssc_geo_coupling_workspace_size(nN, nM, d, k, PN, PM, R, dt)
+    if reuse_forward:
+        if workspace is None or workspace.numel() < nb:
+            raise ValueError("reuse_forward needs the forward's workspace")
+        name = "ssc_geo_coupling_bwd_reuse"
+    else:
+        name = "ssc_geo_coupling_bwd"
     ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
-    check("ssc_geo_coupling_bwd", lib().ssc_geo_coupling_bwd(
+    check(name, getattr(lib(), name)(
         _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
         _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
         _ptr(O), O.stride(0), _ptr(lse), _ptr(dO), dO.stride(0),

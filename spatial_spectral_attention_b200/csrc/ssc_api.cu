@@ -442,12 +442,14 @@ int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const v
   return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
 }
 
-int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
-                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
-                         const int* memN, int PN, const int* offM, const int* memM, int PM,
-                         const int* topk, int R, const float* O, int ldo, const float* lse,
-                         const float* dO, int lddo, float* dQ, int lddq, float* dK, int lddk,
-                         float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+namespace {
+
+int geo_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN, int nM,
+            int d, int k, float scale, int dtype, const int* offN, const int* memN, int PN,
+            const int* offM, const int* memM, int PM, const int* topk, int R, const float* O,
+            int ldo, const float* lse, const float* dO, int lddo, float* dQ, int lddq, float* dK,
+            int lddk, float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream,
+            bool reuse) {
   int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
   if (rc) return rc;
   if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
@@ -461,8 +463,9 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const v
   WaitCtl ctl = make_ctl();
   GeoWs w;
   geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
-  if ((rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
-                      topk, R, w, st, ctl)))
+  // the patch-major operands and the schedule: rebuilt here, or left by the forward
+  if (!reuse && (rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM,
+                                memM, PM, topk, R, w, st, ctl)))
     return rc;
   cudaError_t e;
   if (dtype == SSC_F32) {
@@ -501,6 +504,31 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const v
                          dK, lddk, dV, lddv, st, ctl, w.dKg)) != cudaSuccess)
     return SSC_ERR_CUDA;
   return cuda_status(launch_scatter_rows_f32(w.dKg, d, memM, nM, nM, d, dK, lddk, ctl.status, st));
+}
+
+}  // namespace
+
+int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
+                         const int* memN, int PN, const int* offM, const int* memM, int PM,
+                         const int* topk, int R, const float* O, int ldo, const float* lse,
+                         const float* dO, int lddo, float* dQ, int lddq, float* dK, int lddk,
+                         float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  return geo_bwd(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, offN, memN, PN, offM, memM, PM,
+                 topk, R, O, ldo, lse, dO, lddo, dQ, lddq, dK, lddk, dV, lddv, ws, ws_bytes, stream,
+                 false);
+}
+
+int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk, const void* V,
+                               int ldv, int nN, int nM, int d, int k, float scale, int dtype,
+                               const int* offN, const int* memN, int PN, const int* offM,
+                               const int* memM, int PM, const int* topk, int R, const float* O,
+                               int ldo, const float* lse, const float* dO, int lddo, float* dQ,
+                               int lddq, float* dK, int lddk, float* dV, int lddv, void* ws,
+                               size_t ws_bytes, ssc_stream_t stream) {
+  return geo_bwd(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, offN, memN, PN, offM, memM, PM,
+                 topk, R, O, ldo, lse, dO, lddo, dQ, lddq, dK, lddk, dV, lddv, ws, ws_bytes, stream,
+                 true);
 }
 
 }  // extern "C"

@@ -164,6 +164,37 @@ def test_geo_all_patches_selected_equals_dense():
         assert_close(a, b.double().cpu().numpy(), TOL_BF16, nm)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_geo_backward_reusing_the_forward_workspace(dtype):
+    # ssc_geo_coupling_bwd_reuse takes the patch-major operands and the schedule
+    # from the forward's workspace; the results match the rebuilding call (up to
+    # the order of the atomic dK / dQ additions) and the oracle
+    pair = synth.make_workload("geo_60k", n=5000)
+    P, R = 40, 6
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    t = _geo_tables(pair, P, R, dtype)
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, dtype)
+    tabs = [as_i32(t[x]) for x in ("off_N", "mem_N", "off_M", "mem_M", "topk")]
+    dt = 0 if dtype == "bf16" else 1
+    nb = api.lib().ssc_geo_coupling_workspace_size(pair.n, pair.n, pair.d, pair.k, P, P, R, dt)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, *tabs, workspace=ws)
+    got = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, need_dV=True,
+                                   workspace=ws, reuse_forward=True)
+    again = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, need_dV=True,
+                                     workspace=ws, reuse_forward=True)
+    plain = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, need_dV=True)
+    _status_ok()
+    ref = oracle.geo_bwd(Q64, K64, V64, dO64, pair.scale, t["off_N"], t["mem_N"], t["off_M"],
+                         t["mem_M"], t["topk"])
+    for a, b, c, nm in zip(got, again, plain, ("dQ", "dK", "dV")):
+        assert_close(a, ref[nm], tol, nm)
+        for other in (b, c):
+            np.testing.assert_allclose(a.cpu().numpy(), other.cpu().numpy(), rtol=1e-4, atol=1e-6)
+    with pytest.raises(ValueError):
+        api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, reuse_forward=True)
+
+
 @pytest.mark.parametrize("name", ["geo_60k", "geo_160k_warped"])
 def test_geo_bf16_full_size(name):
     pair = synth.make_workload(name)
