@@ -45,8 +45,8 @@ def pair_flops(d, k, need_dv):
 # capture of this bench's own launch (dram__bytes_read.sum + dram__bytes_write.sum,
 # a 1-pass metric set; summary in profiles/tc_bwd_dqk_kernel_dense60k_dram.md).
 # It stands only while the kernel's source text is the one that was captured.
-DQK_TRAFFIC = {"kernel_sha256_16": "187ae6fa33bfecf9", "n": 60000, "d": 128, "k": 196,
-               "read_bytes": 209.80e6, "write_bytes": 67.15e6}
+DQK_TRAFFIC = {"kernel_sha256_16": "462d3ed1072e8022", "n": 60000, "d": 128, "k": 196,
+               "read_bytes": 178.83e6, "write_bytes": 84.00e6}
 
 
 def dqk_kernel_hash():

@@ -353,10 +353,14 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           break;
         }
         tc_fence_after();
+        // 32-column chunks wholly past the segment's last key (nkeys is uniform
+        // over the tile, so these branches are warp-uniform): not loaded, no
+        // exponentials, P = 0
         float x[NC][32];
         const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
 #pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, reinterpret_cast<uint32_t(&)[32]>(x[c]));
+        for (int c = 0; c < NC; ++c)
+          if (col0 + 32 * c < nkeys) tmem_ld32(sa + 32 * c, reinterpret_cast<uint32_t(&)[32]>(x[c]));
         tmem_ld_wait();
         if (nkeys < 128) {
 #pragma unroll
@@ -365,9 +369,10 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
             for (int i = 0; i < 32; ++i)
               if (col0 + 32 * c + i >= nkeys) x[c][i] = -INFINITY;
         }
-        float mx = max32(x[0]);
+        float mx = -INFINITY;
 #pragma unroll
-        for (int c = 1; c < NC; ++c) mx = fmaxf(mx, max32(x[c]));
+        for (int c = 0; c < NC; ++c)
+          if (col0 + 32 * c < nkeys) mx = fmaxf(mx, max32(x[c]));
         if (NWG > 1) {
           s_pmax[g & 1][wg][lrow] = mx;
           mbar_arrive(&bar_xmax);
@@ -411,7 +416,12 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         float rs[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[NC][16];
 #pragma unroll
-        for (int c = 0; c < NC; ++c)
+        for (int c = 0; c < NC; ++c) {
+          if (col0 + 32 * c >= nkeys) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[c][i] = 0u;
+            continue;
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
@@ -419,6 +429,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
             rs[i & 3] += a0 + a1;
             pk[c][i] = pack_bf16x2(a0, a1);
           }
+        }
         l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         // P over this thread's columns: TMEM columns buf*128 + col0/2 ...
         const uint32_t pa = tmem_lane_addr(tmem, warp, buf * 128 + col0 / 2);
@@ -1310,6 +1321,11 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
         for (int c = 0; c < NC; ++c) {
           const int cbase = col0 + 32 * c;
           const bool full = live_row && cbase + 32 <= sg.nkeys;
+          if (kFixed && cbase >= sg.nkeys) {  // wholly past the segment's last key: no exponentials
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pr[c][i] = 0.f;
+            continue;
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             float v = ex2_approx(fmaf(__uint_as_float(sv[c][i]), p.scale_log2, -lse2));
