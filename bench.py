@@ -42,9 +42,9 @@ def pair_flops(d, k, need_dv):
 
 
 # DRAM traffic of tc_bwd_dqk_kernel on the dense 60k workload, from one ncu
-# capture of this bench's own launch (dram__bytes_read.sum + dram__bytes_write.sum,
-# a 1-pass metric set; summary in profiles/tc_bwd_dqk_kernel_dense60k_dram.md).
-# It stands only while the kernel's source text is the one that was captured.
+# capture of this bench's own launch at n = 60k (dram__bytes_read.sum +
+# dram__bytes_write.sum, a 1-pass metric set).  It stands only while the
+# kernel's source text is the one that was captured.
 DQK_TRAFFIC = {"kernel_sha256_16": "462d3ed1072e8022", "n": 60000, "d": 128, "k": 196,
                "read_bytes": 178.83e6, "write_bytes": 84.00e6}
 
@@ -67,6 +67,9 @@ def dqk_traffic(n, d, k):
     if (n, d, k) != (t["n"], t["d"], t["k"]) or dqk_kernel_hash() != t["kernel_sha256_16"]:
         return None
     return t["read_bytes"] + t["write_bytes"]
+
+
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, nominal (no sparsity)
 
 
 def peaks():
@@ -203,6 +206,52 @@ def run_geo_sweep(api, synth, torch, dev, need_dv, fpp, bpp):
     return out
 
 
+def run_fps_timing(api, synth, torch, dev, reps=5):
+    """FPS + Voronoi + patch tables per shape on device-resident points, warmed:
+    the FPS kernel's own launch time (CUDA events around each launch, on its
+    stream) per call and per round, and the whole call.  60k (P 480) and the
+    160k warped pair's target shape (P 1280)."""
+    stream = torch.cuda.current_stream()
+    out = []
+    for name in ("geo_60k", "geo_160k_warped"):
+        gp = synth.make_workload(name)
+        pts = torch.tensor(gp.pts_N).to(dev)
+        for _ in range(2):
+            api.ssc_fps_patches(pts, gp.P)
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        api.ssc_profile_enable(True)
+        for e in evs:
+            e[0].record(stream)
+            api.ssc_fps_patches(pts, gp.P)
+            e[1].record(stream)
+        api.ssc_profile_enable(False)
+        torch.cuda.synchronize()
+        kms, kn = api.ssc_profile_read(api.PROF_FPS)
+        kms /= max(kn, 1)
+        call_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        out.append({"workload": name, "n": gp.n, "P": gp.P, "fps_kernel_ms": round(kms, 4),
+                    "us_per_round": round(kms * 1e3 / gp.P, 3), "call_ms": round(call_ms, 4),
+                    "calls": reps})
+        del pts
+    return out
+
+
+def geo_tables_flops(offN, offM, topk, d, k, need_dv):
+    """Support (algorithmic) and tile-padded (executed) (i, j) pair counts of one
+    Geo step from the patch tables, and the flops per pair."""
+    sN = np.diff(offN.cpu().numpy()).astype(np.float64)
+    sM = np.diff(offM.cpu().numpy()).astype(np.float64)
+    t = topk.cpu().numpy()
+    U = sM[t].sum(axis=1)
+    pairs = float((sN * U).sum())
+    tilesN = np.ceil(sN / 128.0) * 128.0
+    Upad = (np.ceil(sM / 128.0) * 128.0)[t].sum(axis=1)
+    pairs_exec = float((tilesN * Upad).sum())
+    fpp, bpp = pair_flops(d, k, need_dv)
+    return pairs, pairs_exec, fpp, bpp
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ws, rank, local):
     import torch
@@ -242,19 +291,12 @@ def run_ours(args, ws, rank, local):
     if gpair is not None:
         gQ, gK, gV = bf(gpair.F_N).to(dev), bf(gpair.F_M).to(dev), bf(gpair.Phi_M).to(dev)
         gdO = torch.tensor(gpair.dO).to(dev)
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
         _, _, offN, memN = api.ssc_fps_patches(torch.tensor(gpair.pts_N).to(dev), gpair.P)
         _, _, offM, memM = api.ssc_fps_patches(torch.tensor(gpair.pts_M).to(dev), gpair.P)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        fps_ms = t0.elapsed_time(t1) / 2
         gws = torch.empty(api.lib().ssc_geo_coupling_workspace_size(
             gpair.n, gpair.n, gpair.d, gpair.k, gpair.P, gpair.P, gpair.R, 0),
             dtype=torch.uint8, device=dev)
-        geo = dict(Q=gQ, K=gK, V=gV, dO=gdO, offN=offN, memN=memN, offM=offM, memM=memM,
-                   fps_ms=fps_ms, ws=gws)
+        geo = dict(Q=gQ, K=gK, V=gV, dO=gdO, offN=offN, memN=memN, offM=offM, memM=memM, ws=gws)
 
     def geo_step():
         g = geo
@@ -397,6 +439,26 @@ def run_ours(args, ws, rank, local):
                            "+ this backward"}
         barrier(ws)
 
+    # ---- per-kernel launch times of the Geo step (library events on the
+    # launching stream), L2 flushed before each step
+    geo_kern = None
+    if geo:
+        gsteps = max(3, min(args.steps, 5))
+        torch.cuda.synchronize()
+        api.ssc_profile_enable(True)
+        for _ in range(gsteps):
+            flush.zero_()
+            topk_last = geo_step()
+        api.ssc_profile_enable(False)
+        torch.cuda.synchronize()
+        geo_kern = {nm: api.ssc_profile_read(kid) for nm, kid in (
+            ("fwd", api.PROF_FWD), ("bwd_dqk", api.PROF_BWD_DQK), ("bwd_dv", api.PROF_BWD_DV),
+            ("pool", api.PROF_POOL), ("scores", api.PROF_SCORES), ("topk", api.PROF_TOPK),
+            ("gather", api.PROF_GATHER))}
+        geo_kern = {nm: (ms / gsteps, n // gsteps) for nm, (ms, n) in geo_kern.items()}
+        geo_kern["_topk"] = topk_last
+    fps_timing = run_fps_timing(api, synth, torch, dev) if (geo and rank == 0) else None
+
     pk = peaks()
     tflops = ws * flops_step / (dense_ms * 1e-3) / 1e12
     # dominant kernel: the dQ/dK backward kernel (2/3 of the flops), its average
@@ -433,12 +495,15 @@ def run_ours(args, ws, rank, local):
                   "fwd_kernel_ms": round(kfwd_ms / max(kfwd_n, 1), 4),
                   "bwd_kernel_ms": round(kbwd_mean, 4),
                   "frac_of_peak": round(tflops / ws / pk["tflops"], 4),
+                  "frac_of_datasheet_peak": round(tflops / ws / DATASHEET_BF16_TFLOPS, 4),
                   "peak_gib": round(peak_gib, 3),
                   "with_dV": with_dv},
         "roofline": {"bound": "tensor", "kernel": "tc_bwd_dqk_kernel (dense backward, dQ and dK)",
                      "achieved": round(achieved, 2), "peak": pk["tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / pk["tflops"], 4), "peak_source": pk["source"] +
                      " burst bf16 (MEASURED_PEAKS.json bf16_tflops)",
+                     "frac_of_datasheet_peak": round(achieved / DATASHEET_BF16_TFLOPS, 4),
+                     "frac_model_flops": round(achieved_model / pk["tflops"], 4),
                      "flops_per_launch": bwd_flops, "flop_convention": "executed (S recompute included)",
                      "achieved_model_flops": round(achieved_model, 2),
                      "launches_timed": kbwd_n, "traffic": dqk_traffic(n, d, k),
@@ -459,12 +524,56 @@ def run_ours(args, ws, rank, local):
                                     "tables, workspace and outputs",
                             "sizes": run_geo_sweep(api, synth, torch, dev, args.need_dv, fpp, bpp)}
     if geo:
-        U = float(np.mean(np.diff(geo["offM"].cpu().numpy()))) * gpair.R
-        gflops = float(gpair.n) * U * (fpp + bpp)
+        pairs, pairs_exec, gfpp, gbpp = geo_tables_flops(geo["offN"], geo["offM"],
+                                                         geo_kern["_topk"], gpair.d, gpair.k,
+                                                         args.need_dv)
+        gflops = pairs * (gfpp + gbpp)
+        gd, gk, gn = gpair.d, gpair.k, gpair.n
+        kp = (gk + 15) // 16 * 16
+        kp = kp + 16 if kp % 64 == 48 else kp
+
+        def kern(nm, flops=None, nbytes=None, bound="tensor"):
+            ms, cnt = geo_kern[nm]
+            if cnt == 0:
+                return None
+            r = {"ms": round(ms, 4), "launches_per_step": cnt}
+            if flops is not None:
+                a = flops / (ms * 1e-3) / 1e12
+                r.update({"bound": "tensor", "achieved": round(a, 2), "peak": pk["tflops"],
+                          "unit": "TFLOP/s", "frac": round(a / pk["tflops"], 4),
+                          "flops": flops})
+            if nbytes is not None:
+                g = nbytes / (ms * 1e-3) / 1e9
+                r.update({"algorithmic_bytes": nbytes, "achieved_gbs": round(g, 1),
+                          "hbm_frac": round(g / pk["hbm"], 4)})
+                if flops is None:
+                    r.update({"bound": bound, "peak": pk["hbm"], "unit": "GB/s"})
+            return r
+
+        geo_roof = {
+            "fwd": kern("fwd", pairs * gfpp, 2.0 * gn * (gd + gd + kp) + 4.0 * gn * (gk + 1)),
+            "bwd_dqk": kern("bwd_dqk", pairs * (gbpp - (2 * gk if args.need_dv else 0)),
+                            2.0 * gn * (gd + gd + kp + kp) + 4.0 * gn * (2 * gd + 2)),
+            "pool": kern("pool", None, 2.0 * (2.0 * gn * gd) + 2 * 4.0 * gn, "hbm"),
+            "scores": kern("scores", None, 8.0 * gpair.P * gpair.P + 2 * 8.0 * gpair.P * gd, "hbm"),
+            "topk": kern("topk", None, 8.0 * gpair.P * gpair.P, "hbm"),
+            "gather": kern("gather", None, 2 * 2.0 * gn * (gd + gd + kp), "hbm"),
+            "flop_convention": "support pairs sum_p |p| |U(p)| x per-pair flops (no tile padding)",
+            "bytes_convention": "one read of each input row and one write of each output row "
+                                "per launch (L2 re-reads not counted)",
+            "peak_source": pk["source"] + " (MEASURED_PEAKS.json: bf16_tflops, hbm_gbs)",
+        }
         res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_ms, 4),
                       "tflops": round(gflops / (geo_ms * 1e-3) / 1e12, 2),
-                      "support_per_row": round(U, 1), "fps_ms_per_shape": round(geo["fps_ms"], 3),
-                      "note": "step = scores/top-R + fwd + bwd (the backward reuses the forward's patch-major operands and schedule from the workspace); FPS per shape, outside the step"}
+                      "frac_of_peak": round(gflops / (geo_ms * 1e-3) / 1e12 / pk["tflops"], 4),
+                      "support_pairs": pairs, "tile_pairs": pairs_exec,
+                      "tile_fill": round(pairs / pairs_exec, 4),
+                      "support_per_row": round(pairs / gpair.n, 1),
+                      "roofline": geo_roof,
+                      "fps": fps_timing,
+                      "note": "step = scores/top-R + fwd + bwd (the backward reuses the forward's "
+                              "patch-major operands and schedule from the workspace); FPS per "
+                              "shape, outside the step, timed warm on resident points"}
     return res
 
 

@@ -130,12 +130,23 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex,
  *   current); make that first call before capturing any stream into a graph.
  *   Every call shares the array: calls that overlap on the GPU (different
  *   streams or host threads) race and must be serialised by the caller; each
- *   call clears the counters it needs zeroed.  No device allocation is made. */
+ *   call clears the counters it needs zeroed.  No device allocation is made.
+ *   The looked-up address is kept for the rest of the process, so a program
+ *   that resets a device's primary context (cudaDeviceReset) must not call
+ *   this entry point on that device afterwards. */
 #define SSC_FPS_NOALLOC_MAX_N 262144
 #define SSC_FPS_NOALLOC_MAX_P 65535
 int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_vertex,
                             int* centers, int* owner, int* offsets, int* members,
                             ssc_stream_t stream);
+
+/* Test hook of the FPS launch (the pages have no counterpart): 8 or 16 forces
+ * the thread-block cluster size of later ssc_fps_patches* calls (16 still
+ * falls back to 8 where the device cannot hold such a cluster); 0 restores
+ * the automatic choice.  With 8 CTAs, point counts above 8 x 16384 take the
+ * path that keeps the per-point state in the workspace instead of on chip.
+ * Other values are SSC_ERR_INVALID_ARG.  Results do not depend on it. */
+int ssc_debug_fps_cluster_size(int cl);
 
 /* Launch timing (a measurement hook; the pages have no counterpart).
  * ssc_profile_enable(1) clears the record and starts recording: every later
@@ -150,8 +161,13 @@ int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_vertex,
 #define SSC_PROF_DENSE_FWD 0 /* dense forward on CTA pairs (tc_fwd_pair_kernel) */
 #define SSC_PROF_FWD 1       /* single-CTA forward (Geo, and dense when pairs are not used) */
 #define SSC_PROF_BWD_DQK 2   /* backward dQ/dK kernel (tc_bwd_dqk_kernel) */
-#define SSC_PROF_BWD_DV 3    /* optional dV pass (tc_bwd_kernel) */
-#define SSC_PROF_KERNELS 4
+#define SSC_PROF_BWD_DV 3    /* optional dV pass (tc_dv_kernel dense, tc_bwd_kernel Geo) */
+#define SSC_PROF_FPS 4       /* FPS rounds (fps_cluster_kernel / fps_cluster_mem_kernel) */
+#define SSC_PROF_POOL 5      /* patch-mean pooling, one launch per shape */
+#define SSC_PROF_SCORES 6    /* patch score matrix */
+#define SSC_PROF_TOPK 7      /* top-R selection */
+#define SSC_PROF_GATHER 8    /* bf16 row gathers (patch-major Q, K, V; V re-pack) */
+#define SSC_PROF_KERNELS 9
 int ssc_profile_enable(int on);
 int ssc_profile_read(int kernel, double* total_ms, int* launches);
 

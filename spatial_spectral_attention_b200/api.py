@@ -59,6 +59,7 @@ def ssc_kernel_launches():
 
 
 PROF_DENSE_FWD, PROF_FWD, PROF_BWD_DQK, PROF_BWD_DV = 0, 1, 2, 3
+PROF_FPS, PROF_POOL, PROF_SCORES, PROF_TOPK, PROF_GATHER = 4, 5, 6, 7, 8
 
 
 def ssc_profile_enable(on=True, clear=True):

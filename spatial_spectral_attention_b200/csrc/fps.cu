@@ -15,11 +15,13 @@
 // Each round a CTA reduces its candidate, pushes it into every CTA's shared
 // memory through DSMEM, and one cluster barrier later every CTA knows the next
 // centre.  No grid-wide synchronisation.
+#include <atomic>
 #include <cfloat>
 #include <climits>
 #include <cooperative_groups.h>
 
 #include "internal.h"
+#include "ssc.h"
 
 namespace cg = cooperative_groups;
 
@@ -311,15 +313,22 @@ __global__ void __launch_bounds__(512) sort_segments_kernel(const int* __restric
   }
 }
 
+std::atomic<int> g_cl_forced{0};
+
+// 16-CTA clusters where the device allows non-portable cluster sizes, else 8
+// (the query runs once, thread-safely, on first use; a forced size wins).
 int fps_cluster_size() {
-  static int cl = -1;
-  if (cl < 0) {
-    cl = 8;
-    if (cudaFuncSetAttribute(fps_cluster_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             1) == cudaSuccess)
-      cl = 16;
+  const int forced = g_cl_forced.load(std::memory_order_relaxed);
+  if (forced) return forced;
+  static const int cl = [] {
+    const int r = cudaFuncSetAttribute(fps_cluster_kernel<1>,
+                                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                          cudaSuccess
+                      ? 16
+                      : 8;
     cudaGetLastError();
-  }
+    return r;
+  }();
   return cl;
 }
 
@@ -345,10 +354,17 @@ cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   count_launch();
-  return cudaLaunchKernelEx(&cfg, kern, pts, n, P, seed, per, centers, owner);
+  prof_launch_begin(st);
+  e = cudaLaunchKernelEx(&cfg, kern, pts, n, P, seed, per, centers, owner);
+  prof_launch_end(st, SSC_PROF_FPS);
+  return e;
 }
 
 }  // namespace
+
+void fps_force_cluster_size(int cl) {
+  g_cl_forced.store(cl == 8 || cl == 16 ? cl : 0, std::memory_order_relaxed);
+}
 
 size_t fps_workspace_bytes(int n, int P) {
   Carve c(nullptr);
@@ -414,8 +430,10 @@ cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* ce
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     count_launch();
+    prof_launch_begin(st);
     e = cudaLaunchKernelEx(&cfg, fps_cluster_mem_kernel, pts, n, P, seed, centers, owner, best,
                            chosen);
+    prof_launch_end(st, SSC_PROF_FPS);
   }
   if (e != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(counts, 0, sizeof(int) * P, st)) != cudaSuccess) return e;

@@ -12,7 +12,9 @@
 // library holds it until the process exits.  Host code cannot use the array's
 // name as a device address; the address is looked up once per device with
 // cudaGetSymbolAddress, with that device current, on the first call made on
-// that device.  All calls share the one array and it keeps the last call's
+// that device, and kept for the rest of the process (a host program that
+// resets the device's primary context must not call this entry point on it
+// again).  All calls share the one array and it keeps the last call's
 // contents: the counters that must start at zero are cleared by every call
 // (on the stream, like the rest of the work), and calls that overlap on the
 // GPU -- on different streams or from different host threads -- race on it.
@@ -57,7 +59,7 @@ extern "C" int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_
   const int rc = scratch_address(&ws);
   if (rc != SSC_OK) return rc;
   (void)cudaGetLastError();
-  ssc::WaitCtl ctl{nullptr, 0};
+  const ssc::WaitCtl ctl = ssc::library_wait_ctl();
   return ssc::launch_fps_patches(pts, n, P, seed_vertex, centers, owner, offsets, members, ws,
                                  static_cast<cudaStream_t>(stream), ctl) == cudaSuccess
              ? SSC_OK

@@ -46,8 +46,15 @@ struct Carve {
   }
 };
 
+// The wait control every call passes to its kernels: the library's device
+// status word on the current device and the current wait limit (ssc_api.cu).
+WaitCtl library_wait_ctl();
+
 // ------------------------------------------------------------ fps.cu
 size_t fps_workspace_bytes(int n, int P);
+// Test hook: 0 = pick the FPS cluster size from the device (16 where allowed,
+// else 8); 8 or 16 forces that size for later calls.
+void fps_force_cluster_size(int cl);
 cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* centers, int* owner,
                                int* offsets, int* members, void* ws, cudaStream_t st,
                                const WaitCtl& ctl);

@@ -17,6 +17,7 @@
 #include <climits>
 
 #include "internal.h"
+#include "ssc.h"
 
 namespace ssc {
 namespace {
@@ -296,12 +297,16 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
       if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem)) !=
           cudaSuccess)
         return e;
+      prof_launch_begin(st);
       kern<<<P, 128, rows_smem, st>>>(F, ld, n, d, off, mem, mu, status);
     } else if (dtype == 1) {
+      prof_launch_begin(st);
       pool_kernel<true><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
     } else {
+      prof_launch_begin(st);
       pool_kernel<false><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
     }
+    prof_launch_end(st, SSC_PROF_POOL);
     count_launch();
     return cudaGetLastError();
   };
@@ -313,9 +318,13 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   if ((pe = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sc_smem)) != cudaSuccess)
     return pe;
+  prof_launch_begin(st);
   scores_kernel<<<grid, 256, sc_smem, st>>>(muN, PN, muM, PM, d, sc);
+  prof_launch_end(st, SSC_PROF_SCORES);
   count_launch();
+  prof_launch_begin(st);
   topk_kernel<<<PN, 256, 0, st>>>(sc, PM, R, topk);
+  prof_launch_end(st, SSC_PROF_TOPK);
   count_launch();
   return cudaGetLastError();
 }

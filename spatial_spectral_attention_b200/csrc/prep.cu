@@ -13,6 +13,7 @@
 #include <type_traits>
 
 #include "internal.h"
+#include "ssc.h"
 
 namespace ssc {
 namespace {
@@ -394,12 +395,14 @@ cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const
       const long long total = (long long)rows * (out_ld / (vec_ok == 2 ? 8 : 4));
       const int gb = (int)std::max<long long>(1, std::min<long long>((total + 255) / 256, 148LL * 16));
       const auto* ib = static_cast<const __nv_bfloat16*>(in);
+      prof_launch_begin(st);
       if (vec_ok == 2)
         gather_bf16_pieces<8><<<gb, 256, 0, st>>>(ib, in_ld, map, rows, src_rows, cols, out, out_ld,
                                                   ones_col, status);
       else
         gather_bf16_pieces<4><<<gb, 256, 0, st>>>(ib, in_ld, map, rows, src_rows, cols, out, out_ld,
                                                   ones_col, status);
+      prof_launch_end(st, SSC_PROF_GATHER);
       count_launch();
       return cudaGetLastError();
     }

@@ -38,6 +38,12 @@ WaitCtl make_ctl() {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SSC_OK : SSC_ERR_CUDA; }
 
+}  // namespace
+
+WaitCtl ssc::library_wait_ctl() { return make_ctl(); }
+
+namespace {
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_common(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN,
@@ -234,6 +240,12 @@ int ssc_debug_wait_timeout(unsigned long long limit_ns, ssc_stream_t stream) {
 }
 
 // ------------------------------------------------------------ patches
+int ssc_debug_fps_cluster_size(int cl) {
+  if (cl != 0 && cl != 8 && cl != 16) return SSC_ERR_INVALID_ARG;
+  fps_force_cluster_size(cl);
+  return SSC_OK;
+}
+
 size_t ssc_fps_patches_workspace_size(int n, int P) {
   if (n < 1 || P < 1) return 0;
   return fps_workspace_bytes(n, P);

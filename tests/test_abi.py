@@ -81,9 +81,17 @@ def test_profile_record_arguments_are_checked_on_the_host():
     L = _abi.lib()
     ms, n = ctypes.c_double(-1.0), ctypes.c_int(-1)
     assert L.ssc_profile_enable(3) == 1  # SSC_ERR_INVALID_ARG
-    assert L.ssc_profile_read(4, ctypes.byref(ms), ctypes.byref(n)) == 1
+    assert L.ssc_profile_read(1000, ctypes.byref(ms), ctypes.byref(n)) == 1
+    assert L.ssc_profile_read(-1, ctypes.byref(ms), ctypes.byref(n)) == 1
     assert L.ssc_profile_read(0, None, ctypes.byref(n)) == 1
     # an empty record reads as zero launches without touching the device
     assert L.ssc_profile_enable(1) == 0 and L.ssc_profile_enable(0) == 0
     assert L.ssc_profile_read(2, ctypes.byref(ms), ctypes.byref(n)) == 0
     assert n.value == 0 and ms.value == 0.0
+
+
+def test_fps_cluster_size_hook_checks_its_argument():
+    L = _abi.lib()
+    assert L.ssc_debug_fps_cluster_size(5) == 1
+    assert L.ssc_debug_fps_cluster_size(8) == 0
+    assert L.ssc_debug_fps_cluster_size(0) == 0

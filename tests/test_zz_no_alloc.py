@@ -35,6 +35,25 @@ def test_noalloc_matches_workspace_call_twice():
             assert torch.equal(g, r)
 
 
+def test_noalloc_memory_resident_path_near_its_limit():
+    # with 8-CTA clusters, n > 131072 keeps the running distances in the
+    # scratch array instead of on chip; n close to the 262144 limit fills
+    # most of the array
+    L = _abi.lib()
+    assert L.ssc_debug_fps_cluster_size(8) == 0
+    try:
+        n, P = 250000, 40
+        pts = torch.tensor(synth.sphere_points(n, np.random.default_rng(3)).astype(np.float32)).cuda()
+        for _ in range(2):
+            got = _raw_noalloc(pts, P)
+            ref = api.ssc_fps_patches(pts, P)
+            torch.cuda.synchronize()
+            for g, r in zip(got, ref):
+                assert torch.equal(g, r)
+    finally:
+        assert L.ssc_debug_fps_cluster_size(0) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     L = _abi.lib()
     big = 262145
