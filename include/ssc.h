@@ -167,7 +167,9 @@ int ssc_debug_fps_cluster_size(int cl);
 #define SSC_PROF_SCORES 6    /* patch score matrix */
 #define SSC_PROF_TOPK 7      /* top-R selection */
 #define SSC_PROF_GATHER 8    /* bf16 row gathers (patch-major Q, K, V; V re-pack) */
-#define SSC_PROF_KERNELS 9
+#define SSC_PROF_LIN_REDUCE 9 /* linear coupling: phi(X)^T B reductions */
+#define SSC_PROF_LIN_ROWS 10  /* linear coupling: row-tile products (O, dQ, dK, dV) */
+#define SSC_PROF_KERNELS 11
 int ssc_profile_enable(int on);
 int ssc_profile_read(int kernel, double* total_ms, int* launches);
 
@@ -275,6 +277,47 @@ int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk,
                                float* dQ, int lddq, float* dK, int lddk,
                                float* dV, int lddv,
                                void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Linear-attention (ELU) coupling: the approximate coupling of the project   */
+/* page's Table 1 (row "Linear attention (ELU)"); the digest's               */
+/* "Interpretation" describes linear attention as replacing the softmax with */
+/* a low-rank feature map.  Feature map phi(x) = elu(x) + 1 (x + 1 for x > 0,  */
+/* exp(x) otherwise) on every descriptor entry; weights <phi(Q_i), phi(K_j)>, */
+/* each row normalised by its weight sum:                                    */
+/*   O_i = sum_j <phi(Q_i), phi(K_j)> V_j / den_i,                            */
+/*   den_i = sum_j <phi(Q_i), phi(K_j)>,                                      */
+/* evaluated as phi(Q_i) (sum_j phi(K_j)^T V_j) / <phi(Q_i), sum_j phi(K_j)>, */
+/* linear in nN + nM.  There is no scale (the map has none).                 */
+/* Q [nN, ldq], K [nM, ldk], V [nM, ldv] bf16 (Q and K 16-byte aligned with  */
+/* ldq, ldk multiples of 8; V any stride, re-packed when needed); d in       */
+/* {64, 128}, 1 <= k <= 255.  phi(Q), phi(K), the d x (k+1) sums and dO/den  */
+/* are rounded to bf16 for the tensor cores, accumulation is fp32.  Outputs  */
+/* fp32: O [nN, ldo] (16-byte aligned), den [nN].                            */
+/* ------------------------------------------------------------------------ */
+
+size_t ssc_linear_coupling_workspace_size(int nN, int nM, int d, int k);
+
+int ssc_linear_coupling_fwd(const void* Q, int ldq, const void* K, int ldk,
+                            const void* V, int ldv, int nN, int nM, int d, int k,
+                            float* O, int ldo, float* den,
+                            void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* Backward for dL/dO = dO (fp32 [nN, lddo]), given the forward's O and den:
+ *   D_i = <dO_i, O_i>, dW_ij = (<dO_i, V_j> - D_i) / den_i for the weights
+ *   W_ij = <phi(Q_i), phi(K_j)>, dQ_i = phi'(Q_i) * sum_j dW_ij phi(K_j),
+ *   dK_j = phi'(K_j) * sum_i dW_ij phi(Q_i), dV_j = sum_i W_ij dO_i / den_i,
+ * with phi'(x) = 1 for x > 0 and exp(x) otherwise; evaluated in the same
+ * factored form as the forward.  dO is rounded to bf16 once.  dV may be NULL;
+ * dQ [nN, lddq], dK [nM, lddk], dV [nM, lddv] fp32 (16-byte aligned) are
+ * overwritten. */
+int ssc_linear_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
+                            const void* V, int ldv, int nN, int nM, int d, int k,
+                            const float* O, int ldo, const float* den,
+                            const float* dO, int lddo,
+                            float* dQ, int lddq, float* dK, int lddk,
+                            float* dV, int lddv,
+                            void* ws, size_t ws_bytes, ssc_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -43,6 +43,10 @@ SIGNATURES = {
     "ssc_geo_coupling_bwd_reuse": (I, [P, I, P, I, P, I, I, I, I, I, F, I,
                                        P, P, I, P, P, I, P, I, P, I, P, P, I,
                                        P, I, P, I, P, I, P, Z, P]),
+    "ssc_linear_coupling_workspace_size": (Z, [I, I, I, I]),
+    "ssc_linear_coupling_fwd": (I, [P, I, P, I, P, I, I, I, I, I, P, I, P, P, Z, P]),
+    "ssc_linear_coupling_bwd": (I, [P, I, P, I, P, I, I, I, I, I, P, I, P, P, I,
+                                    P, I, P, I, P, I, P, Z, P]),
 }
 
 _lib = None

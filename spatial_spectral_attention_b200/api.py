@@ -60,6 +60,7 @@ def ssc_kernel_launches():
 
 PROF_DENSE_FWD, PROF_FWD, PROF_BWD_DQK, PROF_BWD_DV = 0, 1, 2, 3
 PROF_FPS, PROF_POOL, PROF_SCORES, PROF_TOPK, PROF_GATHER = 4, 5, 6, 7, 8
+PROF_LIN_REDUCE, PROF_LIN_ROWS = 9, 10
 
 
 def ssc_profile_enable(on=True, clear=True):
@@ -243,4 +244,46 @@ def ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, scale, offN, memN, offM, memM, top
         _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
         _ptr(O), O.stride(0), _ptr(lse), _ptr(dO), dO.stride(0),
         _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(), _stream()))
+    return dQ, dK, dV
+
+
+def _bf16_qkv(Q, K, V):
+    _cuda(Q, K, V)
+    if not (Q.dtype == K.dtype == V.dtype == torch.bfloat16):
+        raise ValueError("the linear coupling takes bf16 Q, K and V")
+    return _rowmajor(Q), _rowmajor(K), _rowmajor(V)
+
+
+def ssc_linear_coupling_fwd(Q, K, V, workspace=None):
+    """Linear-attention (ELU) coupling: O (fp32 [nN,k]) and den (fp32 [nN])."""
+    ldq, ldk, ldv = _bf16_qkv(Q, K, V)
+    nN, d = Q.shape
+    nM, k = V.shape
+    O = torch.empty((nN, k), dtype=torch.float32, device=Q.device)
+    den = torch.empty(nN, dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_linear_coupling_workspace_size(nN, nM, d, k)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    check("ssc_linear_coupling_fwd", lib().ssc_linear_coupling_fwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, _ptr(O), k, _ptr(den),
+        _ptr(ws), ws.numel(), _stream()))
+    return O, den
+
+
+def ssc_linear_coupling_bwd(Q, K, V, O, den, dO, need_dV=False, workspace=None):
+    """Gradients (dQ, dK, dV or None) of the linear coupling for upstream dO (fp32)."""
+    ldq, ldk, ldv = _bf16_qkv(Q, K, V)
+    _cuda(O, den, dO)
+    nN, d = Q.shape
+    nM, k = V.shape
+    dev = Q.device
+    dQ = torch.empty((nN, d), dtype=torch.float32, device=dev)
+    dK = torch.empty((nM, d), dtype=torch.float32, device=dev)
+    dV = torch.empty((nM, k), dtype=torch.float32, device=dev) if need_dV else None
+    O, dO, den = O.contiguous(), dO.contiguous(), den.contiguous()
+    nb = lib().ssc_linear_coupling_workspace_size(nN, nM, d, k)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    check("ssc_linear_coupling_bwd", lib().ssc_linear_coupling_bwd(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, _ptr(O), O.stride(0), _ptr(den),
+        _ptr(dO), dO.stride(0), _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(),
+        _stream()))
     return dQ, dK, dV

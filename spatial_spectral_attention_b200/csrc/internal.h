@@ -203,6 +203,35 @@ cudaError_t launch_tc_fwd_pair(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
                                float scale, float* O, int ldo, float* lse, float* part,
                                int sum_col, cudaStream_t st, const WaitCtl& ctl);
 
+// ------------------------------------------------------------ linear.cu (ELU linear attention)
+// Columns of the bf16 operands that carry [V | 1] and Y: k + 1 rounded to 16.
+int lin_kv(int k);
+// Upper bound on the partial sums the reduction over n rows leaves (its
+// workspace holds that many [128 x 256] fp32 blocks, one per CTA cluster).
+int lin_reduce_grid(int n);
+// The weight matrix a reduction produces: W [128 x 256] and W^T [256 x 128]
+// in bf16 (zero outside d x nb), and the fp32 W when W32 != nullptr.
+struct LinWeights {
+  __nv_bfloat16* W;
+  __nv_bfloat16* WT;
+  float* W32;
+};
+// W = phi(X)^T B over n rows: X [n, ldx] with d columns, B [n, ldb] with bwidth
+// columns (read as zero beyond), nb = N (multiple of 16, <= 256); ones_col >= 0
+// sets that column of B to one on every row.
+cudaError_t launch_lin_reduce(const __nv_bfloat16* X, int ldx, const __nv_bfloat16* B, int ldb,
+                              int n, int d, int bwidth, int nb, int ones_col, float* part,
+                              LinWeights w, cudaStream_t st, const WaitCtl& ctl);
+// Row-tile products against a resident weight matrix (mode 0: forward
+// O = phi(A) W^T / den; 1: dV = phi(A) W^T; 2: out = (A W) * phi'(X)).
+cudaError_t launch_lin_rows(int mode, const __nv_bfloat16* A, int lda, int awidth, int n,
+                            const __nv_bfloat16* Wmat, int d, int k, int nmma, int ksteps,
+                            int ones_col, const __nv_bfloat16* X, int ldx, float* out, int ldout,
+                            float* den, cudaStream_t st, const WaitCtl& ctl);
+// Y rows [g / den, -<g, O> / den, 0 ...] with g = bf16(dO), ldy columns.
+cudaError_t launch_lin_prep(const float* dO, int lddo, const float* O, int ldo, const float* den,
+                            int n, int k, __nv_bfloat16* Y, int ldy, cudaStream_t st);
+
 // Test hook: a kernel that waits on a barrier nothing arrives on.
 cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl);
 

@@ -543,4 +543,130 @@ int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk, c
                  true);
 }
 
+// ------------------------------------------------------------ linear (ELU)
+namespace {
+
+struct LinWs {
+  __nv_bfloat16* Vp;  // V re-packed with a pitch of lin_kv(k) when its rows are not 16-byte aligned
+  __nv_bfloat16* Y;   // backward rows [dO / den, -D / den]
+  float* part;        // per-CTA partial sums of the reductions
+  LinWeights w1, w2;  // [KV | z] and [dKV | dz]
+};
+
+size_t lin_ws(void* base, int nN, int nM, int k, LinWs* w) {
+  Carve c(base);
+  LinWs x;
+  const int kv = lin_kv(k);
+  x.Vp = c.take<__nv_bfloat16>((size_t)nM * kv);
+  x.Y = c.take<__nv_bfloat16>((size_t)nN * kv);
+  x.part = c.take<float>((size_t)std::max(lin_reduce_grid(nN), lin_reduce_grid(nM)) * 128 * 256);
+  for (LinWeights* lw : {&x.w1, &x.w2}) {
+    lw->W = c.take<__nv_bfloat16>(128 * 256);
+    lw->WT = c.take<__nv_bfloat16>(256 * 128);
+    lw->W32 = nullptr;
+  }
+  if (w) *w = x;
+  return c.used + 256;
+}
+
+int lin_check(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN,
+              int nM, int d, int k) {
+  if (!Q || !K || !V) return SSC_ERR_INVALID_ARG;
+  if (nN < 1 || nM < 1 || k < 1) return SSC_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SSC_ERR_UNSUPPORTED;
+  if (k > 255) return SSC_ERR_UNSUPPORTED;
+  if (ldq < d || ldk < d || ldv < k) return SSC_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || ldq % 8 || ldk % 8) return SSC_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(V) & 1u) return SSC_ERR_ALIGNMENT;
+  return SSC_OK;
+}
+
+// V as the tensor cores read it: in place when its rows are 16-byte aligned,
+// else re-packed into the workspace (pitch lin_kv(k), zero padded).
+cudaError_t lin_v(const void* V, int ldv, int nM, int k, const LinWs& w, const __nv_bfloat16** Vout,
+                  int* ldout, cudaStream_t st, unsigned* status) {
+  if (ldv % 8 == 0 && aligned16(V)) {
+    *Vout = static_cast<const __nv_bfloat16*>(V);
+    *ldout = ldv;
+    return cudaSuccess;
+  }
+  *Vout = w.Vp;
+  *ldout = lin_kv(k);
+  return launch_gather_rows_bf16(V, ldv, 0, nullptr, nM, nM, k, w.Vp, lin_kv(k), status, st);
+}
+
+}  // namespace
+
+size_t ssc_linear_coupling_workspace_size(int nN, int nM, int d, int k) {
+  if (nN < 1 || nM < 1 || k < 1 || k > 255 || (d != 64 && d != 128)) return 0;
+  return lin_ws(nullptr, nN, nM, k, nullptr);
+}
+
+int ssc_linear_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                            int nN, int nM, int d, int k, float* O, int ldo, float* den, void* ws,
+                            size_t ws_bytes, ssc_stream_t stream) {
+  int rc = lin_check(Q, ldq, K, ldk, V, ldv, nN, nM, d, k);
+  if (rc) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!den) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, lin_ws(nullptr, nN, nM, k, nullptr))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  LinWs w;
+  lin_ws(ws, nN, nM, k, &w);
+  const int kv = lin_kv(k);
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((lin_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  // [KV | z] = phi(K)^T [V | 1]
+  if ((launch_lin_reduce(static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt, nM, d, k, kv, k,
+                             w.part, w.w1, st, ctl)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  // O = phi(Q) KV / phi(Q) z
+  return cuda_status(launch_lin_rows(0, static_cast<const __nv_bfloat16*>(Q), ldq, d, nN, w.w1.WT,
+                                     d, k, kv, 0, -1, nullptr, 0, O, ldo, den, st, ctl));
+}
+
+int ssc_linear_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                            int nN, int nM, int d, int k, const float* O, int ldo,
+                            const float* den, const float* dO, int lddo, float* dQ, int lddq,
+                            float* dK, int lddk, float* dV, int lddv, void* ws, size_t ws_bytes,
+                            ssc_stream_t stream) {
+  int rc = lin_check(Q, ldq, K, ldk, V, ldv, nN, nM, d, k);
+  if (rc) return rc;
+  if (!O || !den || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, lin_ws(nullptr, nN, nM, k, nullptr))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  LinWs w;
+  lin_ws(ws, nN, nM, k, &w);
+  const int kv = lin_kv(k);
+  const auto* Qb = static_cast<const __nv_bfloat16*>(Q);
+  const auto* Kb = static_cast<const __nv_bfloat16*>(K);
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((lin_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  // [KV | z] again (the forward's sums are not kept), then Y and [dKV | dz]
+  if ((launch_lin_reduce(Kb, ldk, Vt, ldvt, nM, d, k, kv, k, w.part, w.w1, st, ctl)) !=
+          cudaSuccess ||
+      (launch_lin_prep(dO, lddo, O, ldo, den, nN, k, w.Y, kv, st)) != cudaSuccess ||
+      (launch_lin_reduce(Qb, ldq, w.Y, kv, nN, d, kv, kv, -1, w.part, w.w2, st, ctl)) !=
+          cudaSuccess)
+    return SSC_ERR_CUDA;
+  // dQ = (Y [KV | z]^T) * phi'(Q);  dK = ([V | 1] [dKV | dz]^T) * phi'(K)
+  if ((launch_lin_rows(2, w.Y, kv, kv, nN, w.w1.W, d, k, 128, kv / 16, -1, Qb, ldq, dQ, lddq,
+                           nullptr, st, ctl)) != cudaSuccess ||
+      (launch_lin_rows(2, Vt, ldvt, k, nM, w.w2.W, d, k, 128, kv / 16, k, Kb, ldk, dK, lddk,
+                           nullptr, st, ctl)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  if (!dV) return SSC_OK;
+  // dV = phi(K) dKV
+  return cuda_status(launch_lin_rows(1, Kb, ldk, d, nM, w.w2.WT, d, k, (k + 15) / 16 * 16, 0, -1,
+                                     nullptr, 0, dV, lddv, nullptr, st, ctl));
+}
+
 }  // extern "C"
