@@ -279,6 +279,83 @@ int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk,
                                void* ws, size_t ws_bytes, ssc_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Batches of shape pairs (a training step of a functional-map pipeline       */
+/* evaluates the coupling for every pair of its batch; project page, Table 1, */
+/* "One ULRSSM training step", and "Only the evaluation of PiPhi changes").   */
+/* `batch` independent pairs of equal sizes are stored back to back: Q        */
+/* [batch][nN][ldq], K [batch][nM][ldk], V [batch][nM][ldv], O [batch][nN]    */
+/* [ldo], lse [batch][nN], dO, dQ like O/Q, dK, dV like K/V (pair b starts    */
+/* b nN rows, resp. b nM rows, after pair 0).  Patch tables per pair:         */
+/* offN [batch][PN+1], memN [batch][nN], offM [batch][PM+1], memM [batch][nM] */
+/* with vertex ids local to the pair, topk [batch][PN][R] with source patches */
+/* local to the pair.  One launch of each kernel covers every pair: the       */
+/* dense calls run a block-diagonal tile schedule (row tiles of pair b visit  */
+/* only the key tiles of pair b), the Geo calls shift the tables of pair b by */
+/* b nN / b nM vertices and b PN / b PM patches into one problem.  Results    */
+/* equal those of the single-pair calls on each pair (the bf16 dense forward  */
+/* uses the single-CTA kernel, so its rounding order differs from the pair    */
+/* kernel's).  Table entries outside their pair's range are dropped and set   */
+/* SSC_ERR_INVALID_ARG in the device status word; they never reach another    */
+/* pair.  Limits: batch nN, batch nM <= 2^30; Geo: batch PN, batch PM <=      */
+/* 65535.  The fp32 check mode of the dense calls runs pair after pair.       */
+/*                                                                            */
+/* The reverse coupling Pi_MN Phi_N = softmax(s F_M F_N^T) Phi_N, which       */
+/* pipelines use to map in the other direction, is the same call with the     */
+/* roles swapped: Q = F_M, K = F_N, V = Phi_N (and, for Geo, the M tables as  */
+/* the target tables, with top-R lists scored from F_M against F_N).  A batch */
+/* may hold pairs of both directions when their sizes agree.                  */
+/* ------------------------------------------------------------------------ */
+
+size_t ssc_dense_coupling_batched_workspace_size(int batch, int nN, int nM, int d, int k,
+                                                 int dtype);
+
+int ssc_dense_coupling_fwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                   const void* V, int ldv, int nN, int nM, int d, int k,
+                                   float scale, int dtype, float* O, int ldo, float* lse,
+                                   void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+int ssc_dense_coupling_bwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                   const void* V, int ldv, int nN, int nM, int d, int k,
+                                   float scale, int dtype, const float* O, int ldo,
+                                   const float* lse, const float* dO, int lddo,
+                                   float* dQ, int lddq, float* dK, int lddk,
+                                   float* dV, int lddv,
+                                   void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+size_t ssc_geo_coupling_batched_workspace_size(int batch, int nN, int nM, int d, int k, int PN,
+                                               int PM, int R, int dtype);
+
+int ssc_geo_coupling_fwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                 const void* V, int ldv, int nN, int nM, int d, int k, float scale,
+                                 int dtype, const int* offN, const int* memN, int PN,
+                                 const int* offM, const int* memM, int PM, const int* topk, int R,
+                                 float* O, int ldo, float* lse,
+                                 void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+int ssc_geo_coupling_bwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                 const void* V, int ldv, int nN, int nM, int d, int k, float scale,
+                                 int dtype, const int* offN, const int* memN, int PN,
+                                 const int* offM, const int* memM, int PM, const int* topk, int R,
+                                 const float* O, int ldo, const float* lse,
+                                 const float* dO, int lddo,
+                                 float* dQ, int lddq, float* dK, int lddk,
+                                 float* dV, int lddv,
+                                 void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* Pooling, scores and top-R for a batch: FN [batch][nN][ldn], FM
+ * [batch][nM][ldm], tables as above; topk [batch][PN][R] (local source
+ * patches), scores [batch][PN][PM] (nullable).  Bit-identical, pair by pair,
+ * to ssc_patch_scores_topk. */
+size_t ssc_patch_scores_topk_batched_workspace_size(int batch, int nN, int nM, int PN, int PM,
+                                                    int d);
+
+int ssc_patch_scores_topk_batched(int batch, const void* FN, int ldn, int nN, const void* FM,
+                                  int ldm, int nM, int d, int dtype, const int* offN,
+                                  const int* memN, int PN, const int* offM, const int* memM, int PM,
+                                  int R, int* topk, double* scores,
+                                  void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Linear-attention (ELU) coupling: the approximate coupling of the project   */
 /* page's Table 1 (row "Linear attention (ELU)"); the digest's               */
 /* "Interpretation" describes linear attention as replacing the softmax with */

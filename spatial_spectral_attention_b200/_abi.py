@@ -43,6 +43,19 @@ SIGNATURES = {
     "ssc_geo_coupling_bwd_reuse": (I, [P, I, P, I, P, I, I, I, I, I, F, I,
                                        P, P, I, P, P, I, P, I, P, I, P, P, I,
                                        P, I, P, I, P, I, P, Z, P]),
+    "ssc_dense_coupling_batched_workspace_size": (Z, [I, I, I, I, I, I]),
+    "ssc_dense_coupling_fwd_batched": (I, [I, P, I, P, I, P, I, I, I, I, I, F, I, P, I, P, P, Z, P]),
+    "ssc_dense_coupling_bwd_batched": (I, [I, P, I, P, I, P, I, I, I, I, I, F, I, P, I, P, P, I,
+                                           P, I, P, I, P, I, P, Z, P]),
+    "ssc_geo_coupling_batched_workspace_size": (Z, [I, I, I, I, I, I, I, I, I]),
+    "ssc_geo_coupling_fwd_batched": (I, [I, P, I, P, I, P, I, I, I, I, I, F, I,
+                                         P, P, I, P, P, I, P, I, P, I, P, P, Z, P]),
+    "ssc_geo_coupling_bwd_batched": (I, [I, P, I, P, I, P, I, I, I, I, I, F, I,
+                                         P, P, I, P, P, I, P, I, P, I, P, P, I,
+                                         P, I, P, I, P, I, P, Z, P]),
+    "ssc_patch_scores_topk_batched_workspace_size": (Z, [I, I, I, I, I, I]),
+    "ssc_patch_scores_topk_batched": (I, [I, P, I, I, P, I, I, I, I, P, P, I, P, P, I, I, P, P, P,
+                                          Z, P]),
     "ssc_linear_coupling_workspace_size": (Z, [I, I, I, I]),
     "ssc_linear_coupling_fwd": (I, [P, I, P, I, P, I, I, I, I, I, P, I, P, P, Z, P]),
     "ssc_linear_coupling_bwd": (I, [P, I, P, I, P, I, I, I, I, I, P, I, P, P, I,

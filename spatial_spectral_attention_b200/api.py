@@ -287,3 +287,126 @@ def ssc_linear_coupling_bwd(Q, K, V, O, den, dO, need_dV=False, workspace=None):
         _ptr(dO), dO.stride(0), _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(),
         _stream()))
     return dQ, dK, dV
+
+
+# ---------------------------------------------------------------- batches of pairs
+def _batched(t):
+    """Leading dimension of a [batch, rows, cols] tensor whose pairs are stored
+    back to back (unit column stride, batch stride = rows x leading dimension)."""
+    if t.dim() != 3 or t.stride(2) != 1 or t.stride(0) != t.shape[1] * t.stride(1):
+        raise ValueError("expected a [batch, rows, cols] tensor with pairs stored back to back")
+    return t.stride(1)
+
+
+def _bqkv(Q, K, V):
+    _cuda(Q, K, V)
+    if not (Q.dtype == K.dtype == V.dtype):
+        raise ValueError("Q, K and V must share one dtype")
+    if not (Q.shape[0] == K.shape[0] == V.shape[0]) or K.shape[1] != V.shape[1]:
+        raise ValueError("Q [B,nN,d], K [B,nM,d] and V [B,nM,k] must agree")
+    return _batched(Q), _batched(K), _batched(V), _dtype_code(Q)
+
+
+def ssc_dense_coupling_fwd_batched(Q, K, V, scale, workspace=None):
+    """Dense coupling of B pairs in one call: O [B,nN,k] fp32 and lse [B,nN]."""
+    ldq, ldk, ldv, dt = _bqkv(Q, K, V)
+    B, nN, d = Q.shape
+    nM, k = V.shape[1], V.shape[2]
+    O = torch.empty((B, nN, k), dtype=torch.float32, device=Q.device)
+    lse = torch.empty((B, nN), dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_dense_coupling_batched_workspace_size(B, nN, nM, d, k, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    check("ssc_dense_coupling_fwd_batched", lib().ssc_dense_coupling_fwd_batched(
+        B, _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(O), k, _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return O, lse
+
+
+def ssc_dense_coupling_bwd_batched(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=None):
+    """Gradients (dQ [B,nN,d], dK [B,nM,d], dV [B,nM,k] or None) of B dense couplings."""
+    ldq, ldk, ldv, dt = _bqkv(Q, K, V)
+    _cuda(O, lse, dO)
+    B, nN, d = Q.shape
+    nM, k = V.shape[1], V.shape[2]
+    dev = Q.device
+    dQ = torch.empty((B, nN, d), dtype=torch.float32, device=dev)
+    dK = torch.empty((B, nM, d), dtype=torch.float32, device=dev)
+    dV = torch.empty((B, nM, k), dtype=torch.float32, device=dev) if need_dV else None
+    O, dO, lse = O.contiguous(), dO.contiguous(), lse.contiguous()
+    nb = lib().ssc_dense_coupling_batched_workspace_size(B, nN, nM, d, k, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    check("ssc_dense_coupling_bwd_batched", lib().ssc_dense_coupling_bwd_batched(
+        B, _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(O), k, _ptr(lse), _ptr(dO), k, _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k,
+        _ptr(ws), ws.numel(), _stream()))
+    return dQ, dK, dV
+
+
+def _btables(offN, memN, offM, memM, topk):
+    _cuda(offN, memN, offM, memM, topk)
+    for t in (offN, memN, offM, memM, topk):
+        if t.dtype != torch.int32:
+            raise ValueError("patch tables must be int32")
+    return (offN.contiguous(), memN.contiguous(), offM.contiguous(), memM.contiguous(),
+            topk.contiguous())
+
+
+def ssc_geo_coupling_fwd_batched(Q, K, V, scale, offN, memN, offM, memM, topk, workspace=None):
+    """Geo-FlashAttention for B pairs: tables offN [B,PN+1], memN [B,nN], offM [B,PM+1],
+    memM [B,nM], topk [B,PN,R] (local indices).  Returns O [B,nN,k], lse [B,nN]."""
+    ldq, ldk, ldv, dt = _bqkv(Q, K, V)
+    offN, memN, offM, memM, topk = _btables(offN, memN, offM, memM, topk)
+    B, nN, d = Q.shape
+    nM, k = V.shape[1], V.shape[2]
+    PN, PM, R = offN.shape[1] - 1, offM.shape[1] - 1, topk.shape[2]
+    O = torch.empty((B, nN, k), dtype=torch.float32, device=Q.device)
+    lse = torch.empty((B, nN), dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_geo_coupling_batched_workspace_size(B, nN, nM, d, k, PN, PM, R, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    check("ssc_geo_coupling_fwd_batched", lib().ssc_geo_coupling_fwd_batched(
+        B, _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
+        _ptr(O), k, _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return O, lse
+
+
+def ssc_geo_coupling_bwd_batched(Q, K, V, O, lse, dO, scale, offN, memN, offM, memM, topk,
+                                 need_dV=False, workspace=None):
+    """Gradients of B Geo couplings (dQ, dK, dV or None), tables as for the forward."""
+    ldq, ldk, ldv, dt = _bqkv(Q, K, V)
+    offN, memN, offM, memM, topk = _btables(offN, memN, offM, memM, topk)
+    _cuda(O, lse, dO)
+    B, nN, d = Q.shape
+    nM, k = V.shape[1], V.shape[2]
+    PN, PM, R = offN.shape[1] - 1, offM.shape[1] - 1, topk.shape[2]
+    dev = Q.device
+    dQ = torch.empty((B, nN, d), dtype=torch.float32, device=dev)
+    dK = torch.empty((B, nM, d), dtype=torch.float32, device=dev)
+    dV = torch.empty((B, nM, k), dtype=torch.float32, device=dev) if need_dV else None
+    O, dO, lse = O.contiguous(), dO.contiguous(), lse.contiguous()
+    nb = lib().ssc_geo_coupling_batched_workspace_size(B, nN, nM, d, k, PN, PM, R, dt)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    check("ssc_geo_coupling_bwd_batched", lib().ssc_geo_coupling_bwd_batched(
+        B, _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
+        _ptr(offN), _ptr(memN), PN, _ptr(offM), _ptr(memM), PM, _ptr(topk), R,
+        _ptr(O), k, _ptr(lse), _ptr(dO), k, _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k,
+        _ptr(ws), ws.numel(), _stream()))
+    return dQ, dK, dV
+
+
+def ssc_patch_scores_topk_batched(FN, FM, offN, memN, offM, memM, R, return_scores=False):
+    """Patch scores and top-R for B pairs: FN [B,nN,d], FM [B,nM,d]; topk [B,PN,R]."""
+    _cuda(FN, FM, offN, memN, offM, memM)
+    ldn, ldm = _batched(FN), _batched(FM)
+    B, nN, d = FN.shape
+    nM = FM.shape[1]
+    PN, PM = offN.shape[1] - 1, offM.shape[1] - 1
+    dev = FN.device
+    topk = torch.empty((B, PN, R), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, PN, PM), dtype=torch.float64, device=dev) if return_scores else None
+    ws = _workspace(lib().ssc_patch_scores_topk_batched_workspace_size(B, nN, nM, PN, PM, d), dev)
+    check("ssc_patch_scores_topk_batched", lib().ssc_patch_scores_topk_batched(
+        B, _ptr(FN), ldn, nN, _ptr(FM), ldm, nM, d, _dtype_code(FN), _ptr(offN.contiguous()),
+        _ptr(memN.contiguous()), PN, _ptr(offM.contiguous()), _ptr(memM.contiguous()), PM, R,
+        _ptr(topk), _ptr(scores), _ptr(ws), ws.numel(), _stream()))
+    return (topk, scores) if return_scores else topk

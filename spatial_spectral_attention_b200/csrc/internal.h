@@ -60,11 +60,15 @@ cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* ce
                                const WaitCtl& ctl);
 
 // ------------------------------------------------------------ patch_topk.cu
-size_t scores_topk_workspace_bytes(int PN, int PM, int d);
+size_t scores_topk_workspace_bytes(int PN, int PM, int d, int batch = 1);
+// batch > 1: FN, FM hold batch shapes back to back (batch nN, batch nM rows)
+// and the tables are the concatenated ones (batch PN and batch PM patches);
+// scores [batch][PN][PM] pair by pair, topk [batch][PN][R] local to the pair.
 cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int ldm, int nM,
                                int d, int dtype, const int* offN, const int* memN, int PN,
                                const int* offM, const int* memM, int PM, int R, int* topk,
-                               double* scores, void* ws, unsigned* status, cudaStream_t st);
+                               double* scores, void* ws, unsigned* status, cudaStream_t st,
+                               int batch = 1);
 
 // ------------------------------------------------------------ prep.cu
 // out[r, 0..cols) = in[map ? map[r] : r, 0..cols) converted to bf16 (in is
@@ -94,6 +98,19 @@ int dense_num_segs(int nM);
 // prefix [ntiles + 1] receives the prefix sums of the tiles' segment counts.
 cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, int* prefix,
                                   cudaStream_t st);
+// Block-diagonal schedule of `batch` dense pairs stored back to back
+// (batch * ceil(nN/128) row tiles, batch * ceil(nM/128) segments, prefix of
+// batch * ceil(nN/128) + 1 entries).
+cudaError_t launch_batched_schedule(int batch, int nN, int nM, RowTile* tiles, KeySeg* segs,
+                                    int* prefix, cudaStream_t st);
+// Per-shape patch tables (off [batch][P+1], mem [batch][n]) as the tables of one
+// problem (off_out [batch P + 1], mem_out [batch n]); bad entries are made
+// out of range and set the bad-index bit.
+cudaError_t launch_concat_tables(const int* off, const int* mem, int P, int n, int batch,
+                                 int* off_out, int* mem_out, unsigned* status, cudaStream_t st);
+// Per-pair top-R lists [batch][PN][R] shifted to the concatenated source patches.
+cudaError_t launch_concat_topk(const int* topk, int PN, int R, int PM, int batch, int* out,
+                               unsigned* status, cudaStream_t st);
 // Geo schedule: per target patch ceil(|p|/128) row tiles that share the list of
 // 128-row pieces of the patch's selected source patches.  Writes the counts to
 // counts[0] (tiles) and counts[1] (segments).  Upper bounds for sizing:

@@ -175,10 +175,14 @@ constexpr int kST = 32;  // score tile (target x source patches)
 constexpr int kSC = 128;  // channels staged per step (one load phase for d <= 128)
 
 // scores[p, q] for a 32 x 32 tile per block; each thread owns 4 outputs and
-// sums its products strictly in channel order.
+// sums its products strictly in channel order.  blockIdx.z selects the pair of
+// a batch (its means and score block follow the previous pair's).
 __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ muN, int PN,
                                                      const double* __restrict__ muM, int PM, int d,
                                                      double* __restrict__ sc) {
+  muN += (size_t)blockIdx.z * PN * d;
+  muM += (size_t)blockIdx.z * PM * d;
+  sc += (size_t)blockIdx.z * PN * PM;
   extern __shared__ double s_ab[];  // a[kST][kSC + 1], then b[kST][kSC + 1]
   double(*a)[kSC + 1] = reinterpret_cast<double(*)[kSC + 1]>(s_ab);
   double(*b)[kSC + 1] = reinterpret_cast<double(*)[kSC + 1]>(s_ab + kST * (kSC + 1));
@@ -265,22 +269,23 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ sc
 
 }  // namespace
 
-size_t scores_topk_workspace_bytes(int PN, int PM, int d) {
+size_t scores_topk_workspace_bytes(int PN, int PM, int d, int batch) {
   Carve c(nullptr);
-  c.take<double>((size_t)PN * d);
-  c.take<double>((size_t)PM * d);
-  c.take<double>((size_t)PN * PM);
+  c.take<double>((size_t)batch * PN * d);
+  c.take<double>((size_t)batch * PM * d);
+  c.take<double>((size_t)batch * PN * PM);
   return c.used + 256;
 }
 
 cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, int ldm, int nM,
                                int d, int dtype, const int* offN, const int* memN, int PN,
                                const int* offM, const int* memM, int PM, int R, int* topk,
-                               double* scores, void* ws, unsigned* status, cudaStream_t st) {
+                               double* scores, void* ws, unsigned* status, cudaStream_t st,
+                               int batch) {
   Carve c(ws);
-  double* muN = c.take<double>((size_t)PN * d);
-  double* muM = c.take<double>((size_t)PM * d);
-  double* sc_ws = c.take<double>((size_t)PN * PM);
+  double* muN = c.take<double>((size_t)batch * PN * d);
+  double* muM = c.take<double>((size_t)batch * PM * d);
+  double* sc_ws = c.take<double>((size_t)batch * PN * PM);
   double* sc = scores ? scores : sc_ws;
   const int pt = d >= 128 ? 128 : 64;
   const int esz = dtype == 1 ? 4 : 2;
@@ -311,9 +316,9 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
     return cudaGetLastError();
   };
   cudaError_t pe;
-  if ((pe = pool(FN, ldn, nN, PN, offN, memN, muN)) != cudaSuccess) return pe;
-  if ((pe = pool(FM, ldm, nM, PM, offM, memM, muM)) != cudaSuccess) return pe;
-  dim3 grid((PM + kST - 1) / kST, (PN + kST - 1) / kST);
+  if ((pe = pool(FN, ldn, batch * nN, batch * PN, offN, memN, muN)) != cudaSuccess) return pe;
+  if ((pe = pool(FM, ldm, batch * nM, batch * PM, offM, memM, muM)) != cudaSuccess) return pe;
+  dim3 grid((PM + kST - 1) / kST, (PN + kST - 1) / kST, batch);
   const int sc_smem = 2 * kST * (kSC + 1) * (int)sizeof(double);
   if ((pe = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sc_smem)) != cudaSuccess)
@@ -323,7 +328,7 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   prof_launch_end(st, SSC_PROF_SCORES);
   count_launch();
   prof_launch_begin(st);
-  topk_kernel<<<PN, 256, 0, st>>>(sc, PM, R, topk);
+  topk_kernel<<<batch * PN, 256, 0, st>>>(sc, PM, R, topk);
   prof_launch_end(st, SSC_PROF_TOPK);
   count_launch();
   return cudaGetLastError();

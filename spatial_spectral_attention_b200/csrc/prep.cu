@@ -206,6 +206,78 @@ __global__ void dense_schedule_kernel(int nN, int nM, RowTile* __restrict__ tile
   }
 }
 
+// Block-diagonal schedule of `batch` dense pairs stored back to back: row
+// tile t of pair b covers query rows b nN + [128 t, ...) and visits only the
+// key tiles of pair b (rows b nM + [128 j, ...)).
+__global__ void batched_schedule_kernel(int batch, int nN, int nM, RowTile* __restrict__ tiles,
+                                        KeySeg* __restrict__ segs, int* __restrict__ prefix) {
+  const int nt = (nN + kTileRows - 1) / kTileRows, ns = (nM + kTileRows - 1) / kTileRows;
+  const long m = (long)batch * max(nt, ns);
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i <= m; i += (long)gridDim.x * blockDim.x) {
+    if (i < (long)batch * nt) {
+      const int b = (int)(i / nt), t = (int)(i % nt);
+      tiles[i] = RowTile{b * nN + t * kTileRows, min(kTileRows, nN - t * kTileRows), b * ns, ns};
+    }
+    if (i < (long)batch * ns) {
+      const int b = (int)(i / ns), j = (int)(i % ns);
+      segs[i] = KeySeg{b * nM + j * kTileRows, min(kTileRows, nM - j * kTileRows)};
+    }
+    if (i <= (long)batch * nt) prefix[i] = (int)(i * ns);
+  }
+}
+
+// Patch tables of `batch` shapes (offsets [batch][P+1] into members
+// [batch][n], vertex ids local to the shape) as the tables of one problem of
+// batch n vertices and batch P patches: offsets and members shifted by b n.
+// Entries outside their shape's range, offsets whose first value is not 0 or
+// last is not n, become out-of-range values that the consumers drop, and set
+// the bad-index bit.
+__global__ void concat_tables_kernel(const int* __restrict__ off, const int* __restrict__ mem,
+                                     int P, int n, int batch, int* __restrict__ off_out,
+                                     int* __restrict__ mem_out, unsigned* status) {
+  const long noff = (long)batch * P, nmem = (long)batch * n;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i <= max(noff, nmem);
+       i += (long)gridDim.x * blockDim.x) {
+    if (i < noff) {
+      const int b = (int)(i / P), q = (int)(i % P);
+      int o = off[(size_t)b * (P + 1) + q];
+      const bool bad = o < 0 || o > n || (q == 0 && o != 0) ||
+                       (q == P - 1 && off[(size_t)b * (P + 1) + P] != n);
+      if (bad) atomicOr(status, kStatusBadIndex);
+      o = min(max(o, 0), n);
+      off_out[i] = b * n + o;
+    }
+    if (i == noff) off_out[i] = batch * n;
+    if (i < nmem) {
+      const int b = (int)(i / n);
+      const int v = mem[i];
+      if (v < 0 || v >= n) {
+        atomicOr(status, kStatusBadIndex);
+        mem_out[i] = -1;
+      } else {
+        mem_out[i] = b * n + v;
+      }
+    }
+  }
+}
+
+// top-R lists [batch][PN][R] with source patches local to the pair, shifted by
+// b PM; entries outside [0, PM) become -1 (dropped downstream, bad-index bit).
+__global__ void concat_topk_kernel(const int* __restrict__ topk, int PN, int R, int PM, int batch,
+                                   int* __restrict__ out, unsigned* status) {
+  const long m = (long)batch * PN * R;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < m; i += (long)gridDim.x * blockDim.x) {
+    const int b = (int)(i / ((long)PN * R));
+    const int q = topk[i];
+    if (q < 0 || q >= PM) {
+      atomicOr(status, kStatusBadIndex);
+      out[i] = -1;
+    } else {
+      out[i] = b * PM + q;
+    }
+  }
+}
+
 // prefix[t] = sum of tiles[0..t).nseg for t <= counts[0] (single block).
 __global__ void __launch_bounds__(1024) tile_prefix_kernel(const RowTile* __restrict__ tiles,
                                                            const int* __restrict__ counts,
@@ -480,6 +552,31 @@ cudaError_t launch_dense_schedule(int nN, int nM, RowTile* tiles, KeySeg* segs, 
                                   cudaStream_t st) {
   const int m = std::max(dense_num_tiles(nN), dense_num_segs(nM)) + 1;
   dense_schedule_kernel<<<grid_for(m, 256), 256, 0, st>>>(nN, nM, tiles, segs, prefix);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_batched_schedule(int batch, int nN, int nM, RowTile* tiles, KeySeg* segs,
+                                    int* prefix, cudaStream_t st) {
+  const long m = (long)batch * std::max(dense_num_tiles(nN), dense_num_segs(nM)) + 1;
+  batched_schedule_kernel<<<grid_for(m, 256), 256, 0, st>>>(batch, nN, nM, tiles, segs, prefix);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_concat_tables(const int* off, const int* mem, int P, int n, int batch,
+                                 int* off_out, int* mem_out, unsigned* status, cudaStream_t st) {
+  const long m = (long)batch * std::max(P, n) + 1;
+  concat_tables_kernel<<<grid_for(m, 256), 256, 0, st>>>(off, mem, P, n, batch, off_out, mem_out,
+                                                         status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_concat_topk(const int* topk, int PN, int R, int PM, int batch, int* out,
+                               unsigned* status, cudaStream_t st) {
+  const long m = (long)batch * PN * R;
+  concat_topk_kernel<<<grid_for(m, 256), 256, 0, st>>>(topk, PN, R, PM, batch, out, status);
   count_launch();
   return cudaGetLastError();
 }

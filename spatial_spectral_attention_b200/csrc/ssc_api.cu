@@ -422,23 +422,14 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
 
 }  // namespace
 
-int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
-                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
-                         const int* memN, int PN, const int* offM, const int* memM, int PM,
-                         const int* topk, int R, float* O, int ldo, float* lse, void* ws,
-                         size_t ws_bytes, ssc_stream_t stream) {
-  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
-  if (rc) return rc;
-  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
-  if ((rc = check_out(O, ldo, k))) return rc;
-  if (!lse) return SSC_ERR_INVALID_ARG;
-  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
-    return SSC_ERR_WORKSPACE;
-  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  WaitCtl ctl = make_ctl();
-  GeoWs w;
-  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
+namespace {
+
+// The Geo forward once the arguments are checked and the workspace carved.
+int geo_fwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN,
+                int nM, int d, int k, float scale, int dtype, const int* offN, const int* memN,
+                int PN, const int* offM, const int* memM, int PM, const int* topk, int R, float* O,
+                int ldo, float* lse, const GeoWs& w, cudaStream_t st, const WaitCtl& ctl) {
+  int rc;
   if ((rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
                       topk, R, w, st, ctl)))
     return rc;
@@ -454,28 +445,15 @@ int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const v
   return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
 }
 
-namespace {
-
-int geo_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN, int nM,
-            int d, int k, float scale, int dtype, const int* offN, const int* memN, int PN,
-            const int* offM, const int* memM, int PM, const int* topk, int R, const float* O,
-            int ldo, const float* lse, const float* dO, int lddo, float* dQ, int lddq, float* dK,
-            int lddk, float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream,
-            bool reuse) {
-  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
-  if (rc) return rc;
-  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
-  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
-  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
-  if (dV && (rc = check_out(dV, lddv, k))) return rc;
-  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
-    return SSC_ERR_WORKSPACE;
-  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  WaitCtl ctl = make_ctl();
-  GeoWs w;
-  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
-  // the patch-major operands and the schedule: rebuilt here, or left by the forward
+// The Geo backward once the arguments are checked and the workspace carved;
+// with reuse the patch-major operands and the schedule are the forward's.
+int geo_bwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN,
+                int nM, int d, int k, float scale, int dtype, const int* offN, const int* memN,
+                int PN, const int* offM, const int* memM, int PM, const int* topk, int R,
+                const float* O, int ldo, const float* lse, const float* dO, int lddo, float* dQ,
+                int lddq, float* dK, int lddk, float* dV, int lddv, const GeoWs& w,
+                cudaStream_t st, const WaitCtl& ctl, bool reuse) {
+  int rc;
   if (!reuse && (rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM,
                                 memM, PM, topk, R, w, st, ctl)))
     return rc;
@@ -518,7 +496,52 @@ int geo_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int l
   return cuda_status(launch_scatter_rows_f32(w.dKg, d, memM, nM, nM, d, dK, lddk, ctl.status, st));
 }
 
+int geo_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv, int nN, int nM,
+            int d, int k, float scale, int dtype, const int* offN, const int* memN, int PN,
+            const int* offM, const int* memM, int PM, const int* topk, int R, const float* O,
+            int ldo, const float* lse, const float* dO, int lddo, float* dQ, int lddq, float* dK,
+            int lddk, float* dV, int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream,
+            bool reuse) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoWs w;
+  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
+  return geo_bwd_run(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, offN, memN, PN, offM,
+                     memM, PM, topk, R, O, ldo, lse, dO, lddo, dQ, lddq, dK, lddk, dV, lddv, w, st,
+                     ctl, reuse);
+}
+
 }  // namespace
+
+int ssc_geo_coupling_fwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
+                         int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
+                         const int* memN, int PN, const int* offM, const int* memM, int PM,
+                         const int* topk, int R, float* O, int ldo, float* lse, void* ws,
+                         size_t ws_bytes, ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, geo_ws(nullptr, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoWs w;
+  geo_ws(ws, nN, nM, d, k, PN, PM, R, dtype, &w);
+  return geo_fwd_run(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, offN, memN, PN, offM, memM,
+                     PM, topk, R, O, ldo, lse, w, st, ctl);
+}
 
 int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const void* V, int ldv,
                          int nN, int nM, int d, int k, float scale, int dtype, const int* offN,
@@ -541,6 +564,288 @@ int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk, c
   return geo_bwd(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, offN, memN, PN, offM, memM, PM,
                  topk, R, O, ldo, lse, dO, lddo, dQ, lddq, dK, lddk, dV, lddv, ws, ws_bytes, stream,
                  true);
+}
+
+// ------------------------------------------------------------ batched pairs
+namespace {
+
+// A batch of pairs stored back to back is one problem of batch times the rows:
+// Q [batch nN, ldq], K and V [batch nM, ld] as matrices.
+bool batch_ok(int batch, int nN, int nM) {
+  return batch >= 1 && (long long)batch * nN <= (1 << 30) && (long long)batch * nM <= (1 << 30);
+}
+
+struct DenseBatchWs {
+  DenseWs w;       // tiles/segs/prefix of the block-diagonal schedule, dOb, Vpad, D
+  void* pair_ws;   // fp32 check mode: the single-pair workspace, reused pair after pair
+};
+
+size_t dense_batch_ws(void* base, int batch, int nN, int nM, int d, int k, int dtype,
+                      DenseBatchWs* out) {
+  Carve c(base);
+  DenseBatchWs x;
+  const int nt = dense_num_tiles(nN), ns = dense_num_segs(nM);
+  x.w.tiles = c.take<RowTile>((size_t)batch * nt);
+  x.w.segs = c.take<KeySeg>((size_t)batch * ns);
+  x.w.prefix = c.take<int>((size_t)batch * nt + 1);
+  x.w.dOb = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)batch * nN * kp_of(k)) : nullptr;
+  x.w.Vpad = dtype == SSC_BF16 ? c.take<__nv_bfloat16>((size_t)batch * nM * kp_of(k)) : nullptr;
+  x.w.D = c.take<float>((size_t)batch * nN);
+  x.w.part = nullptr;
+  const size_t pw = dtype == SSC_F32 ? dense_ws(nullptr, nN, nM, d, k, dtype, nullptr) : 0;
+  x.pair_ws = c.take<uint8_t>(pw);
+  if (out) *out = x;
+  return c.used + 256;
+}
+
+struct GeoBatchWs {
+  int *offN, *memN, *offM, *memM, *topk;  // the concatenated tables
+  GeoWs w;
+};
+
+size_t geo_batch_ws(void* base, int batch, int nN, int nM, int d, int k, int PN, int PM, int R,
+                    int dtype, GeoBatchWs* out) {
+  Carve c(base);
+  GeoBatchWs x;
+  x.offN = c.take<int>((size_t)batch * PN + 1);
+  x.memN = c.take<int>((size_t)batch * nN);
+  x.offM = c.take<int>((size_t)batch * PM + 1);
+  x.memM = c.take<int>((size_t)batch * nM);
+  x.topk = c.take<int>((size_t)batch * PN * R);
+  c.used = round_up(c.used, 256);
+  const size_t g = geo_ws(c.base ? c.base + c.used : nullptr, batch * nN, batch * nM, d, k,
+                          batch * PN, batch * PM, R, dtype, &x.w);
+  c.used += g;
+  if (out) *out = x;
+  return c.used + 256;
+}
+
+// The batched tables: per-shape offsets and members shifted into one problem.
+int geo_batch_tables(int batch, int nN, int nM, const int* offN, const int* memN, int PN,
+                     const int* offM, const int* memM, int PM, const int* topk, int R,
+                     const GeoBatchWs& b, cudaStream_t st, const WaitCtl& ctl) {
+  if (launch_concat_tables(offN, memN, PN, nN, batch, b.offN, b.memN, ctl.status, st) !=
+          cudaSuccess ||
+      launch_concat_tables(offM, memM, PM, nM, batch, b.offM, b.memM, ctl.status, st) !=
+          cudaSuccess ||
+      (topk && launch_concat_topk(topk, PN, R, PM, batch, b.topk, ctl.status, st) != cudaSuccess))
+    return SSC_ERR_CUDA;
+  return SSC_OK;
+}
+
+int check_batched_patches(int batch, const int* offN, const int* memN, int PN, int nN,
+                          const int* offM, const int* memM, int PM, int nM, const int* topk, int R) {
+  if (!batch_ok(batch, nN, nM)) return SSC_ERR_INVALID_ARG;
+  int rc = check_patches(offN, memN, PN, nN, offM, memM, PM, nM, topk, R);
+  if (rc) return rc;
+  if ((long long)batch * PN > 65535 || (long long)batch * PM > 65535) return SSC_ERR_INVALID_ARG;
+  return SSC_OK;
+}
+
+}  // namespace
+
+size_t ssc_dense_coupling_batched_workspace_size(int batch, int nN, int nM, int d, int k,
+                                                 int dtype) {
+  if (!batch_ok(batch, nN, nM) || nN < 1 || nM < 1 || k < 1) return 0;
+  return dense_batch_ws(nullptr, batch, nN, nM, d, k, dtype, nullptr);
+}
+
+int ssc_dense_coupling_fwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                   const void* V, int ldv, int nN, int nM, int d, int k,
+                                   float scale, int dtype, float* O, int ldo, float* lse, void* ws,
+                                   size_t ws_bytes, ssc_stream_t stream) {
+  if (!batch_ok(batch, nN, nM)) return SSC_ERR_INVALID_ARG;
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, dense_batch_ws(nullptr, batch, nN, nM, d, k, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DenseBatchWs b;
+  dense_batch_ws(ws, batch, nN, nM, d, k, dtype, &b);
+  if (dtype == SSC_F32) {
+    // check mode: pair after pair through the single-pair call
+    const size_t pw = dense_ws(nullptr, nN, nM, d, k, dtype, nullptr);
+    const auto* q = static_cast<const float*>(Q);
+    const auto* kk = static_cast<const float*>(K);
+    const auto* v = static_cast<const float*>(V);
+    for (int i = 0; i < batch; ++i)
+      if ((rc = ssc_dense_coupling_fwd(q + (size_t)i * nN * ldq, ldq, kk + (size_t)i * nM * ldk, ldk,
+                                       v + (size_t)i * nM * ldv, ldv, nN, nM, d, k, scale, dtype,
+                                       O + (size_t)i * nN * ldo, ldo, lse + (size_t)i * nN,
+                                       b.pair_ws, pw, stream)))
+        return rc;
+    return SSC_OK;
+  }
+  WaitCtl ctl = make_ctl();
+  cudaError_t e = launch_batched_schedule(batch, nN, nM, b.w.tiles, b.w.segs, b.w.prefix, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, batch * nM, k, b.w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
+           ldvt, batch * nN, batch * nM, d, k, scale, b.w.tiles, b.w.segs, nullptr,
+           batch * dense_num_tiles(nN), b.w.prefix, nullptr, nullptr};
+  return cuda_status(launch_tc_fwd(a, O, ldo, lse, st, ctl));
+}
+
+int ssc_dense_coupling_bwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                   const void* V, int ldv, int nN, int nM, int d, int k,
+                                   float scale, int dtype, const float* O, int ldo,
+                                   const float* lse, const float* dO, int lddo, float* dQ,
+                                   int lddq, float* dK, int lddk, float* dV, int lddv, void* ws,
+                                   size_t ws_bytes, ssc_stream_t stream) {
+  if (!batch_ok(batch, nN, nM)) return SSC_ERR_INVALID_ARG;
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, dense_batch_ws(nullptr, batch, nN, nM, d, k, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DenseBatchWs b;
+  dense_batch_ws(ws, batch, nN, nM, d, k, dtype, &b);
+  if (dtype == SSC_F32) {
+    const size_t pw = dense_ws(nullptr, nN, nM, d, k, dtype, nullptr);
+    const auto* q = static_cast<const float*>(Q);
+    const auto* kk = static_cast<const float*>(K);
+    const auto* v = static_cast<const float*>(V);
+    for (int i = 0; i < batch; ++i)
+      if ((rc = ssc_dense_coupling_bwd(
+               q + (size_t)i * nN * ldq, ldq, kk + (size_t)i * nM * ldk, ldk, v + (size_t)i * nM * ldv,
+               ldv, nN, nM, d, k, scale, dtype, O + (size_t)i * nN * ldo, ldo, lse + (size_t)i * nN,
+               dO + (size_t)i * nN * lddo, lddo, dQ + (size_t)i * nN * lddq, lddq,
+               dK + (size_t)i * nM * lddk, lddk, dV ? dV + (size_t)i * nM * lddv : nullptr, lddv,
+               b.pair_ws, pw, stream)))
+        return rc;
+    return SSC_OK;
+  }
+  WaitCtl ctl = make_ctl();
+  const int kp = (int)kp_of(k);
+  const int rowsN = batch * nN, rowsM = batch * nM;
+  cudaError_t e = launch_batched_schedule(batch, nN, nM, b.w.tiles, b.w.segs, b.w.prefix, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, rowsN, rowsN, k, b.w.dOb, kp, nullptr, 0,
+                           b.w.D, nullptr, ctl.status, st)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dK, lddk, rowsM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dQ, lddq, rowsN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (dV && (e = zero_matrix(dV, lddv, rowsM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, rowsM, k, b.w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
+           ldvt, rowsN, rowsM, d, k, scale, b.w.tiles, b.w.segs, nullptr,
+           batch * dense_num_tiles(nN), b.w.prefix, nullptr, nullptr};
+  // dQ and dK (TMA-reduced into the contiguous key rows), dV query-stationary
+  return cuda_status(launch_tc_bwd(a, b.w.dOb, kp, lse, b.w.D, dQ, lddq, dK, lddk, dV, lddv, st, ctl));
+}
+
+size_t ssc_geo_coupling_batched_workspace_size(int batch, int nN, int nM, int d, int k, int PN,
+                                               int PM, int R, int dtype) {
+  if (!batch_ok(batch, nN, nM) || nN < 1 || nM < 1 || k < 1 || PN < 1 || PM < 1 || R < 1) return 0;
+  return geo_batch_ws(nullptr, batch, nN, nM, d, k, PN, PM, R, dtype, nullptr);
+}
+
+int ssc_geo_coupling_fwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                 const void* V, int ldv, int nN, int nM, int d, int k, float scale,
+                                 int dtype, const int* offN, const int* memN, int PN,
+                                 const int* offM, const int* memM, int PM, const int* topk, int R,
+                                 float* O, int ldo, float* lse, void* ws, size_t ws_bytes,
+                                 ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_batched_patches(batch, offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, geo_batch_ws(nullptr, batch, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoBatchWs b;
+  geo_batch_ws(ws, batch, nN, nM, d, k, PN, PM, R, dtype, &b);
+  if ((rc = geo_batch_tables(batch, nN, nM, offN, memN, PN, offM, memM, PM, topk, R, b, st, ctl)))
+    return rc;
+  return geo_fwd_run(Q, ldq, K, ldk, V, ldv, batch * nN, batch * nM, d, k, scale, dtype, b.offN,
+                     b.memN, batch * PN, b.offM, b.memM, batch * PM, b.topk, R, O, ldo, lse, b.w, st,
+                     ctl);
+}
+
+int ssc_geo_coupling_bwd_batched(int batch, const void* Q, int ldq, const void* K, int ldk,
+                                 const void* V, int ldv, int nN, int nM, int d, int k, float scale,
+                                 int dtype, const int* offN, const int* memN, int PN,
+                                 const int* offM, const int* memM, int PM, const int* topk, int R,
+                                 const float* O, int ldo, const float* lse, const float* dO,
+                                 int lddo, float* dQ, int lddq, float* dK, int lddk, float* dV,
+                                 int lddv, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if ((rc = check_batched_patches(batch, offN, memN, PN, nN, offM, memM, PM, nM, topk, R))) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, geo_batch_ws(nullptr, batch, nN, nM, d, k, PN, PM, R, dtype, nullptr)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  GeoBatchWs b;
+  geo_batch_ws(ws, batch, nN, nM, d, k, PN, PM, R, dtype, &b);
+  if ((rc = geo_batch_tables(batch, nN, nM, offN, memN, PN, offM, memM, PM, topk, R, b, st, ctl)))
+    return rc;
+  return geo_bwd_run(Q, ldq, K, ldk, V, ldv, batch * nN, batch * nM, d, k, scale, dtype, b.offN,
+                     b.memN, batch * PN, b.offM, b.memM, batch * PM, b.topk, R, O, ldo, lse, dO,
+                     lddo, dQ, lddq, dK, lddk, dV, lddv, b.w, st, ctl, false);
+}
+
+size_t ssc_patch_scores_topk_batched_workspace_size(int batch, int nN, int nM, int PN, int PM,
+                                                    int d) {
+  if (batch < 1 || nN < 1 || nM < 1 || PN < 1 || PM < 1 || d < 1) return 0;
+  Carve c(nullptr);
+  c.take<int>((size_t)batch * PN + 1);
+  c.take<int>((size_t)batch * nN);
+  c.take<int>((size_t)batch * PM + 1);
+  c.take<int>((size_t)batch * nM);
+  c.used = round_up(c.used, 256);
+  return c.used + scores_topk_workspace_bytes(PN, PM, d, batch) + 256;
+}
+
+int ssc_patch_scores_topk_batched(int batch, const void* FN, int ldn, int nN, const void* FM,
+                                  int ldm, int nM, int d, int dtype, const int* offN,
+                                  const int* memN, int PN, const int* offM, const int* memM, int PM,
+                                  int R, int* topk, double* scores, void* ws, size_t ws_bytes,
+                                  ssc_stream_t stream) {
+  if (!FN || !FM || !offN || !memN || !offM || !memM || !topk) return SSC_ERR_INVALID_ARG;
+  if (!batch_ok(batch, nN, nM)) return SSC_ERR_INVALID_ARG;
+  if (d < 1 || d > 1024 || ldn < d || ldm < d || nN < 1 || nM < 1) return SSC_ERR_INVALID_ARG;
+  if (dtype != SSC_BF16 && dtype != SSC_F32) return SSC_ERR_INVALID_ARG;
+  if (PN < 1 || PM < 1 || PN > nN || PM > nM || PN > 65535 || PM > 65535) return SSC_ERR_INVALID_ARG;
+  if ((long long)batch * PN > (1 << 30) || (long long)batch * PM > (1 << 30)) return SSC_ERR_INVALID_ARG;
+  if (R < 1 || R > PM) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, ssc_patch_scores_topk_batched_workspace_size(batch, nN, nM, PN, PM, d)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  Carve c(ws);
+  GeoBatchWs b;
+  b.offN = c.take<int>((size_t)batch * PN + 1);
+  b.memN = c.take<int>((size_t)batch * nN);
+  b.offM = c.take<int>((size_t)batch * PM + 1);
+  b.memM = c.take<int>((size_t)batch * nM);
+  c.used = round_up(c.used, 256);
+  int rc = geo_batch_tables(batch, nN, nM, offN, memN, PN, offM, memM, PM, nullptr, R, b, st, ctl);
+  if (rc) return rc;
+  return cuda_status(launch_scores_topk(FN, ldn, nN, FM, ldm, nM, d, dtype, b.offN, b.memN, PN,
+                                        b.offM, b.memM, PM, R, topk, scores, c.base + c.used,
+                                        ctl.status, st, batch));
 }
 
 // ------------------------------------------------------------ linear (ELU)
