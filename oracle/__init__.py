@@ -14,7 +14,8 @@ central finite differences and hand-worked golden cases under tests/golden/.
 from .coupling import dense_fwd, dense_bwd, geo_fwd, geo_bwd, geo_support
 from .patches import fps, csr, pool, scores, topk, patch_pipeline
 from .linear import linear_fwd, linear_bwd
+from .mesh import fps_mesh, sssp
 
 __all__ = ["dense_fwd", "dense_bwd", "geo_fwd", "geo_bwd", "geo_support",
            "fps", "csr", "pool", "scores", "topk", "patch_pipeline",
-           "linear_fwd", "linear_bwd"]
+           "linear_fwd", "linear_bwd", "fps_mesh", "sssp"]

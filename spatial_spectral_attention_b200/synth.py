@@ -169,6 +169,31 @@ def make_workload(name: str, n: int | None = None, seed: int | None = None) -> S
     return make_pair(name=name, **cfg)
 
 
+def sphere_mesh(pts: np.ndarray):
+    """Triangle mesh of points on the unit sphere as an edge graph.
+
+    The convex hull of points on a sphere is their spherical Delaunay
+    triangulation, so its triangles mesh the surface.  Returns the undirected
+    edge graph in CSR form: off int32 [n+1], adj int32 [nnz] (each vertex's
+    neighbours ascending, every edge listed from both ends) and the edge
+    lengths w fp64 [nnz] (Euclidean distance between the fp32 coordinates,
+    the length of the mesh edge)."""
+    from scipy.spatial import ConvexHull
+
+    p32 = np.ascontiguousarray(pts, dtype=np.float32)
+    n = p32.shape[0]
+    tri = ConvexHull(p32.astype(np.float64)).simplices
+    e = np.concatenate([tri[:, [0, 1]], tri[:, [1, 2]], tri[:, [2, 0]]])
+    e = np.concatenate([e, e[:, ::-1]])
+    e = np.unique(e, axis=0)  # sorted by (vertex, neighbour)
+    off = np.zeros(n + 1, np.int64)
+    np.add.at(off, e[:, 0] + 1, 1)
+    off = np.cumsum(off).astype(np.int32)
+    p64 = p32.astype(np.float64)
+    w = np.sqrt(((p64[e[:, 0]] - p64[e[:, 1]]) ** 2).sum(axis=1))
+    return off, e[:, 1].astype(np.int32), w
+
+
 def random_inputs(nN: int, nM: int, d: int, k: int, seed: int, q_scale: float = 1.0):
     """Plain Gaussian Q, K, V, dO (fp32) for shape-edge parity cases."""
     rng = np.random.Generator(np.random.PCG64(seed))
