@@ -117,6 +117,35 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex,
                     int* centers, int* owner, int* offsets, int* members,
                     void* ws, size_t ws_bytes, ssc_stream_t stream);
 
+/* Geodesic patches on a triangle mesh (the digest's "Interpretation":
+ * geodesic farthest-point sampling; project page "Geo-FlashAttention":
+ * geodesic patches), with the geodesic distance read as the shortest path
+ * along mesh edges: edge lengths added in fp64 from the source outward,
+ * minimised over paths.
+ *   adj_off  [n+1] int32, adj [nnz] int32: the edge graph in CSR form (each
+ *            undirected edge listed from both ends; adj_off[0] = 0,
+ *            adj_off[n] = nnz)
+ *   edge_len [nnz] fp64: length of each listed edge (>= 0)
+ * Outputs as ssc_fps_patches: centre t = the vertex farthest from its nearest
+ * centre among 0..t-1 (ties -> lowest vertex index; a vertex no centre
+ * reaches is at +inf, so every connected part receives a centre before any
+ * part receives a second); owner = nearest centre (ties -> lowest patch
+ * index); offsets/members the patch tables.  When P is smaller than the
+ * number of connected parts, vertices no centre reaches keep owner -1 and
+ * are listed in members after the last patch (from offsets[P] to n, in
+ * ascending order), so members is always a permutation of the vertices.
+ * Distances are bit-identical to
+ * Dijkstra's in fp64, so every index is exact.  Requires 1 <= P <= n,
+ * P <= 65535.  Edges with a negative or NaN length or an endpoint out of
+ * range, and offsets out of [0, nnz] or decreasing, are skipped and reported
+ * as SSC_ERR_INVALID_ARG in the device status word. */
+size_t ssc_fps_patches_mesh_workspace_size(int n, int P);
+
+int ssc_fps_patches_mesh(const int* adj_off, const int* adj, const double* edge_len, int n,
+                         int nnz, int P, int seed_vertex, int* centers, int* owner,
+                         int* offsets, int* members, void* ws, size_t ws_bytes,
+                         ssc_stream_t stream);
+
 /* The same patches without a workspace argument, for callers that cannot
  * allocate device memory at all (for instance code embedded in a host program
  * that owns every device allocation and hands over only input and output

@@ -20,7 +20,9 @@
  *    (a vertex no centre reaches has distance +inf, so every connected part
  *    of the mesh receives a centre before a second one in any part);
  *  - the patch of a vertex is its nearest centre, ties to the lowest patch
- *    index (a later centre takes a vertex only when strictly nearer).
+ *    index (a later centre takes a vertex only when strictly nearer); a
+ *    vertex that no centre reaches (fewer centres than connected parts) has
+ *    no patch, owner -1.
  *
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared (see oracle/build.py).
  */

@@ -28,6 +28,8 @@ SIGNATURES = {
     "ssc_fps_patches_workspace_size": (Z, [I, I]),
     "ssc_fps_patches": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
     "ssc_fps_patches_noalloc": (I, [P, I, I, I, P, P, P, P, P]),
+    "ssc_fps_patches_mesh_workspace_size": (Z, [I, I]),
+    "ssc_fps_patches_mesh": (I, [P, P, P, I, I, I, I, P, P, P, P, P, Z, P]),
     "ssc_patch_scores_topk_workspace_size": (Z, [I, I, I]),
     "ssc_patch_scores_topk": (I, [P, I, I, P, I, I, I, I, P, P, I, P, P, I, I, P, P, P, Z, P]),
     "ssc_dense_coupling_workspace_size": (Z, [I, I, I, I, I]),

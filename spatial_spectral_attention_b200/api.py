@@ -129,6 +129,27 @@ def ssc_fps_patches_noalloc(pts, P, seed_vertex=0):
     return centers, owner, offsets, members
 
 
+def ssc_fps_patches_mesh(adj_off, adj, edge_len, P, seed_vertex=0):
+    """Geodesic FPS + patches on a mesh graph: adj_off int32 [n+1], adj int32 [nnz],
+    edge_len fp64 [nnz] (CUDA tensors).  Returns (centers, owner, offsets, members)."""
+    _cuda(adj_off, adj, edge_len)
+    if adj_off.dtype != torch.int32 or adj.dtype != torch.int32 or edge_len.dtype != torch.float64:
+        raise ValueError("adj_off/adj must be int32 and edge_len fp64")
+    adj_off, adj, edge_len = adj_off.contiguous(), adj.contiguous(), edge_len.contiguous()
+    n = adj_off.numel() - 1
+    nnz = adj.numel()
+    dev = adj_off.device
+    centers = torch.empty(P, dtype=torch.int32, device=dev)
+    owner = torch.empty(n, dtype=torch.int32, device=dev)
+    offsets = torch.empty(P + 1, dtype=torch.int32, device=dev)
+    members = torch.empty(n, dtype=torch.int32, device=dev)
+    ws = _workspace(lib().ssc_fps_patches_mesh_workspace_size(n, P), dev)
+    check("ssc_fps_patches_mesh", lib().ssc_fps_patches_mesh(
+        _ptr(adj_off), _ptr(adj), _ptr(edge_len), n, nnz, P, seed_vertex, _ptr(centers),
+        _ptr(owner), _ptr(offsets), _ptr(members), _ptr(ws), ws.numel(), _stream()))
+    return centers, owner, offsets, members
+
+
 def ssc_patch_scores_topk(FN, FM, offN, memN, offM, memM, R, return_scores=False):
     """Patch-mean scores and the top-R source patches of every target patch."""
     _cuda(FN, FM, offN, memN, offM, memM)

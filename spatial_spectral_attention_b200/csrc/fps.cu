@@ -436,6 +436,12 @@ cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* ce
     prof_launch_end(st, SSC_PROF_FPS);
   }
   if (e != cudaSuccess) return e;
+  return launch_patch_tables(owner, n, P, offsets, members, counts, cursor, st);
+}
+
+cudaError_t launch_patch_tables(const int* owner, int n, int P, int* offsets, int* members,
+                                int* counts, int* cursor, cudaStream_t st) {
+  cudaError_t e;
   if ((e = cudaMemsetAsync(counts, 0, sizeof(int) * P, st)) != cudaSuccess) return e;
   const int nb = (int)std::min<long>(1184, (n + 255) / 256);
   count_kernel<<<nb, 256, 0, st>>>(owner, n, counts);

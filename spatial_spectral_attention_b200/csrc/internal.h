@@ -58,6 +58,19 @@ void fps_force_cluster_size(int cl);
 cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* centers, int* owner,
                                int* offsets, int* members, void* ws, cudaStream_t st,
                                const WaitCtl& ctl);
+// Patch tables from owner [n] (every entry in [0, P)): offsets [P+1] and
+// members [n] grouped by patch, ascending vertex id within a patch; counts and
+// cursor are [P] scratch.
+cudaError_t launch_patch_tables(const int* owner, int n, int P, int* offsets, int* members,
+                                int* counts, int* cursor, cudaStream_t st);
+
+// ------------------------------------------------------------ fps_mesh.cu
+size_t fps_mesh_workspace_bytes(int n, int P);
+// Geodesic FPS + nearest-centre patches on a mesh graph (CSR off [n+1], adj
+// [nnz], fp64 edge lengths w [nnz]), then the patch tables.
+cudaError_t launch_fps_mesh(const int* off, const int* adj, const double* w, int n, int nnz, int P,
+                            int seed, int* centers, int* owner, int* offsets, int* members,
+                            void* ws, cudaStream_t st, const WaitCtl& ctl);
 
 // ------------------------------------------------------------ patch_topk.cu
 size_t scores_topk_workspace_bytes(int PN, int PM, int d, int batch = 1);

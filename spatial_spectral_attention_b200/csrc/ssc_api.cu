@@ -263,6 +263,25 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex, int* center
                                         static_cast<cudaStream_t>(stream), c));
 }
 
+size_t ssc_fps_patches_mesh_workspace_size(int n, int P) {
+  if (n < 1 || P < 1) return 0;
+  return fps_mesh_workspace_bytes(n, P);
+}
+
+int ssc_fps_patches_mesh(const int* adj_off, const int* adj, const double* edge_len, int n, int nnz,
+                         int P, int seed_vertex, int* centers, int* owner, int* offsets,
+                         int* members, void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  if (!adj_off || !centers || !owner || !offsets || !members) return SSC_ERR_INVALID_ARG;
+  if (nnz > 0 && (!adj || !edge_len)) return SSC_ERR_INVALID_ARG;
+  if (n < 1 || nnz < 0 || P < 1 || P > n || P > 65535) return SSC_ERR_INVALID_ARG;
+  if (seed_vertex < 0 || seed_vertex >= n) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, fps_mesh_workspace_bytes(n, P))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  WaitCtl c = make_ctl();
+  return cuda_status(launch_fps_mesh(adj_off, adj, edge_len, n, nnz, P, seed_vertex, centers, owner,
+                                     offsets, members, ws, static_cast<cudaStream_t>(stream), c));
+}
+
 size_t ssc_patch_scores_topk_workspace_size(int PN, int PM, int d) {
   if (PN < 1 || PM < 1 || d < 1) return 0;
   return scores_topk_workspace_bytes(PN, PM, d);
