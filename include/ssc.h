@@ -198,7 +198,8 @@ int ssc_debug_fps_cluster_size(int cl);
 #define SSC_PROF_GATHER 8    /* bf16 row gathers (patch-major Q, K, V; V re-pack) */
 #define SSC_PROF_LIN_REDUCE 9 /* linear coupling: phi(X)^T B reductions */
 #define SSC_PROF_LIN_ROWS 10  /* linear coupling: row-tile products (O, dQ, dK, dV) */
-#define SSC_PROF_KERNELS 11
+#define SSC_PROF_BWD_DK 11    /* deterministic backward: key-stationary dK (tc_dk_kernel) */
+#define SSC_PROF_KERNELS 12
 int ssc_profile_enable(int on);
 int ssc_profile_read(int kernel, double* total_ms, int* launches);
 
@@ -250,6 +251,26 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
                            float* dQ, int lddq, float* dK, int lddk,
                            float* dV, int lddv,
                            void* ws, size_t ws_bytes, ssc_stream_t stream);
+
+/* ssc_dense_coupling_bwd with results that are the same bit for bit on
+ * every run (same arguments, same workspace size).  The default backward adds
+ * the dK partials of every query tile in whatever order the reductions
+ * arrive, so its last bits vary from run to run.  This one runs three passes:
+ * dQ query-stationary (the dK work dropped), dK key-stationary (a CTA keeps a
+ * key tile and streams the query tiles past it, recomputing S^T, dP^T and
+ * dS^T), dV key-stationary; each pass uses no more CTAs than there are tiles
+ * of its output, so an output tile receives at most two fp32 additions into
+ * the zeroed result, and two additions commute.  Costs about 1.6x the
+ * flops of the default backward (S and dP are computed twice).  Results
+ * equal the default backward's within the bf16 tolerances.  The fp32 check
+ * mode is already deterministic and is run as is. */
+int ssc_dense_coupling_bwd_deterministic(const void* Q, int ldq, const void* K, int ldk,
+                                         const void* V, int ldv, int nN, int nM, int d, int k,
+                                         float scale, int dtype, const float* O, int ldo,
+                                         const float* lse, const float* dO, int lddo,
+                                         float* dQ, int lddq, float* dK, int lddk,
+                                         float* dV, int lddv,
+                                         void* ws, size_t ws_bytes, ssc_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Geo-FlashAttention (project page, "Geo-FlashAttention"; digest,           */

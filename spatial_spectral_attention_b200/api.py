@@ -60,7 +60,7 @@ def ssc_kernel_launches():
 
 PROF_DENSE_FWD, PROF_FWD, PROF_BWD_DQK, PROF_BWD_DV = 0, 1, 2, 3
 PROF_FPS, PROF_POOL, PROF_SCORES, PROF_TOPK, PROF_GATHER = 4, 5, 6, 7, 8
-PROF_LIN_REDUCE, PROF_LIN_ROWS = 9, 10
+PROF_LIN_REDUCE, PROF_LIN_ROWS, PROF_BWD_DK = 9, 10, 11
 
 
 def ssc_profile_enable(on=True, clear=True):
@@ -188,7 +188,8 @@ def ssc_dense_coupling_fwd(Q, K, V, scale, workspace=None):
     return O, lse
 
 
-def ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=None):
+def ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=None,
+                           deterministic=False):
     """Gradients (dQ, dK, dV or None) of the dense coupling for upstream dO (fp32)."""
     ldq, ldk, ldv, dt = _qkv(Q, K, V)
     _cuda(O, lse, dO)
@@ -201,7 +202,8 @@ def ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=
     O, dO, lse = O.contiguous(), dO.contiguous(), lse.contiguous()
     nb = lib().ssc_dense_coupling_workspace_size(nN, nM, d, k, dt)
     ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
-    check("ssc_dense_coupling_bwd", lib().ssc_dense_coupling_bwd(
+    fn = "ssc_dense_coupling_bwd_deterministic" if deterministic else "ssc_dense_coupling_bwd"
+    check(fn, getattr(lib(), fn)(
         _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale), dt,
         _ptr(O), O.stride(0), _ptr(lse), _ptr(dO), dO.stride(0),
         _ptr(dQ), d, _ptr(dK), d, _ptr(dV), k, _ptr(ws), ws.numel(), _stream()))

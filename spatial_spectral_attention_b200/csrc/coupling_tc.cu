@@ -1025,7 +1025,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG + 128, 1)
 //   dKp  = dS^T Q       (SS, MN-major views) -> flush warpgroup -> dK
 // Shared memory: Q, two K stages, V, dS (no dO tile), which leaves room for
 // the second K stage; a key tile's K load overlaps the previous tile's work.
-template <int NCG, int QCH, int VF, int VR>
+template <int NCG, int QCH, int VF, int VR, bool kNoDK>
 __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     tc_bwd_dqk_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
   static_assert(NCG == 2, "the register split assumes two softmax warpgroups");
@@ -1242,18 +1242,20 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
                    (j > jb || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar_k_empty[st]);
-          // the flush warpgroup has read the previous partial out of TMEM
-          if (it >= 1 && !mbar_wait(&bar_dkp_empty, (it - 1) & 1, p.ctl, abort)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
+          if (!kNoDK) {
+            // the flush warpgroup has read the previous partial out of TMEM
+            if (it >= 1 && !mbar_wait(&bar_dkp_empty, (it - 1) & 1, p.ctl, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // dKp = dS^T Q : A = dS viewed MN-major (M = keys), B = Q MN-major (N = d)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
-                   make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
-          mma_commit(&bar_dkp_full);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + c_dkp, make_sdesc(sS + kk * 2048, kChunk, 1024, kSw128),
+                     make_sdesc(sQ + kk * 2048, kChunk, 1024, kSw128), idesc_dkp, kk > 0);
+            mma_commit(&bar_dkp_full);
+          }
         }
         if (!ok) break;
         mma_commit(&bar_dq_full);
@@ -1419,7 +1421,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     bool ok = true;
     UnitRange ur{s_range[0], s_range[1], s_range[2]};
     int t, jb, je;
-    while (ok && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+    while (ok && !kNoDK && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
       const RowTile tile = p.tiles[t];
       for (int j = jb; j < je; ++j, ++it) {
         const KeySeg sg = p.segs[tile.seg0 + j];
@@ -1875,6 +1877,409 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   }
 }
 
+// ------------------------------------------------------------------ backward, dK (dense, deterministic)
+// Key-stationary dK = scale dS^T Q for the dense coupling: a CTA keeps one key
+// tile (K_j and V_j) and streams the query row tiles i past it,
+//   S^T  = K_j Q_i^T          (SS, both K-major)            -> TMEM [0,128) / [128,256)
+//   dP^T = V_j dO_i^T         (SS, both K-major, K = kp)     -> TMEM [256,384)
+//   P^T  = exp2(S^T s log2e - lse_i log2e),  dS^T = P^T (dP^T - D_i)
+//          -> bf16 pairs over this warpgroup's own S^T columns
+//   dK_j += dS^T Q_i          (TS: dS^T from TMEM, Q_i MN-major) -> TMEM [384, 384 + d)
+// The units (key tile, row tile) are numbered key-tile-major and split evenly
+// over no more CTAs than there are key tiles, so a key tile is shared by at
+// most two CTAs: the first atomic add into the zeroed dK is exact and the
+// second commutes with it, so dK is the same bit for bit on every run.
+// Warps: 0 producer (K_j and V_j once per key tile, Q_i into a 2-stage ring),
+// 1 MMA issuer and TMEM owner, 2..2+4 NWG-1 the dS^T warpgroups (thread = key
+// row; the warpgroups split the 128 query columns), 2+4 NWG the dO producer,
+// whose lanes also stage lse_i log2e (+inf past the last row) and D_i.
+// The MMA issuer runs dP^T_g, dK_{g-1}, S^T_{g+1} per row tile, so dP^T_g
+// overlaps the dS^T work of row tile g-1.
+template <int NWG, int QCH, int VF, int VR>
+__global__ void __launch_bounds__(96 + 128 * NWG, 1)
+    tc_dk_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
+  constexpr bool kFixed = QCH > 0;
+  const int qch = kFixed ? QCH : p.qch;
+  const int vf = kFixed ? VF : p.vf;
+  const int vr = kFixed ? VR : p.vr;
+  const int d16 = kFixed ? 4 * QCH : p.d / 16;
+  constexpr int CW = 128 / NWG;  // query columns per dS^T thread
+  constexpr int NC = CW / 32;
+  constexpr int NSM = 128 * NWG;
+  constexpr int kGWarp = 2 + 4 * NWG;  // dO producer
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_kv_full, bar_kv_empty, bar_q_full[2], bar_q_empty[2], bar_g_full,
+      bar_g_empty, bar_l_full[2], bar_l_empty[2], bar_s_full[2], bar_dp_full, bar_dp_read,
+      bar_p_full[2], bar_dk_full, bar_dk_empty, bar_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ __align__(16) float s_lse2[2][128];  // lse_i log2e of the stage's rows
+  __shared__ __align__(16) float s_D[2][128];     // D_i of the stage's rows
+  __shared__ int s_range[3];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base_u = smem_u32(smem_raw);
+  const uint32_t sbase = (base_u + 1023u) & ~1023u;
+  auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
+  const int qbytes = qch * kChunk;
+  const int vbytes = vtile_bytes(vf, vr);
+  const uint32_t sK = sbase;             // the stationary key tile
+  const uint32_t sV = sK + qbytes;       // its V rows
+  const uint32_t sQ0 = sV + vbytes;      // Q stage s at sQ0 + s * qbytes
+  const int QS = p.vstages;                // Q ring depth (2, or 1 when k is large)
+  const uint32_t sG = sQ0 + QS * qbytes;  // the dO tile (one stage)
+  const int nkt = (p.nk + 127) / 128, nrt = (p.nq + 127) / 128;
+  const uint32_t c_dp = 256, c_dk = 384;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_kv_full, 1);
+    mbar_init(&bar_kv_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_q_full[i], 1);
+      mbar_init(&bar_q_empty[i], 1);
+      mbar_init(&bar_l_full[i], 32);
+      mbar_init(&bar_l_empty[i], NSM);
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_p_full[i], NSM);
+    }
+    mbar_init(&bar_g_full, 1);
+    mbar_init(&bar_g_empty, 1);
+    mbar_init(&bar_dp_full, 1);
+    mbar_init(&bar_dp_read, NSM);
+    mbar_init(&bar_dk_full, 1);
+    mbar_init(&bar_dk_empty, NSM);
+    mbar_init(&bar_drain, 1);
+    s_abort = 0;
+    fence_barrier_init();
+    const long long U = (long long)nkt * nrt;
+    const long long u0 = (long long)blockIdx.x * U / gridDim.x;
+    const long long u1 = (long long)(blockIdx.x + 1) * U / gridDim.x;
+    s_range[0] = nrt > 0 ? (int)(u0 / nrt) : 0;
+    s_range[1] = nrt > 0 ? (int)(u0 % nrt) : 0;
+    s_range[2] = (int)(u1 - u0);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm.q);
+    tma_prefetch_desc(&tm.k);
+    tma_prefetch_desc(&tm.v);
+    tma_prefetch_desc(&tm.g);
+    if (vr) {
+      tma_prefetch_desc(&tm.vr);
+      tma_prefetch_desc(&tm.gr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort = &s_abort;
+
+  if (warp == 0) {
+    // ---------------- producer: K_j and V_j once per key tile, Q_i ring
+    if (lane == 0) {
+      uint32_t g = 0, tcount = 0;
+      int kv_issued = -1;
+      bool ok = true;
+      DvRange r{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && !*abort && dv_next(r, nkt, nrt, t, jb, je)) {
+        if (tcount > 0 && !mbar_wait(&bar_kv_empty, (tcount - 1) & 1, p.ctl, abort)) break;
+        mbar_arrive_expect_tx(&bar_kv_full, qbytes + vbytes);
+        for (int c = 0; c < qch; ++c)
+          tma_load_2d(gptr(sK) + c * kChunk, &tm.k, 64 * c, 128 * t, &bar_kv_full);
+        for (int c = 0; c < vf; ++c)
+          tma_load_2d(gptr(sV) + c * kChunk, &tm.v, 64 * c, 128 * t, &bar_kv_full);
+        if (vr) tma_load_2d(gptr(sV) + vf * kChunk, &tm.vr, 64 * vf, 128 * t, &bar_kv_full);
+        kv_issued = (int)tcount;
+        for (int j = jb; j < je; ++j, ++g) {
+          const int st = g % QS;
+          if (g >= (uint32_t)QS && !mbar_wait(&bar_q_empty[st], ((g / QS) - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_q_full[st], qbytes);
+          for (int c = 0; c < qch; ++c)
+            tma_load_2d(gptr(sQ0 + st * qbytes) + c * kChunk, &tm.q, 64 * c, 128 * j, &bar_q_full[st]);
+        }
+        ++tcount;
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        if (kv_issued >= 0) mbar_wait(&bar_kv_full, kv_issued & 1, p.ctl, &never);
+        for (uint32_t h = g >= (uint32_t)QS ? g - QS : 0; h < g; ++h)
+          mbar_wait(&bar_q_full[h % QS], (h / QS) & 1, p.ctl, &never);
+      }
+    }
+  } else if (warp == kGWarp) {
+    // ---------------- producer: dO_i (one stage, lane 0) and the stage's
+    // lse_i log2e and D_i (all lanes)
+    uint32_t g = 0;
+    bool ok = true;
+    DvRange r{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && !*abort && dv_next(r, nkt, nrt, t, jb, je)) {
+      for (int j = jb; j < je; ++j, ++g) {
+        const int st = g & 1;
+        // the dO stage is free once dP^T of the previous row tile is done; the
+        // lse / D stage once the dS^T of two row tiles back has used it
+        if ((g >= 1 && !mbar_wait(&bar_g_empty, (g - 1) & 1, p.ctl, abort)) ||
+            (g >= 2 && !mbar_wait(&bar_l_empty[st], ((g >> 1) - 1) & 1, p.ctl, abort))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_g_full, vbytes);
+          for (int c = 0; c < vf; ++c)
+            tma_load_2d(gptr(sG) + c * kChunk, &tm.g, 64 * c, 128 * j, &bar_g_full);
+          if (vr) tma_load_2d(gptr(sG) + vf * kChunk, &tm.gr, 64 * vf, 128 * j, &bar_g_full);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = 128 * j + 32 * q + lane;
+          s_lse2[st][32 * q + lane] = row < p.nq ? p.lse_in[row] * kLog2e : INFINITY;
+          s_D[st][32 * q + lane] = row < p.nq ? p.Dvec[row] : 0.f;
+        }
+        mbar_arrive(&bar_l_full[st]);
+      }
+    }
+    if (*abort && lane == 0 && g >= 1) {
+      volatile int never = 0;
+      mbar_wait(&bar_g_full, (g - 1) & 1, p.ctl, &never);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_dk = make_idesc_bf16(128, p.d, 0, 1);
+      const uint32_t rsw = rem_swizzle(vr);
+      const uint32_t rrow = (uint32_t)vr * 2;  // bytes per row of the remainder box
+      uint32_t g0 = 0, tcount = 0;
+      bool ok = true;
+      // S^T_g = K_j Q_g^T into S buffer g & 1 (Q stage g % QS)
+      auto issue_s = [&](uint32_t g) -> bool {
+        const int qs = g % QS;
+        if (!mbar_wait(&bar_q_full[qs], (g / QS) & 1, p.ctl, abort)) return false;
+        tc_fence_after();
+        const uint32_t sq = sQ0 + qs * qbytes;
+#pragma unroll
+        for (int kk = 0; kk < d16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+          mma_ss(tmem + (g & 1) * 128, make_sdesc(sK + off, 16, 1024, kSw128),
+                 make_sdesc(sq + off, 16, 1024, kSw128), idesc_s, kk > 0);
+        }
+        mma_commit(&bar_s_full[g & 1]);
+        return true;
+      };
+      // dK_j += dS^T_g Q_g : A = dS^T (bf16 pairs, each warpgroup's CW query
+      // columns packed at the start of its own CW S columns), B = Q_g MN-major
+      auto issue_dk = [&](uint32_t g, bool first) -> bool {
+        const int st = g & 1, qs = g % QS;
+        if (!mbar_wait(&bar_p_full[st], (g >> 1) & 1, p.ctl, abort)) return false;
+        tc_fence_after();
+        const uint32_t sq = sQ0 + qs * qbytes;
+        const uint32_t a_tmem = tmem + st * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t pcol = 8 * kk + ((16 * kk) / CW) * (CW / 2);
+          mma_ts(tmem + c_dk, a_tmem + pcol, make_sdesc(sq + kk * 2048, kChunk, 1024, kSw128), idesc_dk,
+                 (!first || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bar_q_empty[qs]);
+        return true;
+      };
+      DvRange r{s_range[0], s_range[1], s_range[2]};
+      int t, jb, je;
+      while (ok && dv_next(r, nkt, nrt, t, jb, je)) {
+        const int nu = je - jb;
+        if (!mbar_wait(&bar_kv_full, tcount & 1, p.ctl, abort) ||
+            (tcount > 0 && !mbar_wait(&bar_dk_empty, (tcount - 1) & 1, p.ctl, abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int j = 0; j < min(QS, nu) && ok; ++j) ok = issue_s(g0 + j);
+        for (int j = 0; j < nu && ok; ++j) {
+          const uint32_t g = g0 + j;
+          // dP^T_g = V_j dO_g^T once dO_g is in and dP^T_{g-1} has been read
+          if (!mbar_wait(&bar_g_full, g & 1, p.ctl, abort) ||
+              (g >= 1 && !mbar_wait(&bar_dp_read, (g - 1) & 1, p.ctl, abort))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          int kk = 0;
+#pragma unroll
+          for (int c = 0; c < vf; ++c)
+#pragma unroll
+            for (int u = 0; u < 4; ++u, ++kk) {
+              const uint32_t off = c * kChunk + u * 32;
+              mma_ss(tmem + c_dp, make_sdesc(sV + off, 16, 1024, kSw128),
+                     make_sdesc(sG + off, 16, 1024, kSw128), idesc_s, kk > 0);
+            }
+#pragma unroll
+          for (int u = 0; u < vr / 16; ++u, ++kk) {
+            const uint32_t off = vf * kChunk + u * 32;
+            mma_ss(tmem + c_dp, make_sdesc(sV + off, 16, 8 * rrow, rsw),
+                   make_sdesc(sG + off, 16, 8 * rrow, rsw), idesc_s, kk > 0);
+          }
+          mma_commit(&bar_g_empty);
+          mma_commit(&bar_dp_full);
+          if (QS == 2) {
+            // dK_{g-1}, then S^T_{g+1} into the S buffer dK_{g-1} reads (issued after it)
+            if (j >= 1 && (!issue_dk(g - 1, j == 1) || (j + 1 < nu && !issue_s(g + 1)))) {
+              ok = false;
+              break;
+            }
+          } else {
+            // one Q stage: dK_g must be done with Q_g before Q_{g+1} can load
+            if (!issue_dk(g, j == 0) || (j + 1 < nu && !issue_s(g + 1))) {
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!ok) break;
+        if (QS == 2 && !issue_dk(g0 + nu - 1, nu == 1)) {
+          ok = false;
+          break;
+        }
+        mma_commit(&bar_kv_empty);
+        mma_commit(&bar_dk_full);
+        g0 += nu;
+        ++tcount;
+      }
+      // drain: wait until every tensor-core op issued here has completed
+      mma_commit(&bar_drain);
+      volatile int never = 0;
+      mbar_wait(&bar_drain, 0, p.ctl, &never);
+    }
+  } else if (warp >= 2 && warp < kGWarp) {
+    // ---------------- dS^T (NWG warpgroups): thread = key row (TMEM lane); the
+    // warpgroups split the 128 query columns; epilogue dK per key tile
+    const int wg = (warp - 2) >> 2;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int col0 = wg * CW;
+    uint32_t g0 = 0, tcount = 0;
+    bool ok = true;
+    DvRange r{s_range[0], s_range[1], s_range[2]};
+    int t, jb, je;
+    while (ok && dv_next(r, nkt, nrt, t, jb, je)) {
+      const int nu = je - jb;
+      for (int j = 0; j < nu; ++j) {
+        const uint32_t g = g0 + j;
+        const int buf = g & 1;
+        if (!mbar_wait(&bar_s_full[buf], (g >> 1) & 1, p.ctl, abort) ||
+            !mbar_wait(&bar_l_full[buf], (g >> 1) & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t x[NC][32];
+        const uint32_t sa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(sa + 32 * c, x[c]);
+        tmem_ld_wait();
+        // P^T = exp2(S^T s log2e - lse_i log2e); columns past the last query row
+        // carry lse = +inf and give 0
+        const float4* l4 = reinterpret_cast<const float4*>(&s_lse2[buf][col0]);
+        float pr[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 lv = l4[8 * c + q];
+            pr[c][4 * q] = ex2_approx(fmaf(__uint_as_float(x[c][4 * q]), p.scale_log2, -lv.x));
+            pr[c][4 * q + 1] = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 1]), p.scale_log2, -lv.y));
+            pr[c][4 * q + 2] = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 2]), p.scale_log2, -lv.z));
+            pr[c][4 * q + 3] = ex2_approx(fmaf(__uint_as_float(x[c][4 * q + 3]), p.scale_log2, -lv.w));
+          }
+        if (!mbar_wait(&bar_dp_full, g & 1, p.ctl, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t da = tmem_lane_addr(tmem, warp, c_dp + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(da + 32 * c, x[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_dp_read);  // the dP columns may receive the next dP^T
+        const float4* d4 = reinterpret_cast<const float4*>(&s_D[buf][col0]);
+        uint32_t pk[NC][16];
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 dv = d4[8 * c + q];
+            pk[c][2 * q] = pack_bf16x2(pr[c][4 * q] * (__uint_as_float(x[c][4 * q]) - dv.x),
+                                       pr[c][4 * q + 1] * (__uint_as_float(x[c][4 * q + 1]) - dv.y));
+            pk[c][2 * q + 1] = pack_bf16x2(pr[c][4 * q + 2] * (__uint_as_float(x[c][4 * q + 2]) - dv.z),
+                                           pr[c][4 * q + 3] * (__uint_as_float(x[c][4 * q + 3]) - dv.w));
+          }
+        mbar_arrive(&bar_l_empty[buf]);  // lse and D of this stage are no longer read
+        // packed into the first half of this warpgroup's own S columns (already
+        // read by this thread): the other warpgroup may still be reading its S
+        const uint32_t pa = tmem_lane_addr(tmem, warp, buf * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[buf]);
+      }
+      if (!ok) break;
+      // epilogue: the key tile's dK rows; a key tile shared with another CTA is
+      // added atomically (dK is zeroed by the caller; at most two adds, which
+      // commute)
+      if (!mbar_wait(&bar_dk_full, tcount & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      const int key = 128 * t + lrow;
+      const bool live = key < p.nk;
+      const bool whole = jb == 0 && je == nrt;
+      float* dst = p.dK + (size_t)(live ? key : 0) * p.lddk;
+      const uint32_t ka = tmem_lane_addr(tmem, warp, c_dk);
+      for (int c = wg; c < d16; c += NWG) {
+        uint32_t o[16];
+        tmem_ld16(ka + 16 * c, o);
+        tmem_ld_wait();
+        if (!live) continue;
+        const int c0 = 16 * c;
+        if (p.vec_atomics) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 v = make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                         __uint_as_float(o[i + 2]) * p.scale,
+                                         __uint_as_float(o[i + 3]) * p.scale);
+            if (whole) *reinterpret_cast<float4*>(dst + c0 + i) = v;
+            else atomicAdd(reinterpret_cast<float4*>(dst + c0 + i), v);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (whole) dst[c0 + i] = __uint_as_float(o[i]) * p.scale;
+            else atomicAdd(dst + c0 + i, __uint_as_float(o[i]) * p.scale);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_dk_empty);  // the dK columns may receive the next key tile
+      g0 += nu;
+      ++tcount;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 __global__ void wait_probe_kernel(WaitCtl ctl) {
   __shared__ uint64_t bar;
   __shared__ int s_abort;
@@ -2077,8 +2482,8 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     p.dk_tma = !p.col_map && p.vec_atomics &&
                make_map_f32(&tm.dk, p.dK, a.nKrows, a.d, p.lddk, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
-    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16>
-                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0>;
+    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, false>
+                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     prof_launch_begin(st);
@@ -2107,7 +2512,7 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
 cudaError_t launch_tc_dv_dense(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* dOb, int lddob, const float* lse, int nN,
                                int nM, int d, int k, float scale, float* dV, int lddv,
-                               cudaStream_t st, const WaitCtl& ctl) {
+                               cudaStream_t st, const WaitCtl& ctl, int max_ctas) {
   TcArgs a;
   std::memset(&a, 0, sizeof(a));
   a.Q = Q;
@@ -2143,11 +2548,104 @@ cudaError_t launch_tc_dv_dense(const __nv_bfloat16* Q, int ldq, const __nv_bfloa
   if (smem + (int)fa.sharedSizeBytes > smem_optin()) return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  const int grid = std::max(1, max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms());
   prof_launch_begin(st);
-  kern<<<num_sms(), 96 + 128 * 2, smem, st>>>(tm, p);
+  kern<<<grid, 96 + 128 * 2, smem, st>>>(tm, p);
   prof_launch_end(st, SSC_PROF_BWD_DV);
   count_launch();
   return cudaGetLastError();
+}
+
+cudaError_t launch_tc_bwd_deterministic(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K,
+                                        int ldk, const __nv_bfloat16* V, int ldv,
+                                        const __nv_bfloat16* dOb, int lddob, const float* lse,
+                                        const float* D, const RowTile* tiles, const KeySeg* segs,
+                                        const int* prefix, int nN, int nM, int d, int k,
+                                        float scale, float* dQ, int lddq, float* dK, int lddk,
+                                        float* dV, int lddv, cudaStream_t st, const WaitCtl& ctl) {
+  TcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.ldq = ldq;
+  a.ldk = ldk;
+  a.ldv = ldv;
+  a.nQrows = nN;
+  a.nKrows = nM;
+  a.d = d;
+  a.k = k;
+  a.scale = scale;
+  a.tiles = tiles;
+  a.segs = segs;
+  a.ntiles_host = (nN + 127) / 128;
+  a.tile_prefix = prefix;
+  TcParams p;
+  fill_common(a, p);
+  p.lse_in = lse;
+  p.Dvec = D;
+  p.dQ = dQ;
+  p.lddq = lddq;
+  p.dK = dK;
+  p.lddk = lddk;
+  p.ctl = ctl;
+  p.dOb = dOb;
+  p.lddob = lddob;
+  p.vec_atomics_dq = (lddq % 4 == 0) && (reinterpret_cast<uintptr_t>(dQ) % 16 == 0);
+  p.vec_atomics = (lddk % 4 == 0) && (reinterpret_cast<uintptr_t>(dK) % 16 == 0);
+  TensorMaps tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (!make_map(&tm.q, Q, nN, d, ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.k, K, nM, d, ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.v, V, nM, k, ldv, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm.g, dOb, nN, k, lddob, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (p.vr && (!make_map(&tm.vr, V, nM, k, ldv, p.vr, rem_sw_host(p.vr)) ||
+               !make_map(&tm.gr, dOb, nN, k, lddob, p.vr, rem_sw_host(p.vr))))
+    return cudaErrorInvalidValue;
+  const int vb = vtile_bytes(p.vf, p.vr);
+  const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
+  const int nrt = (nN + 127) / 128, nkt = (nM + 127) / 128;
+  cudaError_t e;
+  {
+    // dQ: no more CTAs than row tiles, so a row tile's dQ gets at most two adds
+    const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
+    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, true>
+                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, true>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    prof_launch_begin(st);
+    kern<<<std::max(1, std::min(num_sms(), nrt)), 128 * (2 + kBwdComputeGroups), smem, st>>>(tm, p);
+    prof_launch_end(st, SSC_PROF_BWD_DQK);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    // dK: key-stationary, no more CTAs than key tiles
+    auto kern = fixed ? tc_dk_kernel<2, 2, 3, 16> : tc_dk_kernel<2, 0, 0, 0>;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    // K and V tiles, two Q stages (one when V rows are long), one dO stage
+    p.vstages = 2;
+    int smem = 1024 + 3 * p.qch * kChunk + 2 * vb;
+    if (smem + (int)fa.sharedSizeBytes > smem_optin()) {
+      p.vstages = 1;
+      smem = 1024 + 2 * p.qch * kChunk + 2 * vb;
+    }
+    if (smem + (int)fa.sharedSizeBytes > smem_optin()) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    prof_launch_begin(st);
+    kern<<<std::max(1, std::min(num_sms(), nkt)), 96 + 128 * 2, smem, st>>>(tm, p);
+    prof_launch_end(st, SSC_PROF_BWD_DK);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (!dV) return cudaSuccess;
+  return launch_tc_dv_dense(Q, ldq, K, ldk, dOb, lddob, lse, nN, nM, d, k, scale, dV, lddv, st, ctl,
+                            nkt);
 }
 
 cudaError_t launch_wait_timeout_probe(cudaStream_t st, const WaitCtl& ctl) {

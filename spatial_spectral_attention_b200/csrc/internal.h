@@ -210,10 +210,24 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
 // Dense dV = P^T dO on tensor cores, key-stationary (dV accumulated per key tile
 // on chip; no partial-dV reductions).  dOb: bf16 dO rows of kp columns, zero
 // padded; lse in row order; dV zeroed by the caller.
+// max_ctas > 0 caps the grid (no more CTAs than key tiles gives every key
+// tile at most two contributions, which makes the result run-to-run exact).
 cudaError_t launch_tc_dv_dense(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk,
                                const __nv_bfloat16* dOb, int lddob, const float* lse, int nN,
                                int nM, int d, int k, float scale, float* dV, int lddv,
-                               cudaStream_t st, const WaitCtl& ctl);
+                               cudaStream_t st, const WaitCtl& ctl, int max_ctas = 0);
+// The dense backward with results identical bit for bit from run to run:
+// dQ query-stationary with each row tile shared by at most two CTAs, dK
+// key-stationary with each key tile shared by at most two CTAs (two fp32 adds
+// into a zeroed output commute), dV likewise.  dQ, dK (and dV) are zeroed by
+// the caller; dOb, lse, D and the dense tile schedule as for launch_tc_bwd.
+cudaError_t launch_tc_bwd_deterministic(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K,
+                                        int ldk, const __nv_bfloat16* V, int ldv,
+                                        const __nv_bfloat16* dOb, int lddob, const float* lse,
+                                        const float* D, const RowTile* tiles, const KeySeg* segs,
+                                        const int* prefix, int nN, int nM, int d, int k,
+                                        float scale, float* dQ, int lddq, float* dK, int lddk,
+                                        float* dV, int lddv, cudaStream_t st, const WaitCtl& ctl);
 // out[map[r]] = in[r] for r < rows (map entries outside [0, dst_rows) are dropped
 // and set the bad-index bit).
 cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, int rows,

@@ -402,6 +402,45 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
                                         nM, d, k, scale, dV, lddv, st, ctl));
 }
 
+int ssc_dense_coupling_bwd_deterministic(const void* Q, int ldq, const void* K, int ldk,
+                                         const void* V, int ldv, int nN, int nM, int d, int k,
+                                         float scale, int dtype, const float* O, int ldo,
+                                         const float* lse, const float* dO, int lddo, float* dQ,
+                                         int lddq, float* dK, int lddk, float* dV, int lddv,
+                                         void* ws, size_t ws_bytes, ssc_stream_t stream) {
+  // the fp32 check mode is deterministic already (query- and key-stationary, no atomics)
+  if (dtype == SSC_F32)
+    return ssc_dense_coupling_bwd(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype, O, ldo, lse, dO,
+                                  lddo, dQ, lddq, dK, lddk, dV, lddv, ws, ws_bytes, stream);
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, dtype);
+  if (rc) return rc;
+  if (!O || !lse || !dO || ldo < k || lddo < k) return SSC_ERR_INVALID_ARG;
+  if ((rc = check_out(dQ, lddq, d)) || (rc = check_out(dK, lddk, d))) return rc;
+  if (dV && (rc = check_out(dV, lddv, k))) return rc;
+  if (!ws_ok(ws, ws_bytes, dense_ws(nullptr, nN, nM, d, k, dtype, nullptr))) return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  DenseWs w;
+  dense_ws(ws, nN, nM, d, k, dtype, &w);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, w.prefix, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  const int kp = (int)kp_of(k);
+  e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
+                      nullptr, ctl.status, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  return cuda_status(launch_tc_bwd_deterministic(
+      static_cast<const __nv_bfloat16*>(Q), ldq, static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt,
+      w.dOb, kp, lse, w.D, w.tiles, w.segs, w.prefix, nN, nM, d, k, scale, dQ, lddq, dK, lddk, dV,
+      lddv, st, ctl));
+}
+
 // ------------------------------------------------------------ geo
 size_t ssc_geo_coupling_workspace_size(int nN, int nM, int d, int k, int PN, int PM, int R,
                                        int dtype) {
