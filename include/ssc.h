@@ -252,6 +252,22 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
                            float* dV, int lddv,
                            void* ws, size_t ws_bytes, ssc_stream_t stream);
 
+/* The dense forward with S = Q K^T on fp8 tensor cores (e4m3 inputs, fp32
+ * accumulation; the pages have no counterpart: a lower-precision variant
+ * whose error against the exact coupling is measured, not a replacement for
+ * the bf16 path).  Q and K (bf16, d = 128) are each divided by their own
+ * scale amax / 448 (amax = largest magnitude of the tensor) and rounded to
+ * e4m3 with saturation; the product is multiplied back by both scales before
+ * the softmax.  P V stays bf16 x bf16.  Same arguments and outputs as
+ * ssc_dense_coupling_fwd (bf16 only, d must be 128, else
+ * SSC_ERR_UNSUPPORTED); its own workspace query. */
+size_t ssc_dense_coupling_fwd_e4m3_workspace_size(int nN, int nM, int d, int k);
+
+int ssc_dense_coupling_fwd_e4m3(const void* Q, int ldq, const void* K, int ldk,
+                                const void* V, int ldv, int nN, int nM, int d, int k,
+                                float scale, float* O, int ldo, float* lse,
+                                void* ws, size_t ws_bytes, ssc_stream_t stream);
+
 /* ssc_dense_coupling_bwd with results that are the same bit for bit on
  * every run (same arguments, same workspace size).  The default backward adds
  * the dK partials of every query tile in whatever order the reductions

@@ -36,6 +36,8 @@ SIGNATURES = {
     "ssc_dense_coupling_fwd": (I, [P, I, P, I, P, I, I, I, I, I, F, I, P, I, P, P, Z, P]),
     "ssc_dense_coupling_bwd": (I, [P, I, P, I, P, I, I, I, I, I, F, I, P, I, P, P, I,
                                    P, I, P, I, P, I, P, Z, P]),
+    "ssc_dense_coupling_fwd_e4m3_workspace_size": (Z, [I, I, I, I]),
+    "ssc_dense_coupling_fwd_e4m3": (I, [P, I, P, I, P, I, I, I, I, I, F, P, I, P, P, Z, P]),
     "ssc_dense_coupling_bwd_deterministic": (I, [P, I, P, I, P, I, I, I, I, I, F, I, P, I, P, P, I,
                                                  P, I, P, I, P, I, P, Z, P]),
     "ssc_geo_coupling_workspace_size": (Z, [I, I, I, I, I, I, I, I]),

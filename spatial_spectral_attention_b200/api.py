@@ -188,6 +188,22 @@ def ssc_dense_coupling_fwd(Q, K, V, scale, workspace=None):
     return O, lse
 
 
+def ssc_dense_coupling_fwd_e4m3(Q, K, V, scale, workspace=None):
+    """Dense forward with Q K^T on e4m3 tensor cores (bf16 Q, K, V; d = 128):
+    O (fp32 [nN,k]) and lse (fp32 [nN])."""
+    ldq, ldk, ldv, dt = _qkv(Q, K, V)
+    nN, d = Q.shape
+    nM, k = V.shape
+    O = torch.empty((nN, k), dtype=torch.float32, device=Q.device)
+    lse = torch.empty(nN, dtype=torch.float32, device=Q.device)
+    nb = lib().ssc_dense_coupling_fwd_e4m3_workspace_size(nN, nM, d, k)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, Q.device)
+    check("ssc_dense_coupling_fwd_e4m3", lib().ssc_dense_coupling_fwd_e4m3(
+        _ptr(Q), ldq, _ptr(K), ldk, _ptr(V), ldv, nN, nM, d, k, float(scale),
+        _ptr(O), k, _ptr(lse), _ptr(ws), ws.numel(), _stream()))
+    return O, lse
+
+
 def ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, scale, need_dV=False, workspace=None,
                            deterministic=False):
     """Gradients (dQ, dK, dV or None) of the dense coupling for upstream dO (fp32)."""

@@ -78,6 +78,7 @@ struct TcParams {
   int nq, nk;        // rows of Q (and of the outputs O, lse, dQ) and of K/V (dK, dV)
   int vstages;       // forward V ring depth
   float scale_log2;  // scale * log2(e)
+  const float* qk_dequant;  // fp8 forward: device factor that turns the e4m3 product into Q K^T
   float scale;
   float* O;
   int ldo;
@@ -126,11 +127,16 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
 // QCH > 0 fixes the operand shape at compile time (d = 64 QCH; V rows of VF
 // full 64-column chunks plus VR remainder columns) so the MMA issue loops are
 // fully unrolled; QCH = 0 reads the shape from the parameters.
-template <int NWG, int QCH, int VF, int VR>
+//
+// kFP8: Q and K arrive as e4m3 copies (d = 128: one 128-byte box per row) and
+// S = Q K^T runs as kind::f8f6f4 MMAs (K = 32 per instruction); the product is
+// multiplied back to Q K^T by the device factor p.qk_dequant, folded into the
+// softmax's exponent scale.  P V stays bf16.
+template <int NWG, int QCH, int VF, int VR, bool kFP8>
 __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     tc_fwd_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
   constexpr bool kFixed = QCH > 0;
-  const int qch = kFixed ? QCH : p.qch;
+  const int qch = kFP8 ? 1 : (kFixed ? QCH : p.qch);
   const int vf = kFixed ? VF : p.vf;
   const int vr = kFixed ? VR : p.vr;
   const int d16 = kFixed ? 4 * QCH : p.d / 16;
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   const uint32_t base_u = smem_u32(smem_raw);
   const uint32_t sbase = (base_u + 1023u) & ~1023u;
   auto gptr = [&](uint32_t sa) { return smem_raw + (sa - base_u); };
-  const int qbytes = qch * kChunk;
+  const int qbytes = kFP8 ? 128 * 128 : qch * kChunk;  // e4m3: 128 rows x 128 bytes
   const int vbytes = vtile_bytes(vf, vr);
   const int VS = p.vstages;  // V ring depth (1 or 2); the K ring has 2 stages
   const uint32_t sQ = sbase;
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_s = kFP8 ? make_idesc_e4m3(128, 128) : make_idesc_bf16(128, 128, 0, 0);
       const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (vf > 0 ? vf : 1), 0, 1);
       const uint32_t idesc_pvr = make_idesc_bf16(128, vr > 0 ? vr : 16, 0, 1);
       const uint32_t o_col = tmem + 256;
@@ -277,11 +283,19 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         tc_fence_after();
         const uint32_t sk = sK0 + st * qbytes;
         const uint32_t d_tmem = tmem + (g & 1) * 128;
+        if (kFP8) {
+          // 4 K-steps of 32 e4m3 values (32 bytes) along the 128-byte rows
 #pragma unroll
-        for (int kk = 0; kk < d16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-          mma_ss(d_tmem, make_sdesc(sQ + off, 16, 1024, kSw128), make_sdesc(sk + off, 16, 1024, kSw128),
-                 idesc_s, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_e4m3(d_tmem, make_sdesc(sQ + kk * 32, 16, 1024, kSw128),
+                        make_sdesc(sk + kk * 32, 16, 1024, kSw128), idesc_s, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < d16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            mma_ss(d_tmem, make_sdesc(sQ + off, 16, 1024, kSw128), make_sdesc(sk + off, 16, 1024, kSw128),
+                   idesc_s, kk > 0);
+          }
         }
         mma_commit(&bar_s_full[g & 1]);
         mma_commit(&bar_k_empty[st]);
@@ -336,6 +350,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = row within the tile
     const int col0 = wg * CW;                 // first S column of this thread
     const int nchunk = p.kp / 16;             // 16-column chunks of O
+    // exponent scale: s log2(e), times the e4m3 dequantisation factor in fp8 mode
+    const float scale_log2 = kFP8 ? p.scale_log2 * *p.qk_dequant : p.scale_log2;
     uint32_t it = 0, tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       const RowTile tile = p.tiles[t];
@@ -383,7 +399,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
 #pragma unroll
           for (int w = 0; w < NWG; ++w) mx = fmaxf(mx, s_pmax[g & 1][w][lrow]);
         }
-        const float m_new = fmaxf(m, mx * p.scale_log2);
+        const float m_new = fmaxf(m, mx * scale_log2);
         const bool need = m_new > m + 8.0f;
         // PV_{g-1} (the previous tile's contribution to O) must be waited for
         // exactly once per tile: the parity wait is only sound when this thread
@@ -424,8 +440,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a0 = ex2_approx(fmaf(x[c][2 * i], p.scale_log2, neg_m));
-            const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], p.scale_log2, neg_m));
+            const float a0 = ex2_approx(fmaf(x[c][2 * i], scale_log2, neg_m));
+            const float a1 = ex2_approx(fmaf(x[c][2 * i + 1], scale_log2, neg_m));
             rs[i & 3] += a0 + a1;
             pk[c][i] = pack_bf16x2(a0, a1);
           }
@@ -2398,34 +2414,61 @@ void fill_common(const TcArgs& a, TcParams& p) {
 
 bool tc_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
 
-cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
-                          const WaitCtl& ctl) {
+namespace {
+
+// e4m3 [rows, cols] (one byte per element) with leading dimension ld bytes,
+// box {128, 128}, 128-byte swizzle; rows past the end read as zero.
+bool make_map_e4m3(CUtensorMap* m, const void* ptr, int rows, int cols, int ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp8: a.Q and a.K point to e4m3 copies (d = 128, ld in bytes) and qk_dequant
+// to the device factor that turns their product into Q K^T.
+cudaError_t launch_fwd_single(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
+                              const WaitCtl& ctl, bool fp8, const float* qk_dequant) {
   TcParams p;
   fill_common(a, p);
   p.O = O;
   p.ldo = ldo;
   p.lse = lse;
   p.ctl = ctl;
+  p.qk_dequant = qk_dequant;
   TensorMaps tm;
   std::memset(&tm, 0, sizeof(tm));
-  if (!make_map(&tm.q, a.Q, a.nQrows, a.d, a.ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm.k, a.K, a.nKrows, a.d, a.ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm.v, a.V, a.nKrows, a.k, a.ldv, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (fp8) {
+    if (a.d != 128 || !make_map_e4m3(&tm.q, a.Q, a.nQrows, a.d, a.ldq) ||
+        !make_map_e4m3(&tm.k, a.K, a.nKrows, a.d, a.ldk))
+      return cudaErrorInvalidValue;
+  } else if (!make_map(&tm.q, a.Q, a.nQrows, a.d, a.ldq, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+             !make_map(&tm.k, a.K, a.nKrows, a.d, a.ldk, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return cudaErrorInvalidValue;
+  }
+  if (!make_map(&tm.v, a.V, a.nKrows, a.k, a.ldv, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (p.vr && !make_map(&tm.vr, a.V, a.nKrows, a.k, a.ldv, p.vr, rem_sw_host(p.vr)))
     return cudaErrorInvalidValue;
   constexpr int NWG = kFwdSoftmaxGroups;
   const bool fixed = p.d == 128 && p.qch == 2 && p.vf == 3 && p.vr == 16;
-  auto kern = fixed ? tc_fwd_kernel<NWG, 2, 3, 16> : tc_fwd_kernel<NWG, 0, 0, 0>;
+  auto kern = fp8 ? (fixed ? tc_fwd_kernel<NWG, 2, 3, 16, true> : tc_fwd_kernel<NWG, 0, 0, 0, true>)
+                 : (fixed ? tc_fwd_kernel<NWG, 2, 3, 16, false> : tc_fwd_kernel<NWG, 0, 0, 0, false>);
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   // two V stages when they fit next to Q and the two K stages, else one
+  const int qtile = fp8 ? 128 * 128 : p.qch * kChunk;
   p.vstages = 2;
-  int smem = 1024 + p.qch * kChunk * 3 + p.vstages * vtile_bytes(p.vf, p.vr);
+  int smem = 1024 + qtile * 3 + p.vstages * vtile_bytes(p.vf, p.vr);
   if (smem + (int)fa.sharedSizeBytes > smem_optin()) {
     p.vstages = 1;
-    smem = 1024 + p.qch * kChunk * 3 + vtile_bytes(p.vf, p.vr);
+    smem = 1024 + qtile * 3 + vtile_bytes(p.vf, p.vr);
   }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -2436,6 +2479,18 @@ cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaSt
   prof_launch_end(st, SSC_PROF_FWD);
   count_launch();
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
+                          const WaitCtl& ctl) {
+  return launch_fwd_single(a, O, ldo, lse, st, ctl, false, nullptr);
+}
+
+cudaError_t launch_tc_fwd_e4m3(const TcArgs& a, const float* qk_dequant, float* O, int ldo,
+                               float* lse, cudaStream_t st, const WaitCtl& ctl) {
+  return launch_fwd_single(a, O, ldo, lse, st, ctl, true, qk_dequant);
 }
 
 cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, const float* lse,

@@ -199,6 +199,18 @@ void prof_launch_end(cudaStream_t st, int kernel);
 bool tc_supported(int d, int k);
 cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
                           const WaitCtl& ctl);
+// The same forward with S = Q K^T on e4m3 tensor cores: a.Q and a.K point to
+// e4m3 copies with d = 128 (ldq, ldk in bytes), qk_dequant to the device
+// factor (scale of Q times scale of K) that restores Q K^T from their product.
+cudaError_t launch_tc_fwd_e4m3(const TcArgs& a, const float* qk_dequant, float* O, int ldo,
+                               float* lse, cudaStream_t st, const WaitCtl& ctl);
+// e4m3 copies of bf16 Q [nN, ldq] and K [nM, ldk] (d columns, rows of d bytes):
+// each tensor divided by its own scale amax / 448 (amax its largest magnitude),
+// rounded to nearest with saturation; *qk_dequant = scale_Q * scale_K.  amax2
+// is [2] scratch.
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16* Q, int ldq, int nN, const __nv_bfloat16* K,
+                                 int ldk, int nM, int d, uint8_t* Q8, uint8_t* K8,
+                                 unsigned* amax2, float* qk_dequant, cudaStream_t st);
 // dQ written (scaled), dK accumulated with atomics (caller zeroes it).
 // dOb: bf16 [nQrows, lddob] (k padded with zeros), lse/D in row order.
 // dK_ord (optional): dK is reduced into this [a.nKrows, d] buffer in the key

@@ -12,6 +12,8 @@
 
 #include <type_traits>
 
+#include <cuda_fp8.h>
+
 #include "internal.h"
 #include "ssc.h"
 
@@ -276,6 +278,36 @@ __global__ void concat_topk_kernel(const int* __restrict__ topk, int PN, int R, 
       out[i] = b * PM + q;
     }
   }
+}
+
+// Largest magnitude of a bf16 matrix [rows, d] (leading dimension ld) into
+// *amax, kept as fp32 bits (non-negative floats order like their bits).
+__global__ void amax_kernel(const __nv_bfloat16* __restrict__ A, int ld, int rows, int d,
+                            unsigned* amax) {
+  float m = 0.f;
+  const long total = (long)rows * d;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x)
+    m = fmaxf(m, fabsf(__bfloat162float(A[(i / d) * ld + i % d])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax, __float_as_uint(m));
+}
+
+// out[r, c] = e4m3(A[r, c] * 448 / amax) with saturation, rows of d bytes.
+__global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ A, int ld, int rows, int d,
+                                     const unsigned* amax, uint8_t* __restrict__ out) {
+  const float am = __uint_as_float(*amax);
+  const float mul = am > 0.f ? 448.0f / am : 1.0f;
+  const long total = (long)rows * d;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x)
+    out[i] = (uint8_t)__nv_cvt_float_to_fp8(__bfloat162float(A[(i / d) * ld + i % d]) * mul,
+                                            __NV_SATFINITE, __NV_E4M3);
+}
+
+// The factor that turns the e4m3 product back into Q K^T: (amaxQ / 448) (amaxK / 448).
+__global__ void dequant_factor_kernel(const unsigned* amax2, float* f) {
+  const float aq = __uint_as_float(amax2[0]), ak = __uint_as_float(amax2[1]);
+  *f = (aq > 0.f ? aq / 448.0f : 1.0f) * (ak > 0.f ? ak / 448.0f : 1.0f);
 }
 
 // prefix[t] = sum of tiles[0..t).nseg for t <= counts[0] (single block).
@@ -578,6 +610,20 @@ cudaError_t launch_concat_topk(const int* topk, int PN, int R, int PM, int batch
   const long m = (long)batch * PN * R;
   concat_topk_kernel<<<grid_for(m, 256), 256, 0, st>>>(topk, PN, R, PM, batch, out, status);
   count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16* Q, int ldq, int nN, const __nv_bfloat16* K,
+                                 int ldk, int nM, int d, uint8_t* Q8, uint8_t* K8,
+                                 unsigned* amax2, float* qk_dequant, cudaStream_t st) {
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(amax2, 0, 2 * sizeof(unsigned), st)) != cudaSuccess) return e;
+  amax_kernel<<<grid_for((long)nN * d, 256), 256, 0, st>>>(Q, ldq, nN, d, amax2);
+  amax_kernel<<<grid_for((long)nM * d, 256), 256, 0, st>>>(K, ldk, nM, d, amax2 + 1);
+  quantize_e4m3_kernel<<<grid_for((long)nN * d, 256), 256, 0, st>>>(Q, ldq, nN, d, amax2, Q8);
+  quantize_e4m3_kernel<<<grid_for((long)nM * d, 256), 256, 0, st>>>(K, ldk, nM, d, amax2 + 1, K8);
+  dequant_factor_kernel<<<1, 1, 0, st>>>(amax2, qk_dequant);
+  count_launch(5);
   return cudaGetLastError();
 }
 

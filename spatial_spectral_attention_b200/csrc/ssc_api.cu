@@ -402,6 +402,54 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
                                         nM, d, k, scale, dV, lddv, st, ctl));
 }
 
+size_t ssc_dense_coupling_fwd_e4m3_workspace_size(int nN, int nM, int d, int k) {
+  if (nN < 1 || nM < 1 || k < 1 || d != 128) return 0;
+  Carve c(nullptr);
+  c.take<uint8_t>((size_t)nN * d);
+  c.take<uint8_t>((size_t)nM * d);
+  c.take<unsigned>(2);
+  c.take<float>(1);
+  c.used = round_up(c.used, 256);
+  return c.used + dense_ws(nullptr, nN, nM, d, k, SSC_BF16, nullptr);
+}
+
+int ssc_dense_coupling_fwd_e4m3(const void* Q, int ldq, const void* K, int ldk, const void* V,
+                                int ldv, int nN, int nM, int d, int k, float scale, float* O,
+                                int ldo, float* lse, void* ws, size_t ws_bytes,
+                                ssc_stream_t stream) {
+  int rc = check_common(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, scale, SSC_BF16);
+  if (rc) return rc;
+  if (d != 128) return SSC_ERR_UNSUPPORTED;
+  if ((rc = check_out(O, ldo, k))) return rc;
+  if (!lse) return SSC_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, ssc_dense_coupling_fwd_e4m3_workspace_size(nN, nM, d, k)))
+    return SSC_ERR_WORKSPACE;
+  (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WaitCtl ctl = make_ctl();
+  Carve c(ws);
+  auto* Q8 = c.take<uint8_t>((size_t)nN * d);
+  auto* K8 = c.take<uint8_t>((size_t)nM * d);
+  auto* amax2 = c.take<unsigned>(2);
+  auto* deq = c.take<float>(1);
+  c.used = round_up(c.used, 256);
+  DenseWs w;
+  dense_ws(c.base + c.used, nN, nM, d, k, SSC_BF16, &w);
+  cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, w.prefix, st);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
+  if ((e = launch_quantize_e4m3(static_cast<const __nv_bfloat16*>(Q), ldq, nN,
+                                static_cast<const __nv_bfloat16*>(K), ldk, nM, d, Q8, K8, amax2, deq,
+                                st)) != cudaSuccess)
+    return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt;
+  int ldvt;
+  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  TcArgs a{reinterpret_cast<const __nv_bfloat16*>(Q8), reinterpret_cast<const __nv_bfloat16*>(K8), Vt,
+           d, d, ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix,
+           nullptr, nullptr};
+  return cuda_status(launch_tc_fwd_e4m3(a, deq, O, ldo, lse, st, ctl));
+}
+
 int ssc_dense_coupling_bwd_deterministic(const void* Q, int ldq, const void* K, int ldk,
                                          const void* V, int ldv, int nN, int nM, int d, int k,
                                          float scale, int dtype, const float* O, int ldo,
