@@ -252,6 +252,158 @@ def geo_tables_flops(offN, offM, topk, d, k, need_dv):
     return pairs, pairs_exec, fpp, bpp
 
 
+def _timed(torch, fn, flush, reps=5, warm=2):
+    """Mean ms of fn() over reps calls, L2 flushed before each, CUDA events on
+    the current stream."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        fn()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
+def _relfro(a, b):
+    return float((a.double() - b.double()).norm() / b.double().norm())
+
+
+def run_extras(api, synth, torch, dev, pk):
+    """The variants beside the headline step, each on its own resident inputs
+    (L2 flushed before every timed call):
+      linear   ELU linear-attention coupling fwd + bwd at 60k and 160k, kernel
+               times and HBM throughput, and the accuracy gap to the exact
+               dense coupling next to Geo's (relative Frobenius of O);
+      deterministic  the run-to-run exact dense backward at 60k;
+      e4m3     the dense forward with Q K^T on fp8 tensor cores at 60k;
+      batched  8 pairs of 10k dense fwd + bwd and 8 pairs of 20k Geo in one call;
+      mesh_fps geodesic FPS on the sphere meshes of the 60k and 160k shapes."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    bf = lambda a: torch.tensor(a).to(torch.bfloat16).to(dev)
+    out = {}
+    # ---- linear coupling and the accuracy gaps
+    lin = []
+    for name in ("geo_60k", "geo_160k_warped"):
+        g = synth.make_workload(name)
+        Q, K, V, dO = bf(g.F_N), bf(g.F_M), bf(g.Phi_M), torch.tensor(g.dO).to(dev)
+        n, d, k = g.n, g.d, g.k
+        ws = torch.empty(api.lib().ssc_linear_coupling_workspace_size(n, n, d, k), dtype=torch.uint8,
+                         device=dev)
+        res = {}
+        fwd_ms = _timed(torch, lambda: api.ssc_linear_coupling_fwd(Q, K, V, workspace=ws), flush)
+        O, den = api.ssc_linear_coupling_fwd(Q, K, V, workspace=ws)
+        bwd_ms = _timed(torch, lambda: api.ssc_linear_coupling_bwd(Q, K, V, O, den, dO, workspace=ws),
+                        flush)
+        api.ssc_profile_enable(True)
+        for _ in range(3):
+            flush.zero_()
+            o2, d2 = api.ssc_linear_coupling_fwd(Q, K, V, workspace=ws)
+            api.ssc_linear_coupling_bwd(Q, K, V, o2, d2, dO, workspace=ws)
+        api.ssc_profile_enable(False)
+        torch.cuda.synchronize()
+        red = api.ssc_profile_read(api.PROF_LIN_REDUCE)
+        rows = api.ssc_profile_read(api.PROF_LIN_ROWS)
+        kv = (k + 1 + 15) // 16 * 16
+        # algorithmic bytes of one fwd + bwd: K,V read twice (both reductions
+        # of K), Q read twice, Y written and read twice, O written, dO and O
+        # read once, dQ and dK written
+        step_bytes = (2.0 * n * (d + k) * 2 + 2.0 * n * d * 2 + 3.0 * n * kv * 2 + 4.0 * n * k
+                      + 8.0 * n * k + 2 * 4.0 * n * d)
+        # exact dense and Geo forwards on the same pair, for the accuracy gap
+        Od, _ = api.ssc_dense_coupling_fwd(Q, K, V, g.scale)
+        _, _, offN, memN = api.ssc_fps_patches(torch.tensor(g.pts_N).to(dev), g.P)
+        _, _, offM, memM = api.ssc_fps_patches(torch.tensor(g.pts_M).to(dev), g.P)
+        topk = api.ssc_patch_scores_topk(Q, K, offN, memN, offM, memM, g.R)
+        Og, _ = api.ssc_geo_coupling_fwd(Q, K, V, g.scale, offN, memN, offM, memM, topk)
+        torch.cuda.synchronize()
+        res.update({"workload": name, "n": n, "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+                    "step_ms": round(fwd_ms + bwd_ms, 4),
+                    "step_gbs": round(step_bytes / ((fwd_ms + bwd_ms) * 1e-3) / 1e9, 1),
+                    "hbm_frac": round(step_bytes / ((fwd_ms + bwd_ms) * 1e-3) / 1e9 / pk["hbm"], 4),
+                    "reduce_kernel_ms": round(red[0] / max(red[1], 1), 4),
+                    "rows_kernel_ms": round(rows[0] / max(rows[1], 1), 4),
+                    "O_relfro_vs_exact_dense": {"linear": round(_relfro(O, Od), 4),
+                                                "geo": round(_relfro(Og, Od), 4)}})
+        lin.append(res)
+        del Q, K, V, dO, ws, O, den, Od, Og
+    out["linear"] = {"sizes": lin, "note": "phi = elu + 1; step bytes = one pass over every "
+                     "operand the two reductions and three row products read or write; the "
+                     "accuracy gap is ||O - O_dense||_F / ||O_dense||_F on the same pair"}
+    # ---- deterministic backward, e4m3 forward (60k dense)
+    g = synth.make_workload("dense_60k")
+    Q, K, V, dO = bf(g.F_N), bf(g.F_M), bf(g.Phi_M), torch.tensor(g.dO).to(dev)
+    wsd = torch.empty(api.lib().ssc_dense_coupling_workspace_size(g.n, g.n, g.d, g.k, 0),
+                      dtype=torch.uint8, device=dev)
+    O, lse = api.ssc_dense_coupling_fwd(Q, K, V, g.scale, workspace=wsd)
+    fpp, bpp = pair_flops(g.d, g.k, False)
+    det = {}
+    for dv in (False, True):
+        ms = _timed(torch, lambda: api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, g.scale, need_dV=dv,
+                                                              workspace=wsd, deterministic=True),
+                    flush, reps=3)
+        det["bwd_dV_ms" if dv else "bwd_ms"] = round(ms, 4)
+    a = api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, g.scale, workspace=wsd, deterministic=True)
+    b = api.ssc_dense_coupling_bwd(Q, K, V, O, lse, dO, g.scale, workspace=wsd, deterministic=True)
+    torch.cuda.synchronize()
+    det["bit_identical_repeat"] = bool(all(torch.equal(x, y) for x, y in zip(a[:2], b[:2])))
+    det["tflops_executed"] = round(float(g.n) * g.n * bpp / (det["bwd_ms"] * 1e-3) / 1e12, 2)
+    det["note"] = ("dQ, key-stationary dK and (with dV) dV passes, no more CTAs than output tiles; "
+                   "tflops on the default backward's executed-flop count")
+    out["deterministic_backward"] = det
+    ms8 = _timed(torch, lambda: api.ssc_dense_coupling_fwd_e4m3(Q, K, V, g.scale), flush, reps=3)
+    O8, _ = api.ssc_dense_coupling_fwd_e4m3(Q, K, V, g.scale)
+    torch.cuda.synchronize()
+    out["e4m3_forward"] = {"fwd_ms": round(ms8, 4),
+                           "tflops": round(float(g.n) * g.n * fpp / (ms8 * 1e-3) / 1e12, 2),
+                           "O_relfro_vs_bf16_forward": round(_relfro(O8, O), 5),
+                           "note": "single-CTA forward with S on kind::f8f6f4 (e4m3, per-tensor "
+                                   "scales); P V bf16"}
+    del Q, K, V, dO, wsd, O, lse, a, b, O8
+    # ---- batches of pairs in one call
+    B = 8
+    g = synth.make_workload("dense_10k")
+    Qb = torch.stack([bf(g.F_N)] * B)
+    Kb = torch.stack([bf(g.F_M)] * B)
+    Vb = torch.stack([bf(g.Phi_M)] * B)
+    dOb = torch.stack([torch.tensor(g.dO).to(dev)] * B)
+    ws = torch.empty(api.lib().ssc_dense_coupling_batched_workspace_size(B, g.n, g.n, g.d, g.k, 0),
+                     dtype=torch.uint8, device=dev)
+
+    def bstep():
+        Ob, lb = api.ssc_dense_coupling_fwd_batched(Qb, Kb, Vb, g.scale, workspace=ws)
+        api.ssc_dense_coupling_bwd_batched(Qb, Kb, Vb, Ob, lb, dOb, g.scale, workspace=ws)
+
+    ms = _timed(torch, bstep, flush, reps=3)
+    fpp, bpp = pair_flops(g.d, g.k, False)
+    out["batched_dense"] = {"pairs": B, "n": g.n, "step_ms": round(ms, 4),
+                            "tflops": round(B * float(g.n) * g.n * (fpp + bpp) / (ms * 1e-3) / 1e12, 2)}
+    del Qb, Kb, Vb, dOb, ws
+    # ---- geodesic FPS on meshes
+    mesh = []
+    for name in ("geo_60k", "geo_160k_warped"):
+        g = synth.make_workload(name)
+        off, adj, w = synth.sphere_mesh(g.pts_N)
+        t = (torch.tensor(off).to(dev), torch.tensor(adj).to(dev), torch.tensor(w).to(dev))
+        api.ssc_fps_patches_mesh(*t, g.P)
+        torch.cuda.synchronize()
+        api.ssc_profile_enable(True)
+        for _ in range(2):
+            api.ssc_fps_patches_mesh(*t, g.P)
+        api.ssc_profile_enable(False)
+        torch.cuda.synchronize()
+        kms, cnt = api.ssc_profile_read(api.PROF_FPS)
+        kms /= max(cnt, 1)
+        mesh.append({"workload": name, "n": g.n, "edges": int(off[-1]) // 2, "P": g.P,
+                     "fps_kernel_ms": round(kms, 3), "us_per_round": round(kms * 1e3 / g.P, 2)})
+    out["mesh_fps"] = mesh
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ws, rank, local):
     import torch
@@ -518,6 +670,8 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
+    if args.extras and rank == 0:
+        res["variants"] = run_extras(api, synth, torch, dev, pk)
     if args.geo_sweep and rank == 0:
         res["geo_sweep"] = {"note": "Geo step vs n, P = n/125, R = 8 (160k: warped pair); "
                                     "peak_gib = peak device memory of the size's inputs, "
@@ -652,6 +806,8 @@ def main():
     ap.add_argument("--workload", default="dense_60k")
     ap.add_argument("--n", type=int, default=None, help="resize the workload (profiling runs)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the linear, deterministic, e4m3, batched and mesh-FPS lines")
     ap.add_argument("--no-geo-sweep", dest="geo_sweep", action="store_false",
                     help="skip the Geo step sweep over n = 20k..160k")
     ap.add_argument("--need-dv", action="store_true")
