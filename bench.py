@@ -54,7 +54,7 @@ def dqk_kernel_hash():
     path = os.path.join(ROOT, "spatial_spectral_attention_b200", "csrc", "coupling_tc.cu")
     try:
         s = open(path).read()
-        i = s.index("template <int NCG, int QCH, int VF, int VR>\n__global__ void "
+        i = s.index("template <int NCG, int QCH, int VF, int VR, bool kNoDK>\n__global__ void "
                     "__launch_bounds__(128 * (2 + NCG), 1)\n    tc_bwd_dqk_kernel(")
         j = s.index("\n}\n", i) + 3
     except (OSError, ValueError):

@@ -122,6 +122,16 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return t[0];
 }
 
+// Row tile of this CTA's r-th pass: the tile list is cut into bands of
+// gridDim.x tiles walked in alternate directions, so that with the tiles
+// sorted by decreasing work (the Geo schedule does that) the passes pair
+// long tiles with short ones.  Every index in [0, ntiles) belongs to exactly
+// one (CTA, pass); a CTA is done at its first index >= ntiles.
+__device__ __forceinline__ int snake_tile(int r) {
+  const int G = gridDim.x, c = blockIdx.x;
+  return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
 // NWG softmax warpgroups split every query row's 128 key columns: thread
 // (wg, lane row) owns columns [wg*CW, (wg+1)*CW) of the S tile, CW = 128/NWG.
 // QCH > 0 fixes the operand shape at compile time (d = 64 QCH; V rows of VF
@@ -206,7 +216,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       int q_issued = -1;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++tcount) {
+      for (int r = 0, t = snake_tile(0); t < ntiles && !*abort; t = snake_tile(++r), ++tcount) {
         const RowTile tile = p.tiles[t];
         if (tcount > 0 && !mbar_wait(&bar_q_empty, (tcount - 1) & 1, p.ctl, abort)) break;
         mbar_arrive_expect_tx(&bar_q_full, qbytes);
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     // reads a stage completes)
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+      for (int r = 0, t = snake_tile(0); t < ntiles && !*abort; t = snake_tile(++r)) {
         const RowTile tile = p.tiles[t];
         bool ok = true;
         for (int j = 0; j < tile.nseg; ++j, ++it) {
@@ -301,7 +311,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         mma_commit(&bar_k_empty[st]);
         return true;
       };
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+      for (int r = 0, t = snake_tile(0); t < ntiles && ok; t = snake_tile(++r), ++tcount) {
         const RowTile tile = p.tiles[t];
         const int nk = tile.nseg;
         if (!mbar_wait(&bar_q_full, tcount & 1, p.ctl, abort)) {
@@ -310,6 +320,9 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         }
         tc_fence_after();
         for (int j = 0; j < std::min(2, nk) && ok; ++j) ok = issue_s(it + j);
+        // Q is free once the tile's last S MMA completes: the next tile's Q
+        // (and its first S MMAs) then overlap this tile's last P.V and epilogue
+        if (ok && nk <= 2) mma_commit(&bar_q_empty);
         for (int j = 0; j < nk && ok; ++j) {
           const uint32_t g = it + j;
           const int buf = g & 1, vst = g % VS;
@@ -334,9 +347,11 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           }
           mma_commit(&bar_v_empty[vst]);
           mma_commit(&bar_o_full);
-          if (j + 2 < nk) ok = issue_s(g + 2);
+          if (j + 2 < nk) {
+            ok = issue_s(g + 2);
+            if (ok && j + 3 == nk) mma_commit(&bar_q_empty);
+          }
         }
-        mma_commit(&bar_q_empty);
         it += nk;
       }
       // drain: wait until every tensor-core op issued here has completed
@@ -353,7 +368,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     // exponent scale: s log2(e), times the e4m3 dequantisation factor in fp8 mode
     const float scale_log2 = kFP8 ? p.scale_log2 * *p.qk_dequant : p.scale_log2;
     uint32_t it = 0, tcount = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+    for (int r = 0, t = snake_tile(0); t < ntiles; t = snake_tile(++r), ++tcount) {
       const RowTile tile = p.tiles[t];
       const int nk = tile.nseg;
       float m = -INFINITY, l = 0.f;

@@ -59,9 +59,22 @@ __device__ __forceinline__ Cand warp_min(Cand c) {
   return c;
 }
 
+// A CTA's candidate as it travels through distributed shared memory: its
+// largest dot, index and coordinates (so the next round needs no global load).
+struct CandXYZ {
+  double val;
+  int idx;
+  float x, y, z;
+};
+
 // Cluster FPS: the CTA of rank r owns points [r*per, min(n,(r+1)*per));
 // their coordinates sit in shared memory (structure of arrays), the running
 // largest dot and patch of each point in registers (PPT points per thread).
+// A round: every thread updates its points and its best candidate; the CTA's
+// warps reduce to one candidate; warp 0 pushes it, with the point's
+// coordinates, into slot `rank` of every CTA; after the cluster barrier warp 0
+// reduces the CL slots and publishes the next centre and its coordinates in
+// shared memory, so no round reads the centre from global memory.
 template <int PPT>
 __global__ void __launch_bounds__(kFpsThreads, 1)
     fps_cluster_kernel(const float* __restrict__ pts, int n, int P, int seed, int per,
@@ -71,8 +84,8 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
   const int rank = (int)cluster.block_rank();
   extern __shared__ float sx[];  // [3][PPT * kFpsThreads]
   __shared__ Cand warp_c[kFpsThreads / 32];
-  __shared__ Cand slots[2][16];
-  __shared__ int s_next;
+  __shared__ CandXYZ slots[2][16];
+  __shared__ CandXYZ s_next;
 
   const int tid = threadIdx.x;
   const int cap = PPT * kFpsThreads;
@@ -94,10 +107,10 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
   }
   __syncthreads();
   int c = seed;
+  float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
+        c2 = __ldg(pts + 3 * (size_t)c + 2);
   for (int t = 0; t < P; ++t) {
     if (rank == 0 && tid == 0) centers[t] = c;
-    const float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
-                c2 = __ldg(pts + 3 * (size_t)c + 2);
     Cand mine{DBL_MAX, INT_MAX};
 #pragma unroll
     for (int i = 0; i < PPT; ++i) {
@@ -124,21 +137,30 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
       Cand w = warp_c[tid];
       w = warp_min(w);
       if (tid < CL) {
-        // push this CTA's candidate into slot `rank` of CTA `tid`
-        Cand* dst = cluster.map_shared_rank(&slots[t & 1][rank], tid);
-        dst->val = w.val;
-        dst->idx = w.idx;
+        // push this CTA's candidate, with its coordinates, into slot `rank` of CTA `tid`
+        CandXYZ cx{w.val, w.idx, 0.f, 0.f, 0.f};
+        if (w.idx != INT_MAX) {
+          const int li = w.idx - v0;
+          cx.x = sx[li];
+          cx.y = sx[cap + li];
+          cx.z = sx[2 * cap + li];
+        }
+        *cluster.map_shared_rank(&slots[t & 1][rank], tid) = cx;
       }
     }
     cluster.sync();
     if (tid < 32) {
+      // warp 0 reduces the CL slots (ties to the lower vertex index)
       Cand w{DBL_MAX, INT_MAX};
-      if (tid < CL) w = slots[t & 1][tid];
-      w = warp_min(w);
-      if (tid == 0) s_next = w.idx;
+      if (tid < CL) w = Cand{slots[t & 1][tid].val, slots[t & 1][tid].idx};
+      const Cand win = warp_min(w);
+      if (tid < CL && slots[t & 1][tid].idx == win.idx) s_next = slots[t & 1][tid];
     }
     __syncthreads();
-    c = s_next;
+    c = s_next.idx;
+    c0 = s_next.x;
+    c1 = s_next.y;
+    c2 = s_next.z;
   }
 #pragma unroll
   for (int i = 0; i < PPT; ++i) {

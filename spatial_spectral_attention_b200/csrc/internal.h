@@ -92,6 +92,12 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
 cudaError_t launch_gather_rows_bf16(const void* in, int in_ld, int in_f32, const int* map, int rows,
                                     int src_rows, int cols, __nv_bfloat16* out, int out_ld,
                                     unsigned* status, cudaStream_t st, int ones_col = -1);
+// Three such gathers (no column of ones) in one launch: job j copies rows[j]
+// rows of in[j] (through map[j]) into out[j].
+cudaError_t launch_gather3_bf16(const __nv_bfloat16* const in[3], const int in_ld[3],
+                                const int* const map[3], const int rows[3], const int src_rows[3],
+                                const int cols[3], __nv_bfloat16* const out[3], const int out_ld[3],
+                                unsigned* status, cudaStream_t st);
 // fp32 variant (check mode).
 cudaError_t launch_gather_rows_f32(const float* in, int in_ld, const int* map, int rows,
                                    int src_rows, int cols, float* out, int out_ld, unsigned* status,

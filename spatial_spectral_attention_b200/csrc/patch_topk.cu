@@ -95,15 +95,31 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// One shape's pooling job: descriptors F [n, ld], patch tables off/mem, P
+// patches, means mu [P, d].
+struct PoolSet {
+  const void* F;
+  const int* off;
+  const int* mem;
+  double* mu;
+  int ld, n, P;
+};
+
+// Blocks [0, set_a.P) pool the first shape, the next set_b.P blocks the second.
 template <bool F32>
-__global__ void __launch_bounds__(128) pool_rows_kernel(const void* __restrict__ F, int ld, int n,
-                                                        int d, const int* __restrict__ off,
-                                                        const int* __restrict__ mem,
-                                                        double* __restrict__ mu, unsigned* status) {
+__global__ void __launch_bounds__(128) pool_rows_kernel(const PoolSet set_a, const PoolSet set_b,
+                                                        int d, unsigned* status) {
   constexpr int kEsz = F32 ? 4 : 2;
   extern __shared__ __align__(16) uint8_t s_rows[];  // [2][kPoolRows][d * kEsz]
   __shared__ int s_mem[kPoolStage];
-  const int p = blockIdx.x;
+  const bool second = (int)blockIdx.x >= set_a.P;
+  const PoolSet& S = second ? set_b : set_a;
+  const int p = second ? blockIdx.x - set_a.P : blockIdx.x;
+  const void* __restrict__ F = S.F;
+  const int ld = S.ld, n = S.n;
+  const int* __restrict__ off = S.off;
+  const int* __restrict__ mem = S.mem;
+  double* __restrict__ mu = S.mu;
   int b = off[p], e = off[p + 1];
   if (b < 0 || e <= b || e > n) {
     if (threadIdx.x == 0) atomicOr(status, kStatusBadIndex);
@@ -150,18 +166,28 @@ __global__ void __launch_bounds__(128) pool_rows_kernel(const void* __restrict__
       __syncthreads();  // ... and every thread's
       const uint8_t* buf = s_rows + (k & 1) * kPoolRows * rowb;
       const int rows = min(kPoolRows, nr - k * kPoolRows);
-      for (int r = 0; r < rows; ++r) {
-        if (s_mem[k * kPoolRows + r] < 0) continue;
+      auto elem = [&](int r, int c) -> double {
         const uint8_t* row = buf + r * rowb;
-        if constexpr (F32) {
-          if (c0 < d) s0 = __dadd_rn(s0, (double)reinterpret_cast<const float*>(row)[c0]);
-          if (c1 < d) s1 = __dadd_rn(s1, (double)reinterpret_cast<const float*>(row)[c1]);
-        } else {
-          if (c0 < d)
-            s0 = __dadd_rn(s0, (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c0]));
-          if (c1 < d)
-            s1 = __dadd_rn(s1, (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c1]));
+        if constexpr (F32) return (double)reinterpret_cast<const float*>(row)[c];
+        else return (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c]);
+      };
+      // eight rows' values read ahead, then added strictly in row order
+      for (int r0 = 0; r0 < rows; r0 += 8) {
+        double x0[8], x1[8];
+        bool ok[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int r = r0 + u;
+          ok[u] = r < rows && s_mem[k * kPoolRows + r] >= 0;
+          x0[u] = (ok[u] && c0 < d) ? elem(r, c0) : 0.0;
+          x1[u] = (ok[u] && c1 < d) ? elem(r, c1) : 0.0;
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (ok[u]) {
+            if (c0 < d) s0 = __dadd_rn(s0, x0[u]);
+            if (c1 < d) s1 = __dadd_rn(s1, x1[u]);
+          }
       }
       __syncthreads();  // buffer k & 1 is refilled by issue(k + 2)
     }
@@ -220,28 +246,25 @@ __device__ __forceinline__ bool pick_before(const Pick& a, const Pick& b) {
   return a.s > b.s || (a.s == b.s && a.q < b.q);
 }
 
-// One block per target patch; round r finds the best candidate ranked after
-// the round r-1 winner, so no candidate needs marking.
-__global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ sc, int PM, int R,
-                                                   int* __restrict__ topk) {
-  __shared__ Pick warp_best[8];
-  __shared__ Pick s_prev;
-  const int p = blockIdx.x;
+// One warp per target patch, eight per block: round r scans the score row for
+// the best candidate ranked after the round r-1 winner and the warp agrees on
+// it by xor-shuffles (every lane ends with the winner), so no block barrier is
+// needed.  Because each round only admits candidates ranked after the previous
+// winner, no candidate needs marking.
+__global__ void __launch_bounds__(256) topk_warp_kernel(const double* __restrict__ sc, int PN, int PM,
+                                                        int R, int* __restrict__ topk) {
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (p >= PN) return;  // warp-uniform
   const double* row = sc + (size_t)p * PM;
   Pick prev{DBL_MAX, -1};
-  bool first = true;
   for (int r = 0; r < R; ++r) {
-    Pick mine{-DBL_MAX, INT_MAX};
-    bool have = false;
-    for (int q = threadIdx.x; q < PM; q += blockDim.x) {
-      Pick c{row[q], q};
-      if (!first && !pick_before(prev, c)) continue;
-      if (!have || pick_before(c, mine)) {
-        mine = c;
-        have = true;
-      }
+    Pick mine{-DBL_MAX, INT_MAX};  // no candidate yet
+    for (int q = lane; q < PM; q += 32) {
+      const Pick c{row[q], q};
+      if (r > 0 && !pick_before(prev, c)) continue;
+      if (mine.q == INT_MAX || pick_before(c, mine)) mine = c;
     }
-    if (!have) mine = Pick{-DBL_MAX, INT_MAX};
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       Pick x;
@@ -249,21 +272,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ sc
       x.q = __shfl_xor_sync(0xffffffffu, mine.q, o);
       if (x.q != INT_MAX && (mine.q == INT_MAX || pick_before(x, mine))) mine = x;
     }
-    if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = mine;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      Pick w = warp_best[0];
-      for (int i = 1; i < (int)(blockDim.x / 32); ++i) {
-        Pick x = warp_best[i];
-        if (x.q != INT_MAX && (w.q == INT_MAX || pick_before(x, w))) w = x;
-      }
-      s_prev = w;
-      topk[(size_t)p * R + r] = w.q;
-    }
-    __syncthreads();
-    prev = s_prev;
-    first = false;
-    __syncthreads();
+    if (lane == 0) topk[(size_t)p * R + r] = mine.q;
+    prev = mine;
   }
 }
 
@@ -296,28 +306,31 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   };
   const int rows_smem = 2 * kPoolRows * d * esz;
   auto pool = [&](const void* F, int ld, int n, int P, const int* off, const int* mem, double* mu) {
-    cudaError_t e;
-    if (staged(F, ld)) {
-      auto kern = dtype == 1 ? pool_rows_kernel<true> : pool_rows_kernel<false>;
-      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem)) !=
-          cudaSuccess)
-        return e;
-      prof_launch_begin(st);
-      kern<<<P, 128, rows_smem, st>>>(F, ld, n, d, off, mem, mu, status);
-    } else if (dtype == 1) {
-      prof_launch_begin(st);
-      pool_kernel<true><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
-    } else {
-      prof_launch_begin(st);
-      pool_kernel<false><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
-    }
+    prof_launch_begin(st);
+    if (dtype == 1) pool_kernel<true><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
+    else pool_kernel<false><<<P, pt, 0, st>>>(F, ld, n, d, off, mem, mu, status);
     prof_launch_end(st, SSC_PROF_POOL);
     count_launch();
     return cudaGetLastError();
   };
   cudaError_t pe;
-  if ((pe = pool(FN, ldn, batch * nN, batch * PN, offN, memN, muN)) != cudaSuccess) return pe;
-  if ((pe = pool(FM, ldm, batch * nM, batch * PM, offM, memM, muM)) != cudaSuccess) return pe;
+  if (staged(FN, ldn) && staged(FM, ldm)) {
+    // both shapes in one launch, member rows staged through shared memory
+    auto kern = dtype == 1 ? pool_rows_kernel<true> : pool_rows_kernel<false>;
+    if ((pe = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem)) !=
+        cudaSuccess)
+      return pe;
+    const PoolSet a{FN, offN, memN, muN, ldn, batch * nN, batch * PN};
+    const PoolSet b{FM, offM, memM, muM, ldm, batch * nM, batch * PM};
+    prof_launch_begin(st);
+    kern<<<batch * (PN + PM), 128, rows_smem, st>>>(a, b, d, status);
+    prof_launch_end(st, SSC_PROF_POOL);
+    count_launch();
+    if ((pe = cudaGetLastError()) != cudaSuccess) return pe;
+  } else {
+    if ((pe = pool(FN, ldn, batch * nN, batch * PN, offN, memN, muN)) != cudaSuccess) return pe;
+    if ((pe = pool(FM, ldm, batch * nM, batch * PM, offM, memM, muM)) != cudaSuccess) return pe;
+  }
   dim3 grid((PM + kST - 1) / kST, (PN + kST - 1) / kST, batch);
   const int sc_smem = 2 * kST * (kSC + 1) * (int)sizeof(double);
   if ((pe = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -328,7 +341,7 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   prof_launch_end(st, SSC_PROF_SCORES);
   count_launch();
   prof_launch_begin(st);
-  topk_kernel<<<batch * PN, 256, 0, st>>>(sc, PM, R, topk);
+  topk_warp_kernel<<<(batch * PN + 7) / 8, 256, 0, st>>>(sc, batch * PN, PM, R, topk);
   prof_launch_end(st, SSC_PROF_TOPK);
   count_launch();
   return cudaGetLastError();

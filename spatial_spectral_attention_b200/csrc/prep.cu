@@ -117,6 +117,80 @@ __global__ void gather_bf16_pieces(const __nv_bfloat16* __restrict__ in, int in_
   }
 }
 
+// Up to three bf16 row gathers in one launch (the patch-major Q, K and V of
+// Geo-FlashAttention).  Job j covers the global pieces [begin_j, begin_j+1);
+// its pieces are `vec` elements wide (8: 16 bytes, 4: 8 bytes, 1: one
+// element).  Each thread loads four pieces before it stores them, so four
+// loads per thread are in flight.  Semantics per job as gather_bf16_pieces.
+struct GatherJob {
+  const __nv_bfloat16* in;
+  const int* map;
+  __nv_bfloat16* out;
+  int in_ld, rows, src_rows, cols, out_ld, vec;
+  long long begin;
+};
+struct GatherJobs {
+  GatherJob j[3];
+  long long end;
+};
+
+__device__ __forceinline__ uint4 gather_piece(const GatherJob& g, int i, unsigned* status,
+                                              __nv_bfloat16** dst) {
+  const int pieces = g.out_ld / g.vec;
+  const int li = i - (int)g.begin;
+  const int r = li / pieces;
+  const int c0 = (li - r * pieces) * g.vec;
+  const int src = checked_src(g.map, r, g.src_rows, status);
+  *dst = g.out + (size_t)r * g.out_ld + c0;
+  if (src >= 0 && c0 + g.vec <= g.cols) {
+    const __nv_bfloat16* a = g.in + (size_t)src * g.in_ld + c0;
+    if (g.vec == 8) return __ldg(reinterpret_cast<const uint4*>(a));
+    if (g.vec == 4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(a));
+      return make_uint4(v.x, v.y, 0u, 0u);
+    }
+    return make_uint4(__bfloat16_as_ushort(a[0]), 0u, 0u, 0u);
+  }
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  for (int e = 0; e < g.vec; ++e) {
+    const int c = c0 + e;
+    const uint32_t h = (src >= 0 && c < g.cols) ? __bfloat16_as_ushort(g.in[(size_t)src * g.in_ld + c]) : 0u;
+    w[e >> 1] |= h << (16 * (e & 1));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void put_piece(__nv_bfloat16* dst, int vec, uint4 v) {
+  if (vec == 8) *reinterpret_cast<uint4*>(dst) = v;
+  else if (vec == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(v.x, v.y);
+  else *dst = __ushort_as_bfloat16((unsigned short)(v.x & 0xffffu));
+}
+
+// 32-bit piece indices (the launcher falls back to one launch per job when
+// the pieces do not fit).
+__global__ void gather_jobs_kernel(const GatherJobs jobs, unsigned* status) {
+  const int stride = gridDim.x * blockDim.x;
+  const int end = (int)jobs.end, b1 = (int)jobs.j[1].begin, b2 = (int)jobs.j[2].begin;
+  for (int i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < end; i0 += 4 * stride) {
+    uint4 v[4];
+    __nv_bfloat16* dst[4];
+    int vec[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * stride;
+      vec[u] = 0;
+      if (i < end) {
+        const int jj = i < b1 ? 0 : (i < b2 ? 1 : 2);
+        vec[u] = jobs.j[jj].vec;
+        v[u] = gather_piece(jobs.j[jj], i, status, &dst[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (vec[u]) put_piece(dst[u], vec[u], v[u]);
+  }
+}
+
 __global__ void gather_bf16_from_f32(const float* __restrict__ in, int in_ld,
                                      const int* __restrict__ map, int rows, int src_rows, int cols,
                                      __nv_bfloat16* __restrict__ out, int out_ld, unsigned* status) {
@@ -310,57 +384,6 @@ __global__ void dequant_factor_kernel(const unsigned* amax2, float* f) {
   *f = (aq > 0.f ? aq / 448.0f : 1.0f) * (ak > 0.f ? ak / 448.0f : 1.0f);
 }
 
-// prefix[t] = sum of tiles[0..t).nseg for t <= counts[0] (single block).
-__global__ void __launch_bounds__(1024) tile_prefix_kernel(const RowTile* __restrict__ tiles,
-                                                           const int* __restrict__ counts,
-                                                           int* __restrict__ prefix) {
-  __shared__ int part[1024];
-  const int m = counts[0];
-  const int tid = threadIdx.x;
-  const int per = (m + 1023) / 1024;
-  const int lo = tid * per, hi = min(m, lo + per);
-  int s = 0;
-  for (int i = lo; i < hi; ++i) s += tiles[i].nseg;
-  part[tid] = s;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {
-    const int x = tid >= o ? part[tid - o] : 0;
-    __syncthreads();
-    part[tid] += x;
-    __syncthreads();
-  }
-  int r = part[tid] - s;
-  for (int i = lo; i < hi; ++i) {
-    prefix[i] = r;
-    r += tiles[i].nseg;
-  }
-  if (tid == 1023) prefix[m] = part[1023];
-}
-
-// pieces[p] = row tiles of target patch p; nsegs[p] = 128-row pieces of its
-// selected source patches.
-__global__ void geo_count_kernel(const int* __restrict__ offN, int PN, int nN,
-                                 const int* __restrict__ offM, int PM, int nM,
-                                 const int* __restrict__ topk, int R, int* __restrict__ pieces,
-                                 int* __restrict__ nsegs, unsigned* status) {
-  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < PN; p += gridDim.x * blockDim.x) {
-    const int2 pr = patch_range(offN, p, nN, status);
-    const int rows = pr.y - pr.x;
-    pieces[p] = (rows + kTileRows - 1) / kTileRows;
-    int s = 0;
-    for (int r = 0; r < R; ++r) {
-      const int q = topk[(size_t)p * R + r];
-      if (q < 0 || q >= PM) {
-        atomicOr(status, kStatusBadIndex);
-        continue;
-      }
-      const int2 qr = patch_range(offM, q, nM, status);
-      s += (qr.y - qr.x + kTileRows - 1) / kTileRows;
-    }
-    nsegs[p] = s;
-  }
-}
-
 // Single-block exclusive scan of two int arrays of length m; totals[0..1].
 __global__ void __launch_bounds__(1024) scan2_kernel(const int* __restrict__ a, const int* __restrict__ b,
                                                      int m, int* __restrict__ abase,
@@ -400,15 +423,133 @@ __global__ void __launch_bounds__(1024) scan2_kernel(const int* __restrict__ a, 
   }
 }
 
-// Writes beyond the capacities (possible only for inconsistent tables, e.g.
-// repeated entries in a topk row) are dropped and set the bad-index bit.
-__global__ void geo_fill_kernel(const int* __restrict__ offN, int PN, int nN,
-                                const int* __restrict__ offM, int PM, int nM,
-                                const int* __restrict__ topk, int R, unsigned* status,
-                                const int* __restrict__ tbase, const int* __restrict__ sbase,
-                                const int* __restrict__ nsegs, RowTile* __restrict__ tiles,
-                                KeySeg* __restrict__ segs, int tile_cap, int seg_cap) {
-  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < PN; p += gridDim.x * blockDim.x) {
+// Block-wide exclusive scan of v[0..m) into base[0..m) by one block of
+// kSchedThreads threads (each thread a contiguous run); returns the total.
+constexpr int kSchedThreads = 1024;
+__device__ int block_scan(const int* v, int m, int* base, int* part) {
+  const int tid = threadIdx.x;
+  const int per = (m + kSchedThreads - 1) / kSchedThreads;
+  const int lo = min(m, tid * per), hi = min(m, lo + per);
+  int sacc = 0;
+  for (int i = lo; i < hi; ++i) sacc += v[i];
+  part[tid] = sacc;
+  __syncthreads();
+  for (int o = 1; o < kSchedThreads; o <<= 1) {
+    const int x = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += x;
+    __syncthreads();
+  }
+  int r = part[tid] - sacc;
+  for (int i = lo; i < hi; ++i) {
+    base[i] = r;
+    r += v[i];
+  }
+  const int total = part[kSchedThreads - 1];
+  __syncthreads();  // part is reused by the next scan
+  return total;
+}
+
+// Exclusive prefix of the row tiles with the target patches ordered by
+// decreasing segment count (ties by patch index): base[i] is the first tile of
+// patch i.  Sort key: the patch's segment count below the largest, capped at
+// 7, so the seven largest counts get a bucket each and the rest share the
+// last one.  The eight per-bucket running counts are 16-bit fields of a
+// ulonglong2 (the caller guarantees fewer than 65536 tiles), scanned like
+// block_scan's ints.  Returns the total.
+__device__ __forceinline__ int tile_bucket(int nseg, int maxseg) { return min(7, maxseg - nseg); }
+__device__ __forceinline__ ulonglong2 bucket_field(int b, int count) {
+  const unsigned long long v = (unsigned long long)count << (16 * (b & 3));
+  return b < 4 ? make_ulonglong2(v, 0ull) : make_ulonglong2(0ull, v);
+}
+__device__ __forceinline__ int bucket_count(const ulonglong2& x, int b) {
+  return (int)(((b < 4 ? x.x : x.y) >> (16 * (b & 3))) & 0xffffull);
+}
+__device__ int sorted_tile_scan(const int* pieces, const int* nsegs, int m, int maxseg, int* base,
+                                ulonglong2* part) {
+  const int tid = threadIdx.x;
+  const int per = (m + kSchedThreads - 1) / kSchedThreads;
+  const int lo = min(m, tid * per), hi = min(m, lo + per);
+  ulonglong2 acc = make_ulonglong2(0ull, 0ull);
+  for (int i = lo; i < hi; ++i) {
+    const ulonglong2 f = bucket_field(tile_bucket(nsegs[i], maxseg), pieces[i]);
+    acc.x += f.x;
+    acc.y += f.y;
+  }
+  part[tid] = acc;
+  __syncthreads();
+  for (int o = 1; o < kSchedThreads; o <<= 1) {
+    const ulonglong2 x = tid >= o ? part[tid - o] : make_ulonglong2(0ull, 0ull);
+    __syncthreads();
+    part[tid].x += x.x;
+    part[tid].y += x.y;
+    __syncthreads();
+  }
+  ulonglong2 r = make_ulonglong2(part[tid].x - acc.x, part[tid].y - acc.y);
+  const ulonglong2 tot = part[kSchedThreads - 1];
+  int start[8], total = 0;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    start[b] = total;
+    total += bucket_count(tot, b);
+  }
+  for (int i = lo; i < hi; ++i) {
+    const int b = tile_bucket(nsegs[i], maxseg);
+    int sb = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u == b) sb = start[u];
+    base[i] = sb + bucket_count(r, b);
+    const ulonglong2 f = bucket_field(b, pieces[i]);
+    r.x += f.x;
+    r.y += f.y;
+  }
+  __syncthreads();  // part is reused
+  return total;
+}
+
+// The whole Geo schedule in one block: per target patch its row tiles and
+// source segments (counts), their exclusive scans, the tile and segment
+// lists (row tiles by decreasing segment count), the clamped totals and the
+// tiles' segment prefix sums, in one launch.
+__global__ void __launch_bounds__(kSchedThreads) geo_schedule_kernel(
+    const int* __restrict__ offN, int PN, int nN, const int* __restrict__ offM, int PM, int nM,
+    const int* __restrict__ topk, int R, RowTile* __restrict__ tiles, KeySeg* __restrict__ segs,
+    int* __restrict__ counts, int* __restrict__ prefix, int* __restrict__ pieces,
+    int* __restrict__ nsegs, int* __restrict__ tbase, int* __restrict__ sbase, int tile_cap,
+    int seg_cap, unsigned* status) {
+  __shared__ int part[kSchedThreads];
+  __shared__ ulonglong2 part2[kSchedThreads];
+  __shared__ int s_maxseg, s_tiles;
+  if (threadIdx.x == 0) {
+    s_maxseg = 0;
+    s_tiles = 0;
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < PN; p += kSchedThreads) {
+    const int2 pr = patch_range(offN, p, nN, status);
+    pieces[p] = (pr.y - pr.x + kTileRows - 1) / kTileRows;
+    int sacc = 0;
+    for (int r = 0; r < R; ++r) {
+      const int q = topk[(size_t)p * R + r];
+      if (q < 0 || q >= PM) {
+        atomicOr(status, kStatusBadIndex);
+        continue;
+      }
+      const int2 qr = patch_range(offM, q, nM, status);
+      sacc += (qr.y - qr.x + kTileRows - 1) / kTileRows;
+    }
+    nsegs[p] = sacc;
+    atomicMax(&s_maxseg, sacc);
+    atomicAdd(&s_tiles, pieces[p]);
+  }
+  __syncthreads();
+  // row tiles ordered by decreasing segment count, so that the forward's
+  // alternating walk over bands of tiles balances the CTAs
+  const int ntile = s_tiles < 65536 ? sorted_tile_scan(pieces, nsegs, PN, s_maxseg, tbase, part2)
+                                    : block_scan(pieces, PN, tbase, part);
+  const int nseg = block_scan(nsegs, PN, sbase, part);
+  for (int p = threadIdx.x; p < PN; p += kSchedThreads) {
     const int2 pr = patch_range(offN, p, nN, status);
     const int r0 = pr.x, rows = pr.y - pr.x;
     const int sb = sbase[p];
@@ -421,21 +562,41 @@ __global__ void geo_fill_kernel(const int* __restrict__ offN, int PN, int nN,
       }
       tiles[tbase[p] + i] = RowTile{r0 + t, min(kTileRows, rows - t), sb, ns};
     }
-    int s = sb;
+    int sidx = sb;
     for (int r = 0; r < R; ++r) {
       const int q = topk[(size_t)p * R + r];
       if (q < 0 || q >= PM) continue;
       const int2 qr = patch_range(offM, q, nM, status);
       const int k0 = qr.x, kn = qr.y - qr.x;
-      for (int u = 0; u < kn && s < sb + ns; u += kTileRows)
-        segs[s++] = KeySeg{k0 + u, min(kTileRows, kn - u)};
+      for (int u = 0; u < kn && sidx < sb + ns; u += kTileRows)
+        segs[sidx++] = KeySeg{k0 + u, min(kTileRows, kn - u)};
     }
   }
-}
-
-__global__ void clamp_counts_kernel(int* counts, int tile_cap, int seg_cap) {
-  counts[0] = min(counts[0], tile_cap);
-  counts[1] = min(counts[1], seg_cap);
+  const int m = min(ntile, tile_cap);
+  if (threadIdx.x == 0) {
+    counts[0] = m;
+    counts[1] = min(nseg, seg_cap);
+  }
+  __syncthreads();  // the tile list is complete
+  // prefix[t] = segments of tiles[0..t)
+  const int per = (m + kSchedThreads - 1) / kSchedThreads;
+  const int lo = min(m, (int)threadIdx.x * per), hi = min(m, lo + per);
+  int sacc = 0;
+  for (int i = lo; i < hi; ++i) sacc += tiles[i].nseg;
+  part[threadIdx.x] = sacc;
+  __syncthreads();
+  for (int o = 1; o < kSchedThreads; o <<= 1) {
+    const int x = (int)threadIdx.x >= o ? part[threadIdx.x - o] : 0;
+    __syncthreads();
+    part[threadIdx.x] += x;
+    __syncthreads();
+  }
+  int r = part[threadIdx.x] - sacc;
+  for (int i = lo; i < hi; ++i) {
+    prefix[i] = r;
+    r += tiles[i].nseg;
+  }
+  if (threadIdx.x == kSchedThreads - 1) prefix[m] = part[kSchedThreads - 1];
 }
 
 __global__ void inv_count_kernel(const int* __restrict__ topk, int n, int PM, int* __restrict__ cnt) {
@@ -551,6 +712,48 @@ cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, 
   return cudaGetLastError();
 }
 
+cudaError_t launch_gather3_bf16(const __nv_bfloat16* const in[3], const int in_ld[3],
+                                const int* const map[3], const int rows[3], const int src_rows[3],
+                                const int cols[3], __nv_bfloat16* const out[3], const int out_ld[3],
+                                unsigned* status, cudaStream_t st) {
+  GatherJobs jobs;
+  long long begin = 0;
+  for (int j = 0; j < 3; ++j) {
+    GatherJob& g = jobs.j[j];
+    const uintptr_t ia = reinterpret_cast<uintptr_t>(in[j]), oa = reinterpret_cast<uintptr_t>(out[j]);
+    g.vec = (in_ld[j] % 8 == 0 && out_ld[j] % 8 == 0 && ia % 16 == 0 && oa % 16 == 0)   ? 8
+            : (in_ld[j] % 4 == 0 && out_ld[j] % 4 == 0 && ia % 8 == 0 && oa % 8 == 0) ? 4
+                                                                                      : 1;
+    g.in = in[j];
+    g.map = map[j];
+    g.out = out[j];
+    g.in_ld = in_ld[j];
+    g.rows = rows[j];
+    g.src_rows = src_rows[j];
+    g.cols = cols[j];
+    g.out_ld = out_ld[j];
+    g.begin = begin;
+    begin += (long long)rows[j] * (out_ld[j] / g.vec);
+  }
+  jobs.end = begin;
+  if (begin == 0) return cudaSuccess;
+  if (begin >= (1LL << 30)) {
+    // too many pieces for 32-bit indices: one launch per matrix
+    for (int j = 0; j < 3; ++j) {
+      const cudaError_t e = launch_gather_rows_bf16(in[j], in_ld[j], 0, map[j], rows[j], src_rows[j],
+                                                    cols[j], out[j], out_ld[j], status, st);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((begin + 1023) / 1024, 148LL * 8));
+  prof_launch_begin(st);
+  gather_jobs_kernel<<<blocks, 256, 0, st>>>(jobs, status);
+  prof_launch_end(st, SSC_PROF_GATHER);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather_rows_f32(const float* in, int in_ld, const int* map, int rows,
                                    int src_rows, int cols, float* out, int out_ld, unsigned* status,
                                    cudaStream_t st) {
@@ -642,19 +845,10 @@ cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM
   int* nsegs = scratch + PN;
   int* tbase = scratch + 2 * PN;
   int* sbase = scratch + 3 * PN;
-  geo_count_kernel<<<grid_for(PN, 128), 128, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, pieces,
-                                                      nsegs, status);
-  count_launch();
-  scan2_kernel<<<1, 1024, 0, st>>>(pieces, nsegs, PN, tbase, sbase, counts);
-  count_launch();
   const int tile_cap = geo_max_tiles(nN, PN), seg_cap = geo_max_segs(nM, PM, PN, R);
-  geo_fill_kernel<<<grid_for(PN, 64), 64, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, status,
-                                                    tbase, sbase, nsegs, tiles, segs, tile_cap,
-                                                    seg_cap);
-  count_launch();
-  clamp_counts_kernel<<<1, 1, 0, st>>>(counts, tile_cap, seg_cap);
-  count_launch();
-  tile_prefix_kernel<<<1, 1024, 0, st>>>(tiles, counts, prefix);
+  geo_schedule_kernel<<<1, kSchedThreads, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, tiles, segs,
+                                                   counts, prefix, pieces, nsegs, tbase, sbase,
+                                                   tile_cap, seg_cap, status);
   count_launch();
   return cudaGetLastError();
 }

@@ -505,12 +505,19 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
               const WaitCtl& ctl) {
   cudaError_t e;
   if (dtype == SSC_BF16) {
-    if ((e = launch_gather_rows_bf16(Q, ldq, 0, memN, nN, nN, d, static_cast<__nv_bfloat16*>(w.Qp),
-                                     w.ldq, ctl.status, st)) != cudaSuccess ||
-        (e = launch_gather_rows_bf16(K, ldk, 0, memM, nM, nM, d, static_cast<__nv_bfloat16*>(w.Kp),
-                                     w.ldk, ctl.status, st)) != cudaSuccess ||
-        (e = launch_gather_rows_bf16(V, ldv, 0, memM, nM, nM, k, static_cast<__nv_bfloat16*>(w.Vp),
-                                     w.ldv, ctl.status, st)) != cudaSuccess)
+    // Q, K and V into patch-major order in one launch
+    const __nv_bfloat16* in[3] = {static_cast<const __nv_bfloat16*>(Q),
+                                  static_cast<const __nv_bfloat16*>(K),
+                                  static_cast<const __nv_bfloat16*>(V)};
+    const int in_ld[3] = {ldq, ldk, ldv};
+    const int* map[3] = {memN, memM, memM};
+    const int rows[3] = {nN, nM, nM};
+    const int cols[3] = {d, d, k};
+    __nv_bfloat16* out[3] = {static_cast<__nv_bfloat16*>(w.Qp), static_cast<__nv_bfloat16*>(w.Kp),
+                             static_cast<__nv_bfloat16*>(w.Vp)};
+    const int out_ld[3] = {w.ldq, w.ldk, w.ldv};
+    if ((e = launch_gather3_bf16(in, in_ld, map, rows, rows, cols, out, out_ld, ctl.status, st)) !=
+        cudaSuccess)
       return SSC_ERR_CUDA;
   } else {
     if ((e = launch_gather_rows_f32(static_cast<const float*>(Q), ldq, memN, nN, nN, d,
@@ -586,11 +593,9 @@ int geo_bwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, i
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   // dK is reduced in the patch-major key order (contiguous key rows, so TMA
   // reductions apply) and scattered to vertex order afterwards: memM lists
-  // every source vertex once, so the scatter writes each row of dK once
-  // (dK itself is zeroed too, so that rows of vertices missing from inconsistent
-  // tables read as zero rather than as stale memory)
+  // every source vertex once, so the scatter writes each row of dK once (with
+  // inconsistent tables the results are unspecified, as the header states)
   if ((e = zero_matrix(w.dKg, d, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
   if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
