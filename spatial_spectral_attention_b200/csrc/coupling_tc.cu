@@ -154,9 +154,18 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   constexpr int NC = CW / 32;    // 32-column TMEM loads per thread
   constexpr int NSM = 128 * NWG; // softmax threads
   constexpr int kVWarp = 2 + 4 * NWG;  // warp of the V producer
+  // Fixed shape: V arrives as 16-column blocks in the 32-byte swizzle (4 KB
+  // each, the layout of the remainder box), so that P.V is one MMA of
+  // N = 64 VF + VR per K step instead of one per 64-column chunk plus one
+  // N = 16 MMA for the remainder.
+  constexpr bool kV32 = kFixed;
+  constexpr int kVBlocks = (64 * VF + VR) / 16;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full[2],
-      bar_v_empty[2], bar_s_full[2], bar_p_full[2], bar_o_full, bar_drain, bar_xmax, bar_xsum;
+  // A K stage is free when the S MMA that read it completes (bar_s_full of
+  // the same index); a V stage when its P.V completes (bar_o_full of the
+  // same index with two V stages, bar_v_empty with one).
+  __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_v_full[2], bar_v_empty,
+      bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_drain, bar_xmax, bar_xsum;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   // Partial row maxima / sums exchanged between the softmax warpgroups through
@@ -174,6 +183,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   const uint32_t sQ = sbase;
   const uint32_t sK0 = sQ + qbytes;
   const uint32_t sV0 = sK0 + 2 * qbytes;
+  // epilogue staging: 2 KB per softmax warp, after the V ring
+  const uint32_t sStage = sV0 + p.vstages * vbytes;
   const int ntiles = p.ntiles_dev ? *p.ntiles_dev : p.ntiles_host;
 
   if (threadIdx.x == 0) {
@@ -181,13 +192,12 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     mbar_init(&bar_q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_k_full[i], 1);
-      mbar_init(&bar_k_empty[i], 1);
       mbar_init(&bar_v_full[i], 1);
-      mbar_init(&bar_v_empty[i], 1);
       mbar_init(&bar_s_full[i], 1);
       mbar_init(&bar_p_full[i], NSM);
+      mbar_init(&bar_o_full[i], 1);
     }
-    mbar_init(&bar_o_full, 1);
+    mbar_init(&bar_v_empty, 1);
     mbar_init(&bar_drain, 1);
     mbar_init(&bar_xmax, NSM);
     mbar_init(&bar_xsum, NSM);
@@ -227,7 +237,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         for (int j = 0; j < tile.nseg; ++j, ++it) {
           const int key0 = p.segs[tile.seg0 + j].key0;
           const int st = it & 1;
-          if (it >= 2 && !mbar_wait(&bar_k_empty[st], ((it >> 1) - 1) & 1, p.ctl, abort)) {
+          if (it >= 2 && !mbar_wait(&bar_s_full[st], ((it >> 1) - 1) & 1, p.ctl, abort)) {
             ok = false;
             break;
           }
@@ -257,16 +267,22 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         for (int j = 0; j < tile.nseg; ++j, ++it) {
           const int key0 = p.segs[tile.seg0 + j].key0;
           const int st = it % VS;
-          if (it >= (uint32_t)VS &&
-              !mbar_wait(&bar_v_empty[st], ((it / VS) - 1) & 1, p.ctl, abort)) {
+          if (it >= (uint32_t)VS && !mbar_wait(VS == 2 ? &bar_o_full[st] : &bar_v_empty,
+                                               ((it / VS) - 1) & 1, p.ctl, abort)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bar_v_full[st], vbytes);
           uint8_t* dv = gptr(sV0) + st * vbytes;
-          for (int c = 0; c < vf; ++c)
-            tma_load_2d(dv + c * kChunk, &tm.v, 64 * c, key0, &bar_v_full[st]);
-          if (vr) tma_load_2d(dv + vf * kChunk, &tm.vr, 64 * vf, key0, &bar_v_full[st]);
+          if (kV32) {
+#pragma unroll
+            for (int c = 0; c < kVBlocks; ++c)
+              tma_load_2d(dv + c * 4096, &tm.vr, 16 * c, key0, &bar_v_full[st]);
+          } else {
+            for (int c = 0; c < vf; ++c)
+              tma_load_2d(dv + c * kChunk, &tm.v, 64 * c, key0, &bar_v_full[st]);
+            if (vr) tma_load_2d(dv + vf * kChunk, &tm.vr, 64 * vf, key0, &bar_v_full[st]);
+          }
         }
         if (!ok) break;
       }
@@ -282,6 +298,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
       const uint32_t idesc_s = kFP8 ? make_idesc_e4m3(128, 128) : make_idesc_bf16(128, 128, 0, 0);
       const uint32_t idesc_pv = make_idesc_bf16(128, 64 * (vf > 0 ? vf : 1), 0, 1);
       const uint32_t idesc_pvr = make_idesc_bf16(128, vr > 0 ? vr : 16, 0, 1);
+      const uint32_t idesc_pv32 = make_idesc_bf16(128, 16 * kVBlocks, 0, 1);
       const uint32_t o_col = tmem + 256;
       const uint32_t rsw = rem_swizzle(vr);
       const uint32_t rrow = (uint32_t)vr * 2;  // bytes per row of the remainder box
@@ -308,7 +325,6 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           }
         }
         mma_commit(&bar_s_full[g & 1]);
-        mma_commit(&bar_k_empty[st]);
         return true;
       };
       for (int r = 0, t = snake_tile(0); t < ntiles && ok; t = snake_tile(++r), ++tcount) {
@@ -334,19 +350,27 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
           tc_fence_after();
           const uint32_t sv = sV0 + vst * vbytes;
           const uint32_t a_tmem = tmem + buf * 128;
+          if (kV32) {
+            // B = V: 16-column blocks 4 KB apart, 8-key groups 256 B apart
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            if (vf > 0)
-              mma_ts(o_col, a_tmem + kk * 8, make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128),
-                     idesc_pv, acc);
-            if (vr > 0)
-              mma_ts(o_col + 64 * vf, a_tmem + kk * 8,
-                     make_sdesc(sv + vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
-                     idesc_pvr, acc);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(o_col, a_tmem + kk * 8, make_sdesc(sv + kk * 512, 4096, 256, kSw32), idesc_pv32,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+              if (vf > 0)
+                mma_ts(o_col, a_tmem + kk * 8, make_sdesc(sv + kk * 2048, kChunk, 1024, kSw128),
+                       idesc_pv, acc);
+              if (vr > 0)
+                mma_ts(o_col + 64 * vf, a_tmem + kk * 8,
+                       make_sdesc(sv + vf * kChunk + kk * 16 * rrow, 128 * rrow, 8 * rrow, rsw),
+                       idesc_pvr, acc);
+            }
           }
-          mma_commit(&bar_v_empty[vst]);
-          mma_commit(&bar_o_full);
+          if (VS == 1) mma_commit(&bar_v_empty);
+          mma_commit(&bar_o_full[g & 1]);
           if (j + 2 < nk) {
             ok = issue_s(g + 2);
             if (ok && j + 3 == nk) mma_commit(&bar_q_empty);
@@ -374,6 +398,9 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       int nkeys_next = nk > 0 ? p.segs[tile.seg0].nkeys : 0;
+      // output row of this thread (read now, used by the epilogue)
+      const int row = tile.row0 + lrow;
+      int orow = (lrow < tile.nrows && row < p.nq) ? (p.row_map ? p.row_map[row] : row) : -1;
       for (int j = 0; j < nk; ++j) {
         const uint32_t g = it + j;
         const int buf = g & 1;
@@ -416,16 +443,15 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         }
         const float m_new = fmaxf(m, mx * scale_log2);
         const bool need = m_new > m + 8.0f;
-        // PV_{g-1} (the previous tile's contribution to O) must be waited for
-        // exactly once per tile: the parity wait is only sound when this thread
-        // is never more than one phase behind the barrier.
-        bool o_pending = j > 0;
+        // PV_g completes on bar_o_full[g & 1] (its phase g >> 1 there).  O is
+        // rescaled only after PV_{g-1} has completed; otherwise P_g is handed
+        // over while PV_{g-1} may still run, so the tensor pipe always has the
+        // next P.V queued.
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          if (!mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+          if (!mbar_wait(&bar_o_full[(g - 1) & 1], ((g - 1) >> 1) & 1, p.ctl, abort)) {
             ok = false;
             break;
           }
-          o_pending = false;
           tc_fence_after();
           const float f = need ? ex2_approx(m - m_new) : 1.0f;
           const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
@@ -467,7 +493,10 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
 #pragma unroll
         for (int c = 0; c < NC; ++c) tmem_st16(pa + 16 * c, pk[c]);
         tmem_st_wait();
-        if (o_pending && !mbar_wait(&bar_o_full, (g - 1) & 1, p.ctl, abort)) {
+        // Keep this thread within one phase of bar_o_full[g & 1]: PV_{g-2} is
+        // complete already (S_g, waited for above, was issued after it), so
+        // this wait only advances the phase this thread has observed there.
+        if (g >= 2 && !mbar_wait(&bar_o_full[g & 1], ((g - 2) >> 1) & 1, p.ctl, abort)) {
           ok = false;
           break;
         }
@@ -477,7 +506,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
       if (!ok) break;
       // epilogue: wait for the last PV, combine the partial row sums, O / l, lse
       const uint32_t glast = it + nk - 1;
-      if (!mbar_wait(&bar_o_full, glast & 1, p.ctl, abort)) break;
+      if (!mbar_wait(&bar_o_full[glast & 1], (glast >> 1) & 1, p.ctl, abort)) break;
       tc_fence_after();
       if (NWG > 1) {
         s_psum[wg][lrow] = l;
@@ -487,32 +516,57 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
 #pragma unroll
         for (int w = 0; w < NWG; ++w) l += s_psum[w][lrow];
       }
-      const int row = tile.row0 + lrow;
-      int orow = (lrow < tile.nrows && row < p.nq) ? (p.row_map ? p.row_map[row] : row) : -1;
       if (orow >= p.nq) orow = -1;
       const bool live = orow >= 0;
       if (!live) orow = 0;
-      float* optr = p.O + (size_t)orow * p.ldo;
       const float inv = 1.0f / l;
       const uint32_t oa = tmem_lane_addr(tmem, warp, 256);
+      // O / l goes out through a per-warp staging buffer: 32 rows x 16 columns,
+      // 64-byte rows whose 16-byte units are XOR-swizzled by (row >> 1) & 3 (no
+      // bank conflicts either way).  Each store instruction then writes 64
+      // contiguous bytes of 8 rows instead of 16 bytes of 32 rows.
+      float* stg = reinterpret_cast<float*>(gptr(sStage + (warp - 2) * 2048));
+      const bool vec_ok = (p.ldo & 3) == 0;
+      // the output rows of the 4 rows this lane stores per chunk
+      int orow_r[4];
+      bool live_r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        orow_r[i] = __shfl_sync(0xffffffffu, orow, 8 * i + (lane >> 2));
+        live_r[i] = __shfl_sync(0xffffffffu, live ? 1 : 0, 8 * i + (lane >> 2)) != 0;
+      }
+      // TMEM loads one chunk ahead of the stores
+      uint32_t o[16], o_next[16];
+      if (wg < nchunk) tmem_ld16(oa + 16 * wg, o_next);
       for (int c = wg; c < nchunk; c += NWG) {
-        uint32_t o[16];
-        tmem_ld16(oa + 16 * c, o);
-        tmem_ld_wait();
-        if (live) {
-          const int c0 = 16 * c;
-          if (c0 + 16 <= p.k && (p.ldo & 3) == 0) {
+        tmem_ld_wait(o_next);
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(optr + c0 + i) =
-                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-          } else {
+        for (int i = 0; i < 16; ++i) o[i] = o_next[i];
+        if (c + NWG < nchunk) tmem_ld16(oa + 16 * (c + NWG), o_next);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (c0 + i < p.k) optr[c0 + i] = __uint_as_float(o[i]) * inv;
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<float4*>(stg + lane * 16 + (((u ^ (lane >> 1)) & 3) << 2)) =
+              make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                          __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 8 * i + (lane >> 2), u = lane & 3;
+          const float4 v = *reinterpret_cast<const float4*>(stg + r * 16 + (((u ^ (r >> 1)) & 3) << 2));
+          const int col = 16 * c + 4 * u;
+          if (live_r[i]) {
+            float* dst = p.O + (size_t)orow_r[i] * p.ldo + col;
+            if (vec_ok && col + 4 <= p.k) {
+              *reinterpret_cast<float4*>(dst) = v;
+            } else {
+              if (col < p.k) dst[0] = v.x;
+              if (col + 1 < p.k) dst[1] = v.y;
+              if (col + 2 < p.k) dst[2] = v.z;
+              if (col + 3 < p.k) dst[3] = v.w;
+            }
           }
         }
+        __syncwarp();
       }
       if (live && wg == 0) p.lse[orow] = (m + log2f(l)) * kLn2;
       it += nk;
@@ -1316,14 +1370,25 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
       // this row tile's dO row into TMEM (the previous row tile's MMAs are
       // complete: its dQ was waited for below before getting here)
       {
+        // all of this thread's pieces are loaded before the first TMEM store, so
+        // their latencies overlap (kp <= 256: at most 8 pieces of 16 columns)
         const uint4* src = reinterpret_cast<const uint4*>(p.dOb + (size_t)(live_row ? qrow : 0) * p.lddob);
         const uint32_t da = tmem_lane_addr(tmem, warp, c_do);
-        for (int pc = wg; pc < kp16; pc += NCG) {
-          uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-          if (live_row) {
-            a = src[2 * pc];
-            b = src[2 * pc + 1];
+        uint4 piece[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int pc = wg + NCG * i;
+          piece[2 * i] = piece[2 * i + 1] = make_uint4(0u, 0u, 0u, 0u);
+          if (live_row && pc < kp16) {
+            piece[2 * i] = __ldg(src + 2 * pc);
+            piece[2 * i + 1] = __ldg(src + 2 * pc + 1);
           }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int pc = wg + NCG * i;
+          if (pc >= kp16) break;
+          const uint4 a = piece[2 * i], b = piece[2 * i + 1];
           const uint32_t r[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
           tmem_st8(da + 8 * pc, r);
         }
@@ -1405,41 +1470,58 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
       if (!ok) break;
       if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
       tc_fence_after();
-      // TMEM loads are warp-collective: every lane loads, live rows store
-      int orow = live_row ? (p.row_map ? p.row_map[qrow] : qrow) : -1;
-      const bool store_row = orow >= 0 && orow < p.nq;
+      // dQ / s goes out through a 2 KB staging area inside this warp's own rows
+      // of the dS tile (free: every MMA that read it is complete): 32 rows x
+      // 16 columns per chunk, 16-byte units XOR-swizzled by (row >> 1) & 3, so
+      // that each store or reduction covers 64 contiguous bytes of 8 rows.
       const bool whole = jb == 0 && je == tile.nseg;  // all of the row tile's keys done here
-      if (!store_row) orow = 0;
-      float* dq = p.dQ + (size_t)orow * p.lddq;
+      float* stg = reinterpret_cast<float*>(gptr(sS + wg * kChunk + (warp & 3) * 4096));
+      // output rows of the 4 rows this lane stores per chunk (row 8 i + lane / 4
+      // of the warp's 32)
+      int orow_r[4];
+      bool live_r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int lr = 32 * (warp & 3) + 8 * i + (lane >> 2);
+        const int qr = tile.row0 + lr;
+        int o_r = (lr < tile.nrows && qr < p.nq) ? (p.row_map ? p.row_map[qr] : qr) : -1;
+        live_r[i] = o_r >= 0 && o_r < p.nq;
+        orow_r[i] = live_r[i] ? o_r : 0;
+      }
+      const bool vec_ok = (p.lddq & 3) == 0 && (whole || p.vec_atomics_dq);
       const uint32_t qa = tmem_lane_addr(tmem, warp, c_dq);
       for (int cc = wg; cc < d16; cc += NCG) {
         uint32_t o[16];
-        tmem_ld16(qa + 16 * cc, o);
+        tmem_ld16(qa + 16 * cc, o);  // warp-collective: every lane loads
         tmem_ld_wait();
-        if (!store_row) continue;
-        if (!whole) {
-          // the row tile's keys are split over several CTAs: reduce into dQ
-          if (p.vec_atomics_dq) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              atomicAdd(reinterpret_cast<float4*>(dq + 16 * cc + i),
-                        make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
-                                    __uint_as_float(o[i + 2]) * p.scale,
-                                    __uint_as_float(o[i + 3]) * p.scale));
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<float4*>(stg + lane * 16 + (((u ^ (lane >> 1)) & 3) << 2)) = make_float4(
+              __uint_as_float(o[4 * u]) * p.scale, __uint_as_float(o[4 * u + 1]) * p.scale,
+              __uint_as_float(o[4 * u + 2]) * p.scale, __uint_as_float(o[4 * u + 3]) * p.scale);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 8 * i + (lane >> 2), u = lane & 3;
+          const float4 v = *reinterpret_cast<const float4*>(stg + r * 16 + (((u ^ (r >> 1)) & 3) << 2));
+          if (!live_r[i]) continue;
+          float* dst = p.dQ + (size_t)orow_r[i] * p.lddq + 16 * cc + 4 * u;
+          if (vec_ok) {
+            if (whole) *reinterpret_cast<float4*>(dst) = v;
+            else atomicAdd(reinterpret_cast<float4*>(dst), v);  // the row tile's keys are split over CTAs
+          } else if (whole) {
+            dst[0] = v.x;
+            dst[1] = v.y;
+            dst[2] = v.z;
+            dst[3] = v.w;
           } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) atomicAdd(dq + 16 * cc + i, __uint_as_float(o[i]) * p.scale);
+            atomicAdd(dst, v.x);
+            atomicAdd(dst + 1, v.y);
+            atomicAdd(dst + 2, v.z);
+            atomicAdd(dst + 3, v.w);
           }
-        } else if ((p.lddq & 3) == 0) {
-#pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dq + 16 * cc + i) = make_float4(
-                __uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
-                __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) dq[16 * cc + i] = __uint_as_float(o[i]) * p.scale;
         }
+        __syncwarp();
       }
     }
   } else {
@@ -2479,11 +2561,12 @@ cudaError_t launch_fwd_single(const TcArgs& a, float* O, int ldo, float* lse, cu
   if (e != cudaSuccess) return e;
   // two V stages when they fit next to Q and the two K stages, else one
   const int qtile = fp8 ? 128 * 128 : p.qch * kChunk;
+  const int stage_bytes = 4 * NWG * 2048;  // epilogue staging, 2 KB per softmax warp
   p.vstages = 2;
-  int smem = 1024 + qtile * 3 + p.vstages * vtile_bytes(p.vf, p.vr);
+  int smem = 1024 + qtile * 3 + p.vstages * vtile_bytes(p.vf, p.vr) + stage_bytes;
   if (smem + (int)fa.sharedSizeBytes > smem_optin()) {
     p.vstages = 1;
-    smem = 1024 + qtile * 3 + vtile_bytes(p.vf, p.vr);
+    smem = 1024 + qtile * 3 + vtile_bytes(p.vf, p.vr) + stage_bytes;
   }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

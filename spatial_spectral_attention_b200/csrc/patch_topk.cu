@@ -197,13 +197,151 @@ __global__ void __launch_bounds__(128) pool_rows_kernel(const PoolSet set_a, con
   if (c1 < d) mu[(size_t)p * d + c1] = __ddiv_rn(s1, cnt);
 }
 
+// Warp-per-patch pooling for d = 32 CPL (CPL = 2 or 4 channels per lane):
+// each lane sums its CPL channels as CPL independent chains, strictly in
+// member order (bit-identical to pool_kernel).  The warp stages the member
+// rows of its patch in shared memory with cp.async, kWarpRows rows per chunk
+// and two chunks in flight; member indices go through shared memory too.
+// Four warps (four patches) per block, both shapes in one launch.
+constexpr int kWarpRows = 32;
+template <bool F32, int CPL>
+__global__ void __launch_bounds__(128) pool_warp_kernel(const PoolSet set_a, const PoolSet set_b,
+                                                        unsigned* status) {
+  constexpr int kEsz = F32 ? 4 : 2;
+  constexpr int kRowB = 32 * CPL * kEsz;    // bytes per descriptor row (d = 32 CPL)
+  constexpr int kPieces = kRowB / 16;       // 16-byte pieces per row
+  constexpr int kChunkB = kWarpRows * kRowB;
+  extern __shared__ __align__(16) uint8_t s_pool[];  // [4 warps][2][kWarpRows][kRowB]
+  __shared__ int s_idx[4][2][kWarpRows];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gp = blockIdx.x * 4 + warp;
+  if (gp >= set_a.P + set_b.P) return;  // warp-uniform; no block barrier below
+  const bool second = gp >= set_a.P;
+  const PoolSet& S = second ? set_b : set_a;
+  const int p = second ? gp - set_a.P : gp;
+  const int n = S.n;
+  const int* __restrict__ mem = S.mem;
+  const uint8_t* Fb = static_cast<const uint8_t*>(S.F);
+  const size_t ldb = (size_t)S.ld * kEsz;
+  int b = S.off[p], e = S.off[p + 1];
+  if (b < 0 || e <= b || e > n) {
+    if (lane == 0) atomicOr(status, kStatusBadIndex);
+    b = min(max(b, 0), n);
+    e = min(max(e, b), n);
+  }
+  const int rows = e - b;
+  const int nch = (rows + kWarpRows - 1) / kWarpRows;
+  uint8_t* wbuf = s_pool + warp * 2 * kChunkB;
+  const uint32_t wbase = smem_u32(wbuf);
+  // the member indices of the first 8 chunks, all loaded up front
+  constexpr int kPre = 8;
+  int pre[kPre];
+#pragma unroll
+  for (int j = 0; j < kPre; ++j) {
+    const int r = b + j * kWarpRows + lane;
+    pre[j] = r < e ? mem[r] : -1;
+  }
+  auto issue = [&](int k) {
+    const int r0 = b + k * kWarpRows;
+    int v = -1;
+    if (r0 + lane < e) {
+      if (k < kPre) {
+#pragma unroll
+        for (int j = 0; j < kPre; ++j)
+          if (j == k) v = pre[j];
+      } else {
+        v = mem[r0 + lane];
+      }
+      if (v < 0 || v >= n) {
+        atomicOr(status, kStatusBadIndex);
+        v = -1;
+      }
+    }
+    s_idx[warp][k & 1][lane] = v;
+    __syncwarp();
+    const uint32_t buf = wbase + (k & 1) * kChunkB;
+#pragma unroll
+    for (int j = 0; j < kWarpRows * kPieces / 32; ++j) {
+      const int i = lane + 32 * j;
+      const int r = i / kPieces, pc = i % kPieces;
+      const int vr = s_idx[warp][k & 1][r];
+      if (vr >= 0) cp_async16(buf + r * kRowB + pc * 16, Fb + (size_t)vr * ldb + pc * 16);
+    }
+    cp_async_commit();
+  };
+  double acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
+  if (nch > 0) issue(0);
+  for (int k = 0; k < nch; ++k) {
+    if (k + 1 < nch) {
+      issue(k + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();  // every lane's copies of chunk k are visible
+    const uint8_t* buf = wbuf + (k & 1) * kChunkB + lane * CPL * kEsz;
+    const int nr = min(kWarpRows, rows - k * kWarpRows);
+    for (int r0 = 0; r0 < nr; r0 += 8) {
+      double x[8][CPL];
+      bool ok[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u;
+        ok[u] = r < nr && s_idx[warp][k & 1][r] >= 0;  // the same for every lane
+        if constexpr (F32) {
+          float v[CPL];
+          if (ok[u]) {
+            if constexpr (CPL == 4) {
+              const float4 t = *reinterpret_cast<const float4*>(buf + r * kRowB);
+              v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+            } else {
+              const float2 t = *reinterpret_cast<const float2*>(buf + r * kRowB);
+              v[0] = t.x; v[1] = t.y;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) x[u][c] = ok[u] ? (double)v[c] : 0.0;
+        } else {
+          uint32_t w[CPL / 2];
+          if (ok[u]) {
+            if constexpr (CPL == 4) {
+              const uint2 t = *reinterpret_cast<const uint2*>(buf + r * kRowB);
+              w[0] = t.x; w[1] = t.y;
+            } else {
+              w[0] = *reinterpret_cast<const uint32_t*>(buf + r * kRowB);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            // bf16 -> fp32 is exact: the bf16 bits are the high half of the float
+            const uint32_t h = ok[u] ? ((c & 1) ? (w[c >> 1] & 0xffff0000u) : (w[c >> 1] << 16)) : 0u;
+            x[u][c] = (double)__uint_as_float(h);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (ok[u]) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[c] = __dadd_rn(acc[c], x[u][c]);
+        }
+    }
+    __syncwarp();  // chunk k's buffer is refilled by issue(k + 2)
+  }
+  const double cnt = (double)max(e - b, 1);
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) S.mu[(size_t)p * 32 * CPL + lane * CPL + c] = __ddiv_rn(acc[c], cnt);
+}
+
 constexpr int kST = 32;  // score tile (target x source patches)
 constexpr int kSC = 128;  // channels staged per step (one load phase for d <= 128)
 
 // scores[p, q] for a 32 x 32 tile per block; each thread owns 4 outputs and
 // sums its products strictly in channel order.  blockIdx.z selects the pair of
 // a batch (its means and score block follow the previous pair's).
-__global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ muN, int PN,
+__global__ void __launch_bounds__(256, 2) scores_kernel(const double* __restrict__ muN, int PN,
                                                      const double* __restrict__ muM, int PM, int d,
                                                      double* __restrict__ sc) {
   muN += (size_t)blockIdx.z * PN * d;
@@ -216,10 +354,20 @@ __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ 
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of threads
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int c0 = 0; c0 < d; c0 += kSC) {
-    for (int i = threadIdx.x; i < kST * kSC; i += 256) {
-      int r = i / kSC, cc = i % kSC;
-      a[r][cc] = (p0 + r < PN && c0 + cc < d) ? muN[(size_t)(p0 + r) * d + c0 + cc] : 0.0;
-      b[r][cc] = (q0 + r < PM && c0 + cc < d) ? muM[(size_t)(q0 + r) * d + c0 + cc] : 0.0;
+    // all of this thread's loads in flight before the first store
+    double va[kST * kSC / 256], vb[kST * kSC / 256];
+#pragma unroll
+    for (int j = 0; j < kST * kSC / 256; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      const int r = i / kSC, cc = i % kSC;
+      va[j] = (p0 + r < PN && c0 + cc < d) ? muN[(size_t)(p0 + r) * d + c0 + cc] : 0.0;
+      vb[j] = (q0 + r < PM && c0 + cc < d) ? muM[(size_t)(q0 + r) * d + c0 + cc] : 0.0;
+    }
+#pragma unroll
+    for (int j = 0; j < kST * kSC / 256; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      a[i / kSC][i % kSC] = va[j];
+      b[i / kSC][i % kSC] = vb[j];
     }
     __syncthreads();
     const int cmax = min(kSC, d - c0);
@@ -251,19 +399,39 @@ __device__ __forceinline__ bool pick_before(const Pick& a, const Pick& b) {
 // it by xor-shuffles (every lane ends with the winner), so no block barrier is
 // needed.  Because each round only admits candidates ranked after the previous
 // winner, no candidate needs marking.
-__global__ void __launch_bounds__(256) topk_warp_kernel(const double* __restrict__ sc, int PN, int PM,
-                                                        int R, int* __restrict__ topk) {
+// The lane's share of the row (q = lane + 32 i) is read once into registers
+// when it fits (PM <= 32 kTopkRegs); otherwise every round re-reads the row.
+constexpr int kTopkRegs = 40;
+__global__ void __launch_bounds__(64) topk_warp_kernel(const double* __restrict__ sc, int PN, int PM,
+                                                       int R, int* __restrict__ topk) {
   const int lane = threadIdx.x & 31;
-  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int p = blockIdx.x * 2 + (threadIdx.x >> 5);
   if (p >= PN) return;  // warp-uniform
   const double* row = sc + (size_t)p * PM;
+  const bool in_regs = PM <= 32 * kTopkRegs;
+  double v[kTopkRegs];
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kTopkRegs; ++i) v[i] = lane + 32 * i < PM ? row[lane + 32 * i] : 0.0;
+  }
   Pick prev{DBL_MAX, -1};
   for (int r = 0; r < R; ++r) {
     Pick mine{-DBL_MAX, INT_MAX};  // no candidate yet
-    for (int q = lane; q < PM; q += 32) {
-      const Pick c{row[q], q};
-      if (r > 0 && !pick_before(prev, c)) continue;
-      if (mine.q == INT_MAX || pick_before(c, mine)) mine = c;
+    if (in_regs) {
+#pragma unroll
+      for (int i = 0; i < kTopkRegs; ++i) {
+        const int q = lane + 32 * i;
+        if (q >= PM) break;
+        const Pick c{v[i], q};
+        if (r > 0 && !pick_before(prev, c)) continue;
+        if (mine.q == INT_MAX || pick_before(c, mine)) mine = c;
+      }
+    } else {
+      for (int q = lane; q < PM; q += 32) {
+        const Pick c{row[q], q};
+        if (r > 0 && !pick_before(prev, c)) continue;
+        if (mine.q == INT_MAX || pick_before(c, mine)) mine = c;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -314,7 +482,23 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
     return cudaGetLastError();
   };
   cudaError_t pe;
-  if (staged(FN, ldn) && staged(FM, ldm)) {
+  if ((d == 64 || d == 128) && staged(FN, ldn) && staged(FM, ldm)) {
+    // one warp per patch, both shapes in one launch
+    const PoolSet a{FN, offN, memN, muN, ldn, batch * nN, batch * PN};
+    const PoolSet b{FM, offM, memM, muM, ldm, batch * nM, batch * PM};
+    const int smem = 4 * 2 * kWarpRows * d * esz;
+    auto kern = dtype == 1 ? (d == 128 ? pool_warp_kernel<true, 4> : pool_warp_kernel<true, 2>)
+                           : (d == 128 ? pool_warp_kernel<false, 4> : pool_warp_kernel<false, 2>);
+    if ((pe = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return pe;
+    const int total = batch * (PN + PM);
+    prof_launch_begin(st);
+    kern<<<(total + 3) / 4, 128, smem, st>>>(a, b, status);
+    prof_launch_end(st, SSC_PROF_POOL);
+    count_launch();
+    if ((pe = cudaGetLastError()) != cudaSuccess) return pe;
+  } else if (staged(FN, ldn) && staged(FM, ldm)) {
     // both shapes in one launch, member rows staged through shared memory
     auto kern = dtype == 1 ? pool_rows_kernel<true> : pool_rows_kernel<false>;
     if ((pe = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem)) !=
@@ -341,7 +525,7 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
   prof_launch_end(st, SSC_PROF_SCORES);
   count_launch();
   prof_launch_begin(st);
-  topk_warp_kernel<<<(batch * PN + 7) / 8, 256, 0, st>>>(sc, batch * PN, PM, R, topk);
+  topk_warp_kernel<<<(batch * PN + 1) / 2, 64, 0, st>>>(sc, batch * PN, PM, R, topk);
   prof_launch_end(st, SSC_PROF_TOPK);
   count_launch();
   return cudaGetLastError();

@@ -225,6 +225,79 @@ __global__ void bwd_prep_kernel(const float* __restrict__ dO, int lddo, const fl
                                 float* __restrict__ lse_out, int vec4, unsigned* status) {
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (vec4 && k <= 256) {
+    // 2 rows per warp and step; each lane's (at most 2) float4 of dO and O of
+    // both rows are loaded before any is used.  Per row the arithmetic is
+    // that of the loop below, in the same order.
+    const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int c4n = k >> 2;
+    for (int r0 = 2 * w; r0 < rows; r0 += 2 * warps) {
+      int src0[2];
+      float4 gv[2][2], ov[2][2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) src0[u] = r0 + u < rows ? checked_src(map, r0 + u, src_rows, status) : -1;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int src = src0[u] < 0 ? 0 : src0[u];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int c4 = lane + 32 * i;
+          gv[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          ov[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r0 + u < rows && c4 < c4n) {
+            if (src0[u] >= 0) gv[u][i] = __ldg(reinterpret_cast<const float4*>(dO + (size_t)src * lddo) + c4);
+            ov[u][i] = __ldg(reinterpret_cast<const float4*>(O + (size_t)src * ldo) + c4);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = r0 + u;
+        if (r >= rows) break;
+        const int src = src0[u] < 0 ? 0 : src0[u];
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int c4 = lane + 32 * i;
+          if (c4 >= c4n) break;
+          float4 v = gv[u][i];
+          if (dOb) {
+            const __nv_bfloat162 b01 = __floats2bfloat162_rn(v.x, v.y);
+            const __nv_bfloat162 b23 = __floats2bfloat162_rn(v.z, v.w);
+            reinterpret_cast<uint2*>(dOb + (size_t)r * ldb)[c4] = make_uint2(
+                *reinterpret_cast<const uint32_t*>(&b01), *reinterpret_cast<const uint32_t*>(&b23));
+            v = make_float4(__low2float(b01), __high2float(b01), __low2float(b23), __high2float(b23));
+          }
+          if (dOf) reinterpret_cast<float4*>(dOf + (size_t)r * ldf)[c4] = v;
+          acc = fmaf(v.x, ov[u][i].x, acc);
+          acc = fmaf(v.y, ov[u][i].y, acc);
+          acc = fmaf(v.z, ov[u][i].z, acc);
+          acc = fmaf(v.w, ov[u][i].w, acc);
+        }
+        const float* g = dO + (size_t)src * lddo;
+        const float* o = O + (size_t)src * ldo;
+        for (int c = (k & ~3) + lane; c < k; c += 32) {
+          float v = src0[u] < 0 ? 0.f : g[c];
+          if (dOb) {
+            __nv_bfloat16 b = __float2bfloat16(v);
+            dOb[(size_t)r * ldb + c] = b;
+            v = __bfloat162float(b);
+          }
+          if (dOf) dOf[(size_t)r * ldf + c] = v;
+          acc = fmaf(v, o[c], acc);
+        }
+        if (dOb)
+          for (int c = k + lane; c < ldb; c += 32) dOb[(size_t)r * ldb + c] = __float2bfloat16(0.f);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+          D[r] = acc;
+          if (lse_out) lse_out[r] = src0[u] < 0 ? 0.f : lse[src];
+        }
+      }
+    }
+    return;
+  }
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const int src0 = checked_src(map, r, src_rows, status);
     const int src = src0 < 0 ? 0 : src0;
@@ -508,6 +581,41 @@ __device__ int sorted_tile_scan(const int* pieces, const int* nsegs, int m, int 
   return total;
 }
 
+// Key ranges [k0, k0 + kn) of the source patches topk[p R + r0 + u], u < 8,
+// with every load of the eight issued before any is used (kn = -1: past R or
+// a bad patch index, which sets the bad-index bit).
+__device__ __forceinline__ void source_ranges8(const int* __restrict__ topk, int p, int R, int r0,
+                                               const int* __restrict__ offM, int PM, int nM,
+                                               unsigned* status, int (&k0)[8], int (&kn)[8]) {
+  int q[8], b[8], e[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) q[u] = r0 + u < R ? topk[(size_t)p * R + r0 + u] : -1;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const bool ok = r0 + u < R && q[u] >= 0 && q[u] < PM;
+    b[u] = ok ? offM[q[u]] : 0;
+    e[u] = ok ? offM[q[u] + 1] : 0;
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    k0[u] = 0;
+    kn[u] = -1;
+    if (r0 + u >= R) continue;
+    if (q[u] < 0 || q[u] >= PM) {
+      atomicOr(status, kStatusBadIndex);
+      continue;
+    }
+    int bb = b[u], ee = e[u];
+    if (bb < 0 || ee < bb || ee > nM) {
+      atomicOr(status, kStatusBadIndex);
+      bb = min(max(bb, 0), nM);
+      ee = min(max(ee, bb), nM);
+    }
+    k0[u] = bb;
+    kn[u] = ee - bb;
+  }
+}
+
 // The whole Geo schedule in one block: per target patch its row tiles and
 // source segments (counts), their exclusive scans, the tile and segment
 // lists (row tiles by decreasing segment count), the clamped totals and the
@@ -530,14 +638,12 @@ __global__ void __launch_bounds__(kSchedThreads) geo_schedule_kernel(
     const int2 pr = patch_range(offN, p, nN, status);
     pieces[p] = (pr.y - pr.x + kTileRows - 1) / kTileRows;
     int sacc = 0;
-    for (int r = 0; r < R; ++r) {
-      const int q = topk[(size_t)p * R + r];
-      if (q < 0 || q >= PM) {
-        atomicOr(status, kStatusBadIndex);
-        continue;
-      }
-      const int2 qr = patch_range(offM, q, nM, status);
-      sacc += (qr.y - qr.x + kTileRows - 1) / kTileRows;
+    for (int r0 = 0; r0 < R; r0 += 8) {
+      int k0[8], kn[8];
+      source_ranges8(topk, p, R, r0, offM, PM, nM, status, k0, kn);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (kn[u] > 0) sacc += (kn[u] + kTileRows - 1) / kTileRows;
     }
     nsegs[p] = sacc;
     atomicMax(&s_maxseg, sacc);
@@ -563,13 +669,13 @@ __global__ void __launch_bounds__(kSchedThreads) geo_schedule_kernel(
       tiles[tbase[p] + i] = RowTile{r0 + t, min(kTileRows, rows - t), sb, ns};
     }
     int sidx = sb;
-    for (int r = 0; r < R; ++r) {
-      const int q = topk[(size_t)p * R + r];
-      if (q < 0 || q >= PM) continue;
-      const int2 qr = patch_range(offM, q, nM, status);
-      const int k0 = qr.x, kn = qr.y - qr.x;
-      for (int u = 0; u < kn && sidx < sb + ns; u += kTileRows)
-        segs[sidx++] = KeySeg{k0 + u, min(kTileRows, kn - u)};
+    for (int r0 = 0; r0 < R; r0 += 8) {
+      int k0[8], kn[8];
+      source_ranges8(topk, p, R, r0, offM, PM, nM, status, k0, kn);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        for (int v = 0; v < kn[u] && sidx < sb + ns; v += kTileRows)
+          segs[sidx++] = KeySeg{k0[u] + v, min(kTileRows, kn[u] - v)};
     }
   }
   const int m = min(ntile, tile_cap);
@@ -685,6 +791,30 @@ __global__ void scatter_rows_f32_kernel(const float* __restrict__ in, int in_ld,
                                         unsigned* status) {
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (vec_ok && cols <= 128) {
+    // 4 rows per warp and step, one float4 per lane and row: the map entries,
+    // then all four rows' loads, then the stores
+    const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int c4n = cols >> 2;
+    for (int r0 = 4 * w; r0 < rows; r0 += 4 * warps) {
+      int dst[4];
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dst[u] = r0 + u < rows ? checked_src(map, r0 + u, dst_rows, status) : -1;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (dst[u] >= 0 && lane < c4n)
+          v[u] = __ldg(reinterpret_cast<const float4*>(in + (size_t)(r0 + u) * in_ld) + lane);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (dst[u] < 0) continue;
+        float* o = out + (size_t)dst[u] * out_ld;
+        if (lane < c4n) reinterpret_cast<float4*>(o)[lane] = v[u];
+        for (int c = 4 * c4n + lane; c < cols; c += 32) o[c] = in[(size_t)(r0 + u) * in_ld + c];
+      }
+    }
+    return;
+  }
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const int dst = checked_src(map, r, dst_rows, status);
     if (dst < 0) continue;
@@ -706,8 +836,9 @@ cudaError_t launch_scatter_rows_f32(const float* in, int in_ld, const int* map, 
   if (rows <= 0) return cudaSuccess;
   const int vec_ok = in_ld % 4 == 0 && out_ld % 4 == 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 &&
                      reinterpret_cast<uintptr_t>(out) % 16 == 0;
-  scatter_rows_f32_kernel<<<grid_for(rows, 8), 256, 0, st>>>(in, in_ld, map, rows, dst_rows, cols,
-                                                             out, out_ld, vec_ok, status);
+  const int g = grid_for(rows, vec_ok && cols <= 128 ? 32 : 8);
+  scatter_rows_f32_kernel<<<g, 256, 0, st>>>(in, in_ld, map, rows, dst_rows, cols, out, out_ld,
+                                             vec_ok, status);
   count_launch();
   return cudaGetLastError();
 }
@@ -774,8 +905,8 @@ cudaError_t launch_bwd_prep(const float* dO, int lddo, const float* O, int ldo, 
   const int vec4 = lddo % 4 == 0 && ldo % 4 == 0 && a16(dO) && a16(O) &&
                    (!dOb || (ldb % 4 == 0 && reinterpret_cast<uintptr_t>(dOb) % 8 == 0)) &&
                    (!dOf || (ldf % 4 == 0 && a16(dOf)));
-  bwd_prep_kernel<<<grid_for(rows, 8), 256, 0, st>>>(dO, lddo, O, ldo, lse, map, rows, src_rows, k,
-                                                      dOb, ldb, dOf, ldf, D, lse_out, vec4, status);
+  bwd_prep_kernel<<<grid_for(rows, vec4 && k <= 256 ? 16 : 8), 256, 0, st>>>(
+      dO, lddo, O, ldo, lse, map, rows, src_rows, k, dOb, ldb, dOf, ldf, D, lse_out, vec4, status);
   count_launch();
   return cudaGetLastError();
 }
