@@ -620,7 +620,7 @@ __device__ __forceinline__ void source_ranges8(const int* __restrict__ topk, int
 // source segments (counts), their exclusive scans, the tile and segment
 // lists (row tiles by decreasing segment count), the clamped totals and the
 // tiles' segment prefix sums, in one launch.
-__global__ void __launch_bounds__(kSchedThreads) geo_schedule_kernel(
+__global__ void __launch_bounds__(kSchedThreads, 1) geo_schedule_kernel(
     const int* __restrict__ offN, int PN, int nN, const int* __restrict__ offM, int PM, int nM,
     const int* __restrict__ topk, int R, RowTile* __restrict__ tiles, KeySeg* __restrict__ segs,
     int* __restrict__ counts, int* __restrict__ prefix, int* __restrict__ pieces,
