@@ -89,6 +89,19 @@ int ssc_set_wait_limit_ns(unsigned long long ns);
  * No GPU fault, trap or hang is involved. */
 int ssc_debug_wait_timeout(unsigned long long limit_ns, ssc_stream_t stream);
 
+/* Test hook of the abort path of the tensor-core coupling kernels.  which = 1:
+ * the next launch of the forward kernel (Geo forward, and the dense forward
+ * on fp8 tensor cores); which = 2: the next launch of the dQ/dK backward
+ * kernel (dense and Geo).  In that launch the MMA issuer, after its first S
+ * MMAs, waits on a barrier nothing arrives at.  The bounded wait gives up
+ * after the wait limit (ssc_set_wait_limit_ns), records SSC_ERR_TIMEOUT in the
+ * device status word and raises the kernel's abort flag: every role leaves its
+ * loop, the producers wait for their copies in flight, the issued MMAs drain
+ * and TMEM is freed before the CTAs exit, so the context stays usable.  The
+ * outputs of that launch are undefined.  No GPU fault, trap or hang is
+ * involved.  which = 0 disarms; other values return SSC_ERR_INVALID_ARG. */
+int ssc_debug_stall_next_launch(int which);
+
 /* ------------------------------------------------------------------------ */
 /* Geodesic patches.                                                        */
 /* Source: digest "Interpretation" (geodesic farthest-point sampling) and    */

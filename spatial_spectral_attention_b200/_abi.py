@@ -24,6 +24,7 @@ SIGNATURES = {
     "ssc_device_status": (I, [P, I, ctypes.POINTER(I)]),
     "ssc_set_wait_limit_ns": (I, [U64]),
     "ssc_debug_wait_timeout": (I, [U64, P]),
+    "ssc_debug_stall_next_launch": (I, [I]),
     "ssc_debug_fps_cluster_size": (I, [I]),
     "ssc_fps_patches_workspace_size": (Z, [I, I]),
     "ssc_fps_patches": (I, [P, I, I, I, P, P, P, P, P, Z, P]),

@@ -93,6 +93,12 @@ def ssc_debug_wait_timeout(limit_ns):
     check("ssc_debug_wait_timeout", lib().ssc_debug_wait_timeout(int(limit_ns), _stream()))
 
 
+def ssc_debug_stall_next_launch(which):
+    """Abort-path test hook: 1 = next forward kernel launch, 2 = next dQ/dK
+    backward kernel launch, 0 = disarm."""
+    check("ssc_debug_stall_next_launch", lib().ssc_debug_stall_next_launch(int(which)))
+
+
 def ssc_fps_patches(pts, P, seed_vertex=0):
     """Geodesic FPS + Voronoi patches.  pts: fp32 [n,3] CUDA tensor.
     Returns (centers [P], owner [n], offsets [P+1], members [n]) int32."""

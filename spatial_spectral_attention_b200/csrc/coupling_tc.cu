@@ -97,6 +97,7 @@ struct TcParams {
   int vec_atomics;
   int vec_atomics_dq;
   int dk_tma;  // partial dK reduced by TMA through tm.dk (key rows contiguous, no column map)
+  int debug_stall;  // abort-path test hook: the MMA issuer waits on a barrier nothing arrives at
   WaitCtl ctl;
 };
 
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
   // the same index); a V stage when its P.V completes (bar_o_full of the
   // same index with two V stages, bar_v_empty with one).
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_v_full[2], bar_v_empty,
-      bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_drain, bar_xmax, bar_xsum;
+      bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_drain, bar_xmax, bar_xsum, bar_never;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   // Partial row maxima / sums exchanged between the softmax warpgroups through
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
     }
     mbar_init(&bar_v_empty, 1);
     mbar_init(&bar_drain, 1);
+    mbar_init(&bar_never, 1);  // nothing arrives: the abort-path test hook waits here
     mbar_init(&bar_xmax, NSM);
     mbar_init(&bar_xsum, NSM);
     s_abort = 0;
@@ -339,6 +341,8 @@ __global__ void __launch_bounds__(96 + 128 * NWG, 1)
         // Q is free once the tile's last S MMA completes: the next tile's Q
         // (and its first S MMAs) then overlap this tile's last P.V and epilogue
         if (ok && nk <= 2) mma_commit(&bar_q_empty);
+        // abort-path test hook: the bounded wait gives up and raises *abort
+        if (ok && p.debug_stall && tcount == 0) ok = mbar_wait(&bar_never, 0, p.ctl, abort);
         for (int j = 0; j < nk && ok; ++j) {
           const uint32_t g = it + j;
           const int buf = g & 1, vst = g % VS;
@@ -1125,7 +1129,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full,
       bar_v_empty, bar_s_full, bar_s_read, bar_dp_full, bar_ds_full, bar_do_full, bar_dkp_full,
-      bar_dkp_empty, bar_dq_full, bar_drain, bar_dp_read;
+      bar_dkp_empty, bar_dq_full, bar_drain, bar_dp_read, bar_never;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_range[3];  // first tile, first segment in it, number of units
@@ -1162,6 +1166,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     mbar_init(&bar_dkp_empty, 128);
     mbar_init(&bar_dq_full, 1);
     mbar_init(&bar_drain, 1);
+    mbar_init(&bar_never, 1);  // nothing arrives: the abort-path test hook waits here
     s_abort = 0;
     fence_barrier_init();
     // this CTA's share of the (row tile, key segment) units
@@ -1271,6 +1276,8 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
           return true;
         };
         ok = issue_s(it);
+        // abort-path test hook: the bounded wait gives up and raises *abort
+        if (ok && p.debug_stall && tcount == 0) ok = mbar_wait(&bar_never, 0, p.ctl, abort);
         // Per key tile the tensor pipe runs dP_j, S_{j+1}, dQ_j, dKp_j: the next
         // tile's S is issued as soon as the softmax has read dP_j and runs while
         // it computes dS_j; the softmax then works on S_{j+1} while dQ_j and dKp_j
@@ -2486,6 +2493,13 @@ int smem_optin() {
   return v;
 }
 
+std::atomic<int> g_stall_next{0};
+// 1 for the launch that takes the armed abort-path hook of kernel `which`.
+int take_stall(int which) {
+  int expected = which;
+  return g_stall_next.compare_exchange_strong(expected, 0) ? 1 : 0;
+}
+
 void fill_common(const TcArgs& a, TcParams& p) {
   std::memset(&p, 0, sizeof(p));
   p.tiles = a.tiles;
@@ -2510,6 +2524,8 @@ void fill_common(const TcArgs& a, TcParams& p) {
 }  // namespace
 
 bool tc_supported(int d, int k) { return (d == 64 || d == 128) && k >= 1 && k <= 256; }
+
+void tc_debug_stall_next(int which) { g_stall_next.store(which); }
 
 namespace {
 
@@ -2572,6 +2588,7 @@ cudaError_t launch_fwd_single(const TcArgs& a, float* O, int ldo, float* lse, cu
   if (e != cudaSuccess) return e;
   const int work = a.ntiles_dev ? num_sms() : a.ntiles_host;
   const int grid = std::max(1, std::min(work, num_sms()));
+  p.debug_stall = take_stall(1);
   prof_launch_begin(st);
   kern<<<grid, 96 + 128 * NWG, smem, st>>>(tm, p);
   prof_launch_end(st, SSC_PROF_FWD);
@@ -2639,9 +2656,11 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
                       : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    p.debug_stall = take_stall(2);
     prof_launch_begin(st);
     kern<<<grid, 128 * (2 + kBwdComputeGroups), smem, st>>>(tm, p);
     prof_launch_end(st, SSC_PROF_BWD_DQK);
+    p.debug_stall = 0;
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -203,6 +203,10 @@ void prof_launch_begin(cudaStream_t st);
 void prof_launch_end(cudaStream_t st, int kernel);
 
 bool tc_supported(int d, int k);
+// Abort-path test hook: the next launch of the forward (1) or dQ/dK backward
+// (2) tensor-core kernel stalls its MMA issuer on a barrier nothing arrives at
+// until the bounded wait gives up (0 disarms).
+void tc_debug_stall_next(int which);
 cudaError_t launch_tc_fwd(const TcArgs& a, float* O, int ldo, float* lse, cudaStream_t st,
                           const WaitCtl& ctl);
 // The same forward with S = Q K^T on e4m3 tensor cores: a.Q and a.K point to

@@ -239,6 +239,12 @@ int ssc_debug_wait_timeout(unsigned long long limit_ns, ssc_stream_t stream) {
   return cuda_status(launch_wait_timeout_probe(static_cast<cudaStream_t>(stream), c));
 }
 
+int ssc_debug_stall_next_launch(int which) {
+  if (which < 0 || which > 2) return SSC_ERR_INVALID_ARG;
+  tc_debug_stall_next(which);
+  return SSC_OK;
+}
+
 // ------------------------------------------------------------ patches
 int ssc_debug_fps_cluster_size(int cl) {
   if (cl != 0 && cl != 8 && cl != 16) return SSC_ERR_INVALID_ARG;

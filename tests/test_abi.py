@@ -95,3 +95,11 @@ def test_fps_cluster_size_hook_checks_its_argument():
     assert L.ssc_debug_fps_cluster_size(5) == 1
     assert L.ssc_debug_fps_cluster_size(8) == 0
     assert L.ssc_debug_fps_cluster_size(0) == 0
+
+
+def test_abort_path_hook_checks_its_argument():
+    L = _abi.lib()
+    assert L.ssc_debug_stall_next_launch(3) == 1   # SSC_ERR_INVALID_ARG
+    assert L.ssc_debug_stall_next_launch(-1) == 1
+    assert L.ssc_debug_stall_next_launch(2) == 0   # armed (host-side flag only)
+    assert L.ssc_debug_stall_next_launch(0) == 0   # and disarmed

@@ -244,6 +244,38 @@ def test_wait_timeout_reports_status_without_fault():
     _dense_case(Qn, Kn, Vn, dOn, 0.125, "bf16", need_dV=False)
 
 
+@pytest.mark.parametrize("which", [1, 2])
+def test_coupling_kernel_abort_path_leaves_context_usable(which):
+    # The library's abort-path hook stalls the MMA issuer of the next forward
+    # (1) or dQ/dK backward (2) tensor-core launch on a barrier nothing arrives
+    # at.  The bounded wait gives up after the wait limit: the launch ends with
+    # the timeout status (every role left its loop, the MMAs drained, TMEM was
+    # freed), and the same calls right after it give the oracle's results.
+    pair = synth.make_workload("geo_60k", n=3000)
+    P, R = 24, 5
+    t = _geo_tables(pair, P, R, "bf16")
+    (Q, K, V, dO), (Q64, K64, V64, dO64) = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, "bf16")
+    tabs = [as_i32(t[x]) for x in ("off_N", "mem_N", "off_M", "mem_M", "topk")]
+    api.ssc_device_status(clear=True)
+    api.ssc_set_wait_limit_ns(50_000_000)  # 50 ms
+    try:
+        api.ssc_debug_stall_next_launch(which)
+        O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, *tabs)
+        api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs)
+        assert api.ssc_device_status(clear=True) == 6
+    finally:
+        api.ssc_debug_stall_next_launch(0)
+        api.ssc_set_wait_limit_ns(0)
+    O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, *tabs)
+    dQ, dK, _ = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs)
+    _status_ok()
+    ref = oracle.geo_bwd(Q64, K64, V64, dO64, pair.scale, t["off_N"], t["mem_N"], t["off_M"],
+                         t["mem_M"], t["topk"])
+    assert_close(O, ref["O"], TOL_BF16, "O")
+    assert_close(dQ, ref["dQ"], TOL_BF16, "dQ")
+    assert_close(dK, ref["dK"], TOL_BF16, "dK")
+
+
 def test_profile_record_times_each_coupling_launch():
     torch.manual_seed(0)
     n, d, k = 3000, 128, 196
