@@ -48,30 +48,67 @@ __device__ __forceinline__ double dot3_rn(float a0, float a1, float a2, float b0
   return __dadd_rn(__dadd_rn(p0, p1), p2);
 }
 
-__device__ __forceinline__ Cand warp_min(Cand c) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Cand x;
-    x.val = __shfl_xor_sync(0xffffffffu, c.val, o);
-    x.idx = __shfl_xor_sync(0xffffffffu, c.idx, o);
-    if (cand_before(x, c)) c = x;
-  }
-  return c;
+__device__ __forceinline__ double dot3_rn(double a0, double a1, double a2, double b0, double b1,
+                                          double b2) {
+  return __dadd_rn(__dadd_rn(__dmul_rn(a0, b0), __dmul_rn(a1, b1)), __dmul_rn(a2, b2));
 }
 
-// A CTA's candidate as it travels through distributed shared memory: its
-// largest dot, index and coordinates (so the next round needs no global load).
+// Unsigned key that orders like the double (no NaN here): the sign bit is
+// flipped for non-negative values, every bit for negative ones; -0 is first
+// made +0, since the two compare equal.
+__device__ __forceinline__ unsigned long long order_key(double v) {
+  const long long b = __double_as_longlong(v + 0.0);
+  return b >= 0 ? (unsigned long long)b ^ 0x8000000000000000ull : ~(unsigned long long)b;
+}
+
+// The warp's first candidate in cand_before order, agreed by every lane: three
+// min reductions (key high word, key low word among the lanes holding the
+// smallest high word, vertex index among the lanes holding the smallest key).
+__device__ __forceinline__ Cand warp_min(Cand c) {
+  const unsigned long long k = order_key(c.val);
+  const unsigned hi = (unsigned)(k >> 32), lo = (unsigned)k;
+  const unsigned mh = __reduce_min_sync(0xffffffffu, hi);
+  const unsigned ml = __reduce_min_sync(0xffffffffu, hi == mh ? lo : 0xffffffffu);
+  const bool top = hi == mh && lo == ml;
+  const unsigned mi = __reduce_min_sync(0xffffffffu, top ? (unsigned)c.idx : 0xffffffffu);
+  const unsigned who = __ballot_sync(0xffffffffu, top && (unsigned)c.idx == mi);
+  return Cand{__shfl_sync(0xffffffffu, c.val, __ffs(who) - 1), (int)mi};
+}
+
+// A candidate by the order key of its largest dot (order_key, so that the
+// integer order is the double order) and its vertex index.
+struct KCand {
+  unsigned long long key;
+  int idx;
+};
+__device__ __forceinline__ bool kcand_before(const KCand& a, const KCand& b) {
+  return a.key < b.key || (a.key == b.key && a.idx < b.idx);
+}
+// The warp's first candidate, agreed by every lane (three min reductions).
+__device__ __forceinline__ KCand warp_min_key(const KCand& c) {
+  const unsigned hi = (unsigned)(c.key >> 32), lo = (unsigned)c.key;
+  const unsigned mh = __reduce_min_sync(0xffffffffu, hi);
+  const unsigned ml = __reduce_min_sync(0xffffffffu, hi == mh ? lo : 0xffffffffu);
+  const unsigned mi =
+      __reduce_min_sync(0xffffffffu, (hi == mh && lo == ml) ? (unsigned)c.idx : 0xffffffffu);
+  return KCand{((unsigned long long)mh << 32) | ml, (int)mi};
+}
+
+// A CTA's candidate as it travels through distributed shared memory: its key,
+// index and coordinates (so the next round needs no global load).
 struct CandXYZ {
-  double val;
+  unsigned long long key;
   int idx;
   float x, y, z;
 };
 
 // Cluster FPS: the CTA of rank r owns points [r*per, min(n,(r+1)*per));
 // their coordinates sit in shared memory (structure of arrays), the running
-// largest dot and patch of each point in registers (PPT points per thread).
-// A round: every thread updates its points and its best candidate; the CTA's
-// warps reduce to one candidate; warp 0 pushes it, with the point's
+// largest dot (as its order key) and patch of each point in registers (PPT
+// points per thread).  A round: every thread updates its points; a thread's
+// best candidate, and its warp's, are recomputed only when one of its points
+// changed (largest dots only grow, so an unchanged minimum stays the minimum);
+// warp 0 reduces the warps' candidates and pushes the CTA's, with the point's
 // coordinates, into slot `rank` of every CTA; after the cluster barrier warp 0
 // reduces the CL slots and publishes the next centre and its coordinates in
 // shared memory, so no round reads the centre from global memory.
@@ -82,8 +119,8 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  extern __shared__ float sx[];  // [3][PPT * kFpsThreads]
-  __shared__ Cand warp_c[kFpsThreads / 32];
+  extern __shared__ float sx[];  // [3 or 4][PPT * kFpsThreads]: x, y, z (and |x|_1)
+  __shared__ KCand warp_c[kFpsThreads / 32];
   __shared__ CandXYZ slots[2][16];
   __shared__ CandXYZ s_next;
 
@@ -91,54 +128,97 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
   const int cap = PPT * kFpsThreads;
   const int v0 = rank * per;
   const int cnt = max(0, min(n - v0, per));
+  constexpr bool kFilter = PPT <= 10;
   for (int i = tid; i < cnt; i += kFpsThreads) {
-    sx[i] = pts[3 * (size_t)(v0 + i)];
-    sx[cap + i] = pts[3 * (size_t)(v0 + i) + 1];
-    sx[2 * cap + i] = pts[3 * (size_t)(v0 + i) + 2];
+    const float x = pts[3 * (size_t)(v0 + i)], y = pts[3 * (size_t)(v0 + i) + 1],
+                z = pts[3 * (size_t)(v0 + i) + 2];
+    sx[i] = x;
+    sx[cap + i] = y;
+    sx[2 * cap + i] = z;
+    if (kFilter) sx[3 * cap + i] = fabsf(x) + fabsf(y) + fabsf(z);
   }
-  double best[PPT];
+  // Per point: the order key of its largest dot so far (comparisons of keys
+  // are comparisons of the fp64 values) and its patch.
+  unsigned long long bkey[PPT];
   int own[PPT];
   uint32_t chosen = 0;
+  // fp32 filter (PPT <= 10): bestf = the largest dot rounded toward -inf.  The
+  // exact fp64 dot g of a point and the new centre differs from the fp32 dot
+  // ga (fma chain in the same order) by at most 3 roundings of 2^-24 of
+  // S = |x0 b0| + |x1 b1| + |x2 b2| <= |x|_1 max_k |b_k| (plus 2^-148 when the
+  // products are subnormal); with the margin tol = 2^-20 |x|_1 max_k |b_k| +
+  // 2^-126 (which also covers the rounding of ga + tol and of the fp64 sum),
+  // ga + tol < bestf implies g < best: the point keeps its best and owner, and
+  // the fp64 dot is skipped.  Every other case (including non-finite ga or tol)
+  // takes the exact fp64 comparison, so the results are those of the plain
+  // fp64 definition.
+  float bestf[kFilter ? PPT : 1];
+  const unsigned long long key_lowest = order_key(-DBL_MAX);
 #pragma unroll
   for (int i = 0; i < PPT; ++i) {
-    best[i] = -DBL_MAX;
+    bkey[i] = key_lowest;
     own[i] = -1;
+    if (kFilter) bestf[i] = -INFINITY;
     if (i * kFpsThreads + tid >= cnt) chosen |= 1u << i;  // padding never competes
   }
   __syncthreads();
   int c = seed;
   float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
         c2 = __ldg(pts + 3 * (size_t)c + 2);
+  KCand mine{~0ull, INT_MAX};  // this thread's best candidate
   for (int t = 0; t < P; ++t) {
     if (rank == 0 && tid == 0) centers[t] = c;
-    Cand mine{DBL_MAX, INT_MAX};
+    bool dirty = t == 0;  // a point of this thread changed: recompute its candidate
+    const double d0 = (double)c0, d1 = (double)c1, d2 = (double)c2;
+    const float btol = fmaxf(fabsf(c0), fmaxf(fabsf(c1), fabsf(c2))) * 0x1p-20f;
 #pragma unroll
     for (int i = 0; i < PPT; ++i) {
       const int li = i * kFpsThreads + tid;
       if (v0 + li == c) {
         chosen |= 1u << i;
         own[i] = t;
+        dirty = true;
       }
       if (!(chosen >> i & 1u)) {
-        double g = dot3_rn(sx[li], sx[cap + li], sx[2 * cap + li], c0, c1, c2);
-        if (g > best[i]) {
-          best[i] = g;
-          own[i] = t;
+        const float x0 = sx[li], x1 = sx[cap + li], x2 = sx[2 * cap + li];
+        bool exact = true;
+        if (kFilter) {
+          const float ga = fmaf(x2, c2, fmaf(x1, c1, x0 * c0));
+          const float tol = fmaf(sx[3 * cap + li], btol, FLT_MIN);
+          exact = !(ga + tol < bestf[i] && fabsf(ga) + tol <= FLT_MAX);
         }
-        Cand me{best[i], v0 + li};
-        if (cand_before(me, mine)) mine = me;
+        if (exact) {
+          const double g = dot3_rn((double)x0, (double)x1, (double)x2, d0, d1, d2);
+          const unsigned long long gk = order_key(g);
+          if (gk > bkey[i]) {
+            bkey[i] = gk;
+            own[i] = t;
+            if (kFilter) bestf[i] = __double2float_rd(g);
+            dirty = true;
+          }
+        }
       }
     }
     if (t + 1 == P) break;
-    mine = warp_min(mine);
-    if ((tid & 31) == 0) warp_c[tid >> 5] = mine;
+    if (dirty) {
+      mine = KCand{~0ull, INT_MAX};
+#pragma unroll
+      for (int i = 0; i < PPT; ++i) {
+        const KCand me{bkey[i], v0 + i * kFpsThreads + tid};
+        if (!(chosen >> i & 1u) && kcand_before(me, mine)) mine = me;
+      }
+    }
+    // the warp's candidate (in warp_c across rounds) changes only with a lane's
+    if (__any_sync(0xffffffffu, dirty)) {
+      const KCand w = warp_min_key(mine);
+      if ((tid & 31) == 0) warp_c[tid >> 5] = w;
+    }
     __syncthreads();
     if (tid < 32) {
-      Cand w = warp_c[tid];
-      w = warp_min(w);
+      const KCand w = warp_min_key(warp_c[tid]);
       if (tid < CL) {
         // push this CTA's candidate, with its coordinates, into slot `rank` of CTA `tid`
-        CandXYZ cx{w.val, w.idx, 0.f, 0.f, 0.f};
+        CandXYZ cx{w.key, w.idx, 0.f, 0.f, 0.f};
         if (w.idx != INT_MAX) {
           const int li = w.idx - v0;
           cx.x = sx[li];
@@ -151,9 +231,9 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
     cluster.sync();
     if (tid < 32) {
       // warp 0 reduces the CL slots (ties to the lower vertex index)
-      Cand w{DBL_MAX, INT_MAX};
-      if (tid < CL) w = Cand{slots[t & 1][tid].val, slots[t & 1][tid].idx};
-      const Cand win = warp_min(w);
+      KCand w{~0ull, INT_MAX};
+      if (tid < CL) w = KCand{slots[t & 1][tid].key, slots[t & 1][tid].idx};
+      const KCand win = warp_min_key(w);
       if (tid < CL && slots[t & 1][tid].idx == win.idx) s_next = slots[t & 1][tid];
     }
     __syncthreads();
@@ -358,7 +438,8 @@ template <int PPT>
 cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, int* owner, int CL,
                        cudaStream_t st) {
   auto kern = fps_cluster_kernel<PPT>;
-  const int smem = 3 * PPT * kFpsThreads * (int)sizeof(float);
+  // x, y, z, and |x|_1 for the fp32 filter (PPT <= 10)
+  const int smem = (PPT <= 10 ? 4 : 3) * PPT * kFpsThreads * (int)sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -435,6 +516,7 @@ cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* ce
   else if (ppt <= 2) e = launch_reg<2>(pts, n, P, seed, centers, owner, CL, st);
   else if (ppt <= 4) e = launch_reg<4>(pts, n, P, seed, centers, owner, CL, st);
   else if (ppt <= 8) e = launch_reg<8>(pts, n, P, seed, centers, owner, CL, st);
+  else if (ppt <= 10) e = launch_reg<10>(pts, n, P, seed, centers, owner, CL, st);
   else if (ppt <= 16) e = launch_reg<16>(pts, n, P, seed, centers, owner, CL, st);
   else {
     if (CL > 8)
