@@ -102,27 +102,51 @@ struct CandXYZ {
   float x, y, z;
 };
 
+// Address of the same shared-memory variable in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// 16-byte store into another CTA's shared memory that completes its bytes on
+// that CTA's mbarrier (both addresses in the cluster window).
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, const uint4& v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          raddr),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(rbar)
+      : "memory");
+}
+
 // Cluster FPS: the CTA of rank r owns points [r*per, min(n,(r+1)*per));
 // their coordinates sit in shared memory (structure of arrays), the running
 // largest dot (as its order key) and patch of each point in registers (PPT
 // points per thread).  A round: every thread updates its points; a thread's
 // best candidate, and its warp's, are recomputed only when one of its points
 // changed (largest dots only grow, so an unchanged minimum stays the minimum);
-// warp 0 reduces the warps' candidates and pushes the CTA's, with the point's
-// coordinates, into slot `rank` of every CTA; after the cluster barrier warp 0
-// reduces the CL slots and publishes the next centre and its coordinates in
-// shared memory, so no round reads the centre from global memory.
+// warp 0 reduces the warps' candidates and its lane j stores the CTA's (with
+// the point's coordinates) into slot `rank` of CTA j with st.async, which
+// completes on CTA j's slot barrier of the round's parity.  Each CTA's warp 0
+// then waits on its own barrier (armed once per round for the CL slots: no
+// cluster-wide barrier), reduces the slots and publishes the next centre and
+// its coordinates in shared memory.  The two slot buffers alternate by round:
+// CTA r can store round t + 2 into CTA j's buffer only after receiving CTA j's
+// round t + 1 candidate, which CTA j sends after reading its round t slots.
+// Every wait is bounded; on expiry the status word records the timeout and
+// every CTA leaves its rounds (the others' waits run out in turn).
 template <int PPT>
 __global__ void __launch_bounds__(kFpsThreads, 1)
     fps_cluster_kernel(const float* __restrict__ pts, int n, int P, int seed, int per,
-                       int* __restrict__ centers, int* __restrict__ owner) {
+                       int* __restrict__ centers, int* __restrict__ owner, WaitCtl ctl) {
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   extern __shared__ float sx[];  // [3 or 4][PPT * kFpsThreads]: x, y, z (and |x|_1)
   __shared__ KCand warp_c[kFpsThreads / 32];
-  __shared__ CandXYZ slots[2][16];
+  __shared__ __align__(16) uint4 slots[2][16][2];  // 32 bytes per CTA: key, idx, x, y, z
+  __shared__ uint64_t bar_slot[2];
   __shared__ CandXYZ s_next;
+  __shared__ int s_abort;
 
   const int tid = threadIdx.x;
   const int cap = PPT * kFpsThreads;
@@ -161,13 +185,23 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
     if (kFilter) bestf[i] = -INFINITY;
     if (i * kFpsThreads + tid >= cnt) chosen |= 1u << i;  // padding never competes
   }
+  if (tid == 0) {
+    mbar_init(&bar_slot[0], 1);
+    mbar_init(&bar_slot[1], 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
   __syncthreads();
+  cluster.sync();  // every CTA's slot barriers exist before the first remote store
   int c = seed;
   float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
         c2 = __ldg(pts + 3 * (size_t)c + 2);
   KCand mine{~0ull, INT_MAX};  // this thread's best candidate
   for (int t = 0; t < P; ++t) {
     if (rank == 0 && tid == 0) centers[t] = c;
+    // arm this round's slot barrier for the CL candidates (they may land first:
+    // the barrier's byte count goes below zero until this arrival)
+    if (tid == 0 && t + 1 < P) mbar_arrive_expect_tx(&bar_slot[t & 1], 32u * CL);
     bool dirty = t == 0;  // a point of this thread changed: recompute its candidate
     const double d0 = (double)c0, d1 = (double)c1, d2 = (double)c2;
     const float btol = fmaxf(fabsf(c0), fmaxf(fabsf(c1), fabsf(c2))) * 0x1p-20f;
@@ -217,26 +251,36 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
     if (tid < 32) {
       const KCand w = warp_min_key(warp_c[tid]);
       if (tid < CL) {
-        // push this CTA's candidate, with its coordinates, into slot `rank` of CTA `tid`
-        CandXYZ cx{w.key, w.idx, 0.f, 0.f, 0.f};
+        // this CTA's candidate, with its coordinates, into slot `rank` of CTA `tid`
+        float x = 0.f, y = 0.f, z = 0.f;
         if (w.idx != INT_MAX) {
           const int li = w.idx - v0;
-          cx.x = sx[li];
-          cx.y = sx[cap + li];
-          cx.z = sx[2 * cap + li];
+          x = sx[li];
+          y = sx[cap + li];
+          z = sx[2 * cap + li];
         }
-        *cluster.map_shared_rank(&slots[t & 1][rank], tid) = cx;
+        const uint32_t ra = mapa_shared(smem_u32(&slots[t & 1][rank][0]), tid);
+        const uint32_t rb = mapa_shared(smem_u32(&bar_slot[t & 1]), tid);
+        st_async_v4(ra, make_uint4((uint32_t)w.key, (uint32_t)(w.key >> 32), (uint32_t)w.idx,
+                                   __float_as_uint(x)),
+                    rb);
+        st_async_v4(ra + 16, make_uint4(__float_as_uint(y), __float_as_uint(z), 0u, 0u), rb);
       }
-    }
-    cluster.sync();
-    if (tid < 32) {
-      // warp 0 reduces the CL slots (ties to the lower vertex index)
-      KCand w{~0ull, INT_MAX};
-      if (tid < CL) w = KCand{slots[t & 1][tid].key, slots[t & 1][tid].idx};
-      const KCand win = warp_min_key(w);
-      if (tid < CL && slots[t & 1][tid].idx == win.idx) s_next = slots[t & 1][tid];
+      // the CL candidates of this round in this CTA's slots (ties to the lower vertex)
+      const bool ok = mbar_wait_cluster(&bar_slot[t & 1], (t >> 1) & 1, ctl, &s_abort);
+      KCand x{~0ull, INT_MAX};
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+      if (ok && tid < CL) {
+        a = slots[t & 1][tid][0];
+        b = slots[t & 1][tid][1];
+        x = KCand{((unsigned long long)a.y << 32) | a.x, (int)a.z};
+      }
+      const KCand win = warp_min_key(x);
+      if (ok && tid < CL && x.idx == win.idx)
+        s_next = CandXYZ{x.key, x.idx, __uint_as_float(a.w), __uint_as_float(b.x), __uint_as_float(b.y)};
     }
     __syncthreads();
+    if (s_abort) break;  // a wait ran out: leave the rounds (the status word says so)
     c = s_next.idx;
     c0 = s_next.x;
     c1 = s_next.y;
@@ -436,7 +480,7 @@ int fps_cluster_size() {
 
 template <int PPT>
 cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, int* owner, int CL,
-                       cudaStream_t st) {
+                       cudaStream_t st, const WaitCtl& ctl) {
   auto kern = fps_cluster_kernel<PPT>;
   // x, y, z, and |x|_1 for the fp32 filter (PPT <= 10)
   const int smem = (PPT <= 10 ? 4 : 3) * PPT * kFpsThreads * (int)sizeof(float);
@@ -458,7 +502,7 @@ cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, i
   cfg.numAttrs = 1;
   count_launch();
   prof_launch_begin(st);
-  e = cudaLaunchKernelEx(&cfg, kern, pts, n, P, seed, per, centers, owner);
+  e = cudaLaunchKernelEx(&cfg, kern, pts, n, P, seed, per, centers, owner, ctl);
   prof_launch_end(st, SSC_PROF_FPS);
   return e;
 }
@@ -480,7 +524,7 @@ size_t fps_workspace_bytes(int n, int P) {
 
 cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* centers, int* owner,
                                int* offsets, int* members, void* ws, cudaStream_t st,
-                               const WaitCtl&) {
+                               const WaitCtl& ctl) {
   Carve c(ws);
   int* counts = c.take<int>(P);
   int* cursor = c.take<int>(P);
@@ -512,12 +556,12 @@ cudaError_t launch_fps_patches(const float* pts, int n, int P, int seed, int* ce
   const long per = (n + CL - 1) / CL;
   const long ppt = (per + kFpsThreads - 1) / kFpsThreads;
   cudaError_t e;
-  if (ppt <= 1) e = launch_reg<1>(pts, n, P, seed, centers, owner, CL, st);
-  else if (ppt <= 2) e = launch_reg<2>(pts, n, P, seed, centers, owner, CL, st);
-  else if (ppt <= 4) e = launch_reg<4>(pts, n, P, seed, centers, owner, CL, st);
-  else if (ppt <= 8) e = launch_reg<8>(pts, n, P, seed, centers, owner, CL, st);
-  else if (ppt <= 10) e = launch_reg<10>(pts, n, P, seed, centers, owner, CL, st);
-  else if (ppt <= 16) e = launch_reg<16>(pts, n, P, seed, centers, owner, CL, st);
+  if (ppt <= 1) e = launch_reg<1>(pts, n, P, seed, centers, owner, CL, st, ctl);
+  else if (ppt <= 2) e = launch_reg<2>(pts, n, P, seed, centers, owner, CL, st, ctl);
+  else if (ppt <= 4) e = launch_reg<4>(pts, n, P, seed, centers, owner, CL, st, ctl);
+  else if (ppt <= 8) e = launch_reg<8>(pts, n, P, seed, centers, owner, CL, st, ctl);
+  else if (ppt <= 10) e = launch_reg<10>(pts, n, P, seed, centers, owner, CL, st, ctl);
+  else if (ppt <= 16) e = launch_reg<16>(pts, n, P, seed, centers, owner, CL, st, ctl);
   else {
     if (CL > 8)
       cudaFuncSetAttribute(fps_cluster_mem_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,

@@ -60,6 +60,7 @@ extern "C" int ssc_fps_patches_noalloc(const float* pts, int n, int P, int seed_
   if (rc != SSC_OK) return rc;
   (void)cudaGetLastError();
   const ssc::WaitCtl ctl = ssc::library_wait_ctl();
+  if (!ctl.status) return SSC_ERR_CUDA;
   return ssc::launch_fps_patches(pts, n, P, seed_vertex, centers, owner, offsets, members, ws,
                                  static_cast<cudaStream_t>(stream), ctl) == cudaSuccess
              ? SSC_OK

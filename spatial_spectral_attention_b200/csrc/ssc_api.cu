@@ -265,6 +265,7 @@ int ssc_fps_patches(const float* pts, int n, int P, int seed_vertex, int* center
   if (!ws_ok(ws, ws_bytes, fps_workspace_bytes(n, P))) return SSC_ERR_WORKSPACE;
   (void)cudaGetLastError();  // clear a stale error left by an earlier, unrelated call
   WaitCtl c = make_ctl();
+  if (!c.status) return SSC_ERR_CUDA;
   return cuda_status(launch_fps_patches(pts, n, P, seed_vertex, centers, owner, offsets, members, ws,
                                         static_cast<cudaStream_t>(stream), c));
 }
