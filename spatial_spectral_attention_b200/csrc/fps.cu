@@ -294,6 +294,352 @@ __global__ void __launch_bounds__(kFpsThreads, 1)
   cluster.sync();  // no CTA leaves while others may still write its slots
 }
 
+// Unsigned key that orders like the float (no NaN); -0 is first made +0.
+__device__ __forceinline__ unsigned order_key_f(float v) {
+  const int b = __float_as_int(v + 0.0f);
+  return b >= 0 ? (unsigned)b ^ 0x80000000u : ~(unsigned)b;
+}
+__device__ __forceinline__ float from_order_key_f(unsigned k) {
+  return __int_as_float((int)((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k));
+}
+// Spreads the 10 low bits of v three apart (bit i to bit 3 i).
+__device__ __forceinline__ unsigned spread10(unsigned v) {
+  v &= 1023u;
+  v = (v | (v << 16)) & 0x030000ffu;
+  v = (v | (v << 8)) & 0x0300f00fu;
+  v = (v | (v << 4)) & 0x030c30c3u;
+  v = (v | (v << 2)) & 0x09249249u;
+  return v;
+}
+// Morton code of a point with 10 bits per axis over the box [lo, lo + 1023 / s].
+__device__ __forceinline__ unsigned morton3(float x, float y, float z, const float (&lo)[3],
+                                           const float (&s)[3]) {
+  const float p[3] = {x, y, z};
+  unsigned q[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) q[k] = (unsigned)fminf(fmaxf((p[k] - lo[k]) * s[k], 0.f), 1023.f);
+  return spread10(q[0]) | (spread10(q[1]) << 1) | (spread10(q[2]) << 2);
+}
+
+// Cluster FPS with spatial culling (8 to 10 points per thread).  At the
+// start each CTA sorts its points by Morton code (bitonic sort in shared
+// memory) and lays them out so that warp w holds the 32 PPT consecutive points
+// [32 PPT w, 32 PPT (w + 1)) of that order: a compact group with a reference
+// point g (its centroid) and radius R >= max |p - g| (rounded up).  For every
+// point p of the group and the round's centre c, dot(p, c) <= dot(g, c) +
+// R |c|.  When that bound plus a margin for its fp32 rounding (and for the
+// fp64 dot's) lies below the smallest bestf (largest dot so far, rounded
+// toward -inf) of the group's remaining points, no point of the warp can
+// change in this round and the warp skips its points; otherwise they are
+// updated as in fps_cluster_kernel (fp32 filter, exact fp64 comparison).  The
+// results, and the candidate order (largest dot, then original vertex index),
+// are those of the plain fp64 definition.  The centre's CTA and slot travel
+// with the candidate, so only the thread holding the centre marks it.  The
+// candidate exchange is that of fps_cluster_kernel (st.async into every CTA's
+// slot, completing on the receiver's barrier, bounded waits).
+template <int PPT>
+__global__ void __launch_bounds__(kFpsThreads, 1)
+    fps_cull_kernel(const float* __restrict__ pts, int n, int P, int seed, int per,
+                    int* __restrict__ centers, int* __restrict__ owner, WaitCtl ctl) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  constexpr int cap = PPT * kFpsThreads;
+  constexpr int NS = PPT <= 1 ? 1024 : PPT <= 2 ? 2048 : PPT <= 4 ? 4096 : PPT <= 8 ? 8192 : 16384;
+  // Dynamic shared memory: x, y, z, |x|_1 of every slot (floats), then its
+  // original vertex (int, -1 for padding).  The sort buffer (NS 64-bit keys)
+  // uses the same bytes before they are filled.
+  extern __shared__ float sx[];
+  int* so = reinterpret_cast<int*>(sx + 4 * cap);
+  unsigned long long* sortbuf = reinterpret_cast<unsigned long long*>(sx);
+  __shared__ KCand warp_c[kFpsThreads / 32];
+  __shared__ int warp_slot[kFpsThreads / 32];
+  __shared__ __align__(16) uint4 slots[2][16][2];  // key, idx, x | y, z, slot
+  __shared__ uint64_t bar_slot[2];
+  __shared__ CandXYZ s_next;
+  __shared__ int s_next_rank, s_next_slot;
+  __shared__ unsigned s_box[6];
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int v0 = rank * per;
+  const int cnt = max(0, min(n - v0, per));
+  if (tid == 0) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      s_box[k] = 0xffffffffu;
+      s_box[3 + k] = 0u;
+    }
+    s_next_rank = -1;
+    s_next_slot = 0;
+    s_abort = 0;
+    mbar_init(&bar_slot[0], 1);
+    mbar_init(&bar_slot[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // 1. bounding box of the CTA's points
+  {
+    unsigned mn[3] = {~0u, ~0u, ~0u}, mx[3] = {0u, 0u, 0u};
+    for (int i = tid; i < cnt; i += kFpsThreads)
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const unsigned kk = order_key_f(pts[3 * (size_t)(v0 + i) + k]);
+        mn[k] = min(mn[k], kk);
+        mx[k] = max(mx[k], kk);
+      }
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      mn[k] = __reduce_min_sync(0xffffffffu, mn[k]);
+      mx[k] = __reduce_max_sync(0xffffffffu, mx[k]);
+      if (lane == 0) {
+        atomicMin(&s_box[k], mn[k]);
+        atomicMax(&s_box[3 + k], mx[k]);
+      }
+    }
+  }
+  __syncthreads();
+  // 2. Morton keys and an ascending bitonic sort of (key << 32 | local index)
+  if (cnt > 0) {
+    float lo[3], sc[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      lo[k] = from_order_key_f(s_box[k]);
+      const float ext = from_order_key_f(s_box[3 + k]) - lo[k];
+      sc[k] = ext > 0.f ? 1023.f / ext : 0.f;
+    }
+    for (int s = tid; s < NS; s += kFpsThreads) {
+      unsigned long long e = ~0ull;
+      if (s < cnt)
+        e = ((unsigned long long)morton3(pts[3 * (size_t)(v0 + s)], pts[3 * (size_t)(v0 + s) + 1],
+                                         pts[3 * (size_t)(v0 + s) + 2], lo, sc)
+             << 32) |
+            (unsigned)s;
+      sortbuf[s] = e;
+    }
+    __syncthreads();
+    for (int k = 2; k <= NS; k <<= 1)
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < NS; i += kFpsThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long a = sortbuf[i], b = sortbuf[ixj];
+            if ((a > b) == ((i & k) == 0)) {
+              sortbuf[i] = b;
+              sortbuf[ixj] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+  }
+  // 3. slot (i, tid) = sx index i kFpsThreads + tid holds sorted position
+  //    32 PPT warp + 32 i + lane
+  int perm[PPT];
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    const int s = 32 * PPT * warp + 32 * i + lane;
+    perm[i] = s < cnt ? (int)(sortbuf[s] & 0xffffffffull) : -1;
+  }
+  __syncthreads();  // the sort buffer is read; its bytes become the slot arrays
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    const int li = i * kFpsThreads + tid;
+    float x = 0.f, y = 0.f, z = 0.f;
+    if (perm[i] >= 0) {
+      x = pts[3 * (size_t)(v0 + perm[i])];
+      y = pts[3 * (size_t)(v0 + perm[i]) + 1];
+      z = pts[3 * (size_t)(v0 + perm[i]) + 2];
+    }
+    sx[li] = x;
+    sx[cap + li] = y;
+    sx[2 * cap + li] = z;
+    sx[3 * cap + li] = fabsf(x) + fabsf(y) + fabsf(z);
+    so[li] = perm[i] >= 0 ? v0 + perm[i] : -1;
+    if (perm[i] >= 0 && v0 + perm[i] == seed) {
+      s_next_rank = rank;
+      s_next_slot = li;
+    }
+  }
+  // 4. the warp's group: centroid g and radius R (rounded up: the fp32
+  //    differences, squares, sum and square root stay within 2^-18 of R)
+  float gx = 0.f, gy = 0.f, gz = 0.f, gR = 0.f;
+  {
+    float ax = 0.f, ay = 0.f, az = 0.f, m = 0.f;
+#pragma unroll
+    for (int i = 0; i < PPT; ++i)
+      if (perm[i] >= 0) {
+        const int li = i * kFpsThreads + tid;
+        ax += sx[li];
+        ay += sx[cap + li];
+        az += sx[2 * cap + li];
+        m += 1.f;
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ax += __shfl_xor_sync(0xffffffffu, ax, o);
+      ay += __shfl_xor_sync(0xffffffffu, ay, o);
+      az += __shfl_xor_sync(0xffffffffu, az, o);
+      m += __shfl_xor_sync(0xffffffffu, m, o);
+    }
+    if (m > 0.f) {
+      gx = ax / m;
+      gy = ay / m;
+      gz = az / m;
+    }
+    float r2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < PPT; ++i)
+      if (perm[i] >= 0) {
+        const int li = i * kFpsThreads + tid;
+        const float dx = sx[li] - gx, dy = sx[cap + li] - gy, dz = sx[2 * cap + li] - gz;
+        r2 = fmaxf(r2, fmaf(dz, dz, fmaf(dy, dy, dx * dx)));
+      }
+    r2 = from_order_key_f(__reduce_max_sync(0xffffffffu, order_key_f(r2)));
+    gR = sqrtf(r2) * (1.0f + 0x1p-18f) + FLT_MIN;
+  }
+  const float g1 = fabsf(gx) + fabsf(gy) + fabsf(gz);
+  unsigned long long bkey[PPT];
+  int own[PPT];
+  float bestf[PPT];
+  uint32_t chosen = 0;
+  const unsigned long long key_lowest = order_key(-DBL_MAX);
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    bkey[i] = key_lowest;
+    own[i] = -1;
+    bestf[i] = -INFINITY;
+    if (perm[i] < 0) chosen |= 1u << i;  // padding never competes
+  }
+  __syncthreads();
+  cluster.sync();  // every CTA's slot barriers exist before the first remote store
+  int c = seed, c_rank = s_next_rank, c_slot = s_next_slot;
+  float c0 = __ldg(pts + 3 * (size_t)c), c1 = __ldg(pts + 3 * (size_t)c + 1),
+        c2 = __ldg(pts + 3 * (size_t)c + 2);
+  KCand mine{~0ull, INT_MAX};  // this thread's best candidate and its slot
+  int mslot = 0;
+  float mw = -INFINITY;  // smallest bestf among the warp's remaining points
+  for (int t = 0; t < P; ++t) {
+    if (rank == 0 && tid == 0) centers[t] = c;
+    if (tid == 0 && t + 1 < P) mbar_arrive_expect_tx(&bar_slot[t & 1], 32u * CL);
+    bool dirty = t == 0;
+    if (c_rank == rank && (c_slot & (kFpsThreads - 1)) == tid) {
+#pragma unroll
+      for (int i = 0; i < PPT; ++i)
+        if (i == c_slot / kFpsThreads) {
+          chosen |= 1u << i;
+          own[i] = t;
+        }
+      dirty = true;
+    }
+    // the group bound: skip the warp when no remaining point can change
+    const float cinf = fmaxf(fabsf(c0), fmaxf(fabsf(c1), fabsf(c2)));
+    const float cn = sqrtf(fmaf(c2, c2, fmaf(c1, c1, c0 * c0))) * (1.0f + 0x1p-18f);
+    const float ub = fmaf(gz, c2, fmaf(gy, c1, gx * c0)) + gR * cn;
+    const float um = fmaf(fmaf(g1, cinf, gR * cn), 0x1p-20f, FLT_MIN);
+    const bool skip = ub + um < mw && fabsf(ub) + um <= FLT_MAX;
+    if (!skip) {
+      const double d0 = (double)c0, d1 = (double)c1, d2 = (double)c2;
+      const float btol = cinf * 0x1p-20f;
+#pragma unroll
+      for (int i = 0; i < PPT; ++i) {
+        if (chosen >> i & 1u) continue;
+        const int li = i * kFpsThreads + tid;
+        const float x0 = sx[li], x1 = sx[cap + li], x2 = sx[2 * cap + li];
+        const float ga = fmaf(x2, c2, fmaf(x1, c1, x0 * c0));
+        const float tol = fmaf(sx[3 * cap + li], btol, FLT_MIN);
+        if (ga + tol < bestf[i] && fabsf(ga) + tol <= FLT_MAX) continue;
+        const double g = dot3_rn((double)x0, (double)x1, (double)x2, d0, d1, d2);
+        const unsigned long long gk = order_key(g);
+        if (gk > bkey[i]) {
+          bkey[i] = gk;
+          own[i] = t;
+          bestf[i] = __double2float_rd(g);
+          dirty = true;
+        }
+      }
+    }
+    if (t + 1 == P) break;
+    if (dirty) {
+      mine = KCand{~0ull, INT_MAX};
+#pragma unroll
+      for (int i = 0; i < PPT; ++i) {
+        if (chosen >> i & 1u) continue;
+        const int li = i * kFpsThreads + tid;
+        const KCand me{bkey[i], so[li]};
+        if (kcand_before(me, mine)) {
+          mine = me;
+          mslot = li;
+        }
+      }
+    }
+    if (__any_sync(0xffffffffu, dirty)) {
+      const KCand w = warp_min_key(mine);
+      const unsigned who = __ballot_sync(0xffffffffu, mine.key == w.key && mine.idx == w.idx);
+      const int ws = __shfl_sync(0xffffffffu, mslot, __ffs(who) - 1);
+      if (lane == 0) {
+        warp_c[warp] = w;
+        warp_slot[warp] = ws;
+      }
+      float tb = INFINITY;
+#pragma unroll
+      for (int i = 0; i < PPT; ++i)
+        if (!(chosen >> i & 1u)) tb = fminf(tb, bestf[i]);
+      mw = from_order_key_f(__reduce_min_sync(0xffffffffu, order_key_f(tb)));
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const KCand w = warp_min_key(warp_c[tid]);
+      const unsigned who = __ballot_sync(0xffffffffu, warp_c[tid].key == w.key && warp_c[tid].idx == w.idx);
+      const int wslot = warp_slot[__ffs(who) - 1];
+      if (tid < CL) {
+        // this CTA's candidate, coordinates and slot into slot `rank` of CTA `tid`
+        float x = 0.f, y = 0.f, z = 0.f;
+        if (w.idx != INT_MAX) {
+          x = sx[wslot];
+          y = sx[cap + wslot];
+          z = sx[2 * cap + wslot];
+        }
+        const uint32_t ra = mapa_shared(smem_u32(&slots[t & 1][rank][0]), tid);
+        const uint32_t rb = mapa_shared(smem_u32(&bar_slot[t & 1]), tid);
+        st_async_v4(ra, make_uint4((uint32_t)w.key, (uint32_t)(w.key >> 32), (uint32_t)w.idx,
+                                   __float_as_uint(x)),
+                    rb);
+        st_async_v4(ra + 16, make_uint4(__float_as_uint(y), __float_as_uint(z), (uint32_t)wslot, 0u),
+                    rb);
+      }
+      const bool ok = mbar_wait_cluster(&bar_slot[t & 1], (t >> 1) & 1, ctl, &s_abort);
+      KCand x{~0ull, INT_MAX};
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+      if (ok && tid < CL) {
+        a = slots[t & 1][tid][0];
+        b = slots[t & 1][tid][1];
+        x = KCand{((unsigned long long)a.y << 32) | a.x, (int)a.z};
+      }
+      const KCand win = warp_min_key(x);
+      if (ok && tid < CL && x.idx == win.idx) {
+        s_next = CandXYZ{x.key, x.idx, __uint_as_float(a.w), __uint_as_float(b.x), __uint_as_float(b.y)};
+        s_next_rank = tid;
+        s_next_slot = (int)b.z;
+      }
+    }
+    __syncthreads();
+    if (s_abort) break;  // a wait ran out: leave the rounds (the status word says so)
+    c = s_next.idx;
+    c0 = s_next.x;
+    c1 = s_next.y;
+    c2 = s_next.z;
+    c_rank = s_next_rank;
+    c_slot = s_next_slot;
+  }
+#pragma unroll
+  for (int i = 0; i < PPT; ++i) {
+    const int li = i * kFpsThreads + tid;
+    if (so[li] >= 0) owner[so[li]] = own[i];
+  }
+  cluster.sync();  // no CTA leaves while others may still write its slots
+}
+
 // Fallback for n beyond what the cluster holds on chip: the same rounds with
 // the per-point state in global memory.
 __global__ void __launch_bounds__(kFpsThreads, 1)
@@ -481,9 +827,18 @@ int fps_cluster_size() {
 template <int PPT>
 cudaError_t launch_reg(const float* pts, int n, int P, int seed, int* centers, int* owner, int CL,
                        cudaStream_t st, const WaitCtl& ctl) {
-  auto kern = fps_cluster_kernel<PPT>;
-  // x, y, z, and |x|_1 for the fp32 filter (PPT <= 10)
-  const int smem = (PPT <= 10 ? 4 : 3) * PPT * kFpsThreads * (int)sizeof(float);
+  // 8 to 10 points per thread: the culling kernel (x, y, z, |x|_1 and the
+  // original vertex per slot).  With fewer points per thread a round is bound
+  // by the candidate exchange, not by the point updates, and the sort and the
+  // per-warp bound did not pay (60k on 16 CTAs: 1.59 vs 1.47 us per round);
+  // beyond 10 the culling kernel's state does not fit in shared memory.
+  constexpr bool kCull = PPT >= 8 && PPT <= 10;
+  void (*kern)(const float*, int, int, int, int, int*, int*, WaitCtl);
+  if constexpr (kCull) kern = fps_cull_kernel<PPT>;
+  else kern = fps_cluster_kernel<PPT>;
+  // floats per slot: culling kernel 5 (x, y, z, |x|_1, vertex); cluster kernel
+  // 4 with its fp32 filter (PPT <= 10: x, y, z, |x|_1), else 3
+  const int smem = (kCull ? 5 : (PPT <= 10 ? 4 : 3)) * PPT * kFpsThreads * (int)sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (CL > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
