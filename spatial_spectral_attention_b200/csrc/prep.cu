@@ -496,30 +496,68 @@ __global__ void __launch_bounds__(1024) scan2_kernel(const int* __restrict__ a, 
   }
 }
 
+constexpr int kSchedThreads = 1024;
+__device__ __forceinline__ void add_to(int& a, const int& b) { a += b; }
+__device__ __forceinline__ void add_to(ulonglong2& a, const ulonglong2& b) {
+  a.x += b.x;
+  a.y += b.y;
+}
+__device__ __forceinline__ void sub_from(int& a, const int& b) { a -= b; }
+__device__ __forceinline__ void sub_from(ulonglong2& a, const ulonglong2& b) {
+  a.x -= b.x;
+  a.y -= b.y;
+}
+__device__ __forceinline__ int shfl_up_t(int v, int o) { return __shfl_up_sync(0xffffffffu, v, o); }
+__device__ __forceinline__ ulonglong2 shfl_up_t(ulonglong2 v, int o) {
+  return make_ulonglong2(__shfl_up_sync(0xffffffffu, v.x, o), __shfl_up_sync(0xffffffffu, v.y, o));
+}
+// Exclusive prefix of every thread's x over the block of kSchedThreads threads
+// (warp scans by shuffles, then a scan of the 32 warp totals): three block
+// barriers.  *total receives the sum over the block.  part: 32 entries.
+template <typename T>
+__device__ T block_exclusive(T x, T* part, T* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T inc = x;  // inclusive prefix within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T y = shfl_up_t(inc, o);
+    if (lane >= o) add_to(inc, y);
+  }
+  if (lane == 31) part[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    T w = part[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const T y = shfl_up_t(w, o);
+      if (lane >= o) add_to(w, y);
+    }
+    part[lane] = w;
+  }
+  __syncthreads();
+  T r{};  // the warps before this one, then this warp's lanes before this one
+  if (warp > 0) r = part[warp - 1];
+  *total = part[31];
+  __syncthreads();  // part is reused by the next scan
+  add_to(r, inc);
+  sub_from(r, x);
+  return r;
+}
+
 // Block-wide exclusive scan of v[0..m) into base[0..m) by one block of
 // kSchedThreads threads (each thread a contiguous run); returns the total.
-constexpr int kSchedThreads = 1024;
 __device__ int block_scan(const int* v, int m, int* base, int* part) {
   const int tid = threadIdx.x;
   const int per = (m + kSchedThreads - 1) / kSchedThreads;
   const int lo = min(m, tid * per), hi = min(m, lo + per);
   int sacc = 0;
   for (int i = lo; i < hi; ++i) sacc += v[i];
-  part[tid] = sacc;
-  __syncthreads();
-  for (int o = 1; o < kSchedThreads; o <<= 1) {
-    const int x = tid >= o ? part[tid - o] : 0;
-    __syncthreads();
-    part[tid] += x;
-    __syncthreads();
-  }
-  int r = part[tid] - sacc;
+  int total;
+  int r = block_exclusive(sacc, part, &total);
   for (int i = lo; i < hi; ++i) {
     base[i] = r;
     r += v[i];
   }
-  const int total = part[kSchedThreads - 1];
-  __syncthreads();  // part is reused by the next scan
   return total;
 }
 
@@ -549,17 +587,8 @@ __device__ int sorted_tile_scan(const int* pieces, const int* nsegs, int m, int 
     acc.x += f.x;
     acc.y += f.y;
   }
-  part[tid] = acc;
-  __syncthreads();
-  for (int o = 1; o < kSchedThreads; o <<= 1) {
-    const ulonglong2 x = tid >= o ? part[tid - o] : make_ulonglong2(0ull, 0ull);
-    __syncthreads();
-    part[tid].x += x.x;
-    part[tid].y += x.y;
-    __syncthreads();
-  }
-  ulonglong2 r = make_ulonglong2(part[tid].x - acc.x, part[tid].y - acc.y);
-  const ulonglong2 tot = part[kSchedThreads - 1];
+  ulonglong2 tot;
+  ulonglong2 r = block_exclusive(acc, part, &tot);
   int start[8], total = 0;
 #pragma unroll
   for (int b = 0; b < 8; ++b) {
@@ -577,7 +606,6 @@ __device__ int sorted_tile_scan(const int* pieces, const int* nsegs, int m, int 
     r.x += f.x;
     r.y += f.y;
   }
-  __syncthreads();  // part is reused
   return total;
 }
 
@@ -626,8 +654,8 @@ __global__ void __launch_bounds__(kSchedThreads, 1) geo_schedule_kernel(
     int* __restrict__ counts, int* __restrict__ prefix, int* __restrict__ pieces,
     int* __restrict__ nsegs, int* __restrict__ tbase, int* __restrict__ sbase, int tile_cap,
     int seg_cap, unsigned* status) {
-  __shared__ int part[kSchedThreads];
-  __shared__ ulonglong2 part2[kSchedThreads];
+  __shared__ int part[32];          // warp totals of the block scans
+  __shared__ ulonglong2 part2[32];
   __shared__ int s_maxseg, s_tiles;
   if (threadIdx.x == 0) {
     s_maxseg = 0;
@@ -689,20 +717,13 @@ __global__ void __launch_bounds__(kSchedThreads, 1) geo_schedule_kernel(
   const int lo = min(m, (int)threadIdx.x * per), hi = min(m, lo + per);
   int sacc = 0;
   for (int i = lo; i < hi; ++i) sacc += tiles[i].nseg;
-  part[threadIdx.x] = sacc;
-  __syncthreads();
-  for (int o = 1; o < kSchedThreads; o <<= 1) {
-    const int x = (int)threadIdx.x >= o ? part[threadIdx.x - o] : 0;
-    __syncthreads();
-    part[threadIdx.x] += x;
-    __syncthreads();
-  }
-  int r = part[threadIdx.x] - sacc;
+  int total;
+  int r = block_exclusive(sacc, part, &total);
   for (int i = lo; i < hi; ++i) {
     prefix[i] = r;
     r += tiles[i].nseg;
   }
-  if (threadIdx.x == kSchedThreads - 1) prefix[m] = part[kSchedThreads - 1];
+  if (threadIdx.x == 0) prefix[m] = total;
 }
 
 __global__ void inv_count_kernel(const int* __restrict__ topk, int n, int PM, int* __restrict__ cnt) {
