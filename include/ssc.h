@@ -339,10 +339,15 @@ int ssc_geo_coupling_bwd(const void* Q, int ldq, const void* K, int ldk,
 /* the workspace: the patch-major copies of Q, K and V and the tile schedule  */
 /* (the saved state a training step keeps from its forward; the pages have   */
 /* no counterpart).  Same arguments and results as ssc_geo_coupling_bwd.     */
-/* Contract (not checked): ws is the workspace of a completed or earlier-     */
-/* enqueued ssc_geo_coupling_fwd call on the same stream with the same Q, K,  */
-/* V, sizes, dtype and patch tables, and nothing wrote to ws or to those      */
-/* inputs in between; otherwise the results are those of the stale copies.   */
+/* Contract: ws is the workspace of a completed or earlier-enqueued           */
+/* ssc_geo_coupling_fwd call on the same stream with the same Q, K, V, sizes, */
+/* dtype and patch tables, and nothing wrote to ws or to those inputs in      */
+/* between.  The forward leaves a fingerprint of its call (sizes, dtype and   */
+/* the addresses of Q, K, V and the tables) in the workspace and this call    */
+/* compares it on the device: a workspace of another call sets the bad-      */
+/* argument bit of the device status word (ssc_device_status then reports    */
+/* SSC_ERR_INVALID_ARG) and the gradients are undefined.  Changed contents   */
+/* at the same addresses are not detected.                                   */
 /* The backward itself overwrites only the workspace's backward buffers, so   */
 /* it can be called again on the same forward state.                         */
 int ssc_geo_coupling_bwd_reuse(const void* Q, int ldq, const void* K, int ldk,

@@ -137,9 +137,15 @@ int geo_max_tiles(int nN, int PN);
 int geo_max_segs(int nM, int PM, int PN, int R);
 // topk entries outside [0, PM) are skipped and set the bad-index bit.
 // Offsets outside [0, n] or decreasing are clamped and set the bad-index bit.
+// tag: written with tag_value (a fingerprint of the call) when not null.
 cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
                                 const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
-                                int* prefix, int* scratch, unsigned* status, cudaStream_t st);
+                                int* prefix, int* scratch, unsigned* status, cudaStream_t st,
+                                unsigned long long* tag = nullptr,
+                                unsigned long long tag_value = 0);
+// Sets the bad-index bit of *status when *tag differs from expect.
+cudaError_t launch_check_tag(const unsigned long long* tag, unsigned long long expect,
+                             unsigned* status, cudaStream_t st);
 size_t geo_schedule_scratch_ints(int PN);
 // Transposed selection (for the key-stationary fp32 backward): for every
 // source patch q the ascending list of target patches p with q in topk[p].

@@ -653,13 +653,14 @@ __global__ void __launch_bounds__(kSchedThreads, 1) geo_schedule_kernel(
     const int* __restrict__ topk, int R, RowTile* __restrict__ tiles, KeySeg* __restrict__ segs,
     int* __restrict__ counts, int* __restrict__ prefix, int* __restrict__ pieces,
     int* __restrict__ nsegs, int* __restrict__ tbase, int* __restrict__ sbase, int tile_cap,
-    int seg_cap, unsigned* status) {
+    int seg_cap, unsigned long long* tag, unsigned long long tag_value, unsigned* status) {
   __shared__ int part[32];          // warp totals of the block scans
   __shared__ ulonglong2 part2[32];
   __shared__ int s_maxseg, s_tiles;
   if (threadIdx.x == 0) {
     s_maxseg = 0;
     s_tiles = 0;
+    if (tag) *tag = tag_value;
   }
   __syncthreads();
   for (int p = threadIdx.x; p < PN; p += kSchedThreads) {
@@ -992,7 +993,8 @@ size_t geo_schedule_scratch_ints(int PN) { return 4 * (size_t)PN + 2; }
 
 cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM, int PM, int nM,
                                 const int* topk, int R, RowTile* tiles, KeySeg* segs, int* counts,
-                                int* prefix, int* scratch, unsigned* status, cudaStream_t st) {
+                                int* prefix, int* scratch, unsigned* status, cudaStream_t st,
+                                unsigned long long* tag, unsigned long long tag_value) {
   int* pieces = scratch;
   int* nsegs = scratch + PN;
   int* tbase = scratch + 2 * PN;
@@ -1000,7 +1002,21 @@ cudaError_t launch_geo_schedule(const int* offN, int PN, int nN, const int* offM
   const int tile_cap = geo_max_tiles(nN, PN), seg_cap = geo_max_segs(nM, PM, PN, R);
   geo_schedule_kernel<<<1, kSchedThreads, 0, st>>>(offN, PN, nN, offM, PM, nM, topk, R, tiles, segs,
                                                    counts, prefix, pieces, nsegs, tbase, sbase,
-                                                   tile_cap, seg_cap, status);
+                                                   tile_cap, seg_cap, tag, tag_value, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+namespace {
+__global__ void check_tag_kernel(const unsigned long long* tag, unsigned long long expect,
+                                 unsigned* status) {
+  if (*tag != expect) atomicOr(status, kStatusBadIndex);
+}
+}  // namespace
+
+cudaError_t launch_check_tag(const unsigned long long* tag, unsigned long long expect,
+                             unsigned* status, cudaStream_t st) {
+  check_tag_kernel<<<1, 1, 0, st>>>(tag, expect, status);
   count_launch();
   return cudaGetLastError();
 }

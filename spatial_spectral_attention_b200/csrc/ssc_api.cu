@@ -134,6 +134,7 @@ struct GeoWs {
   int* inv_off;
   int* inv_p;
   int* inv_scratch;
+  unsigned long long* tag;  // fingerprint of the forward that filled the workspace
   int ldq, ldk, ldv, ldg;
 };
 size_t geo_ws(void* base, int nN, int nM, int d, int k, int PN, int PM, int R, int dtype, GeoWs* w) {
@@ -160,8 +161,31 @@ size_t geo_ws(void* base, int nN, int nM, int d, int k, int PN, int PM, int R, i
   x.inv_off = c.take<int>(PM + 1);
   x.inv_p = c.take<int>((size_t)PN * R);
   x.inv_scratch = c.take<int>(invert_topk_scratch_ints(PM));
+  x.tag = c.take<unsigned long long>(1);
   if (w) *w = x;
   return c.used + 256;
+}
+
+// Fingerprint of a Geo call: sizes, dtype and the addresses of its operands
+// and tables (64-bit FNV-1a over the values).
+unsigned long long geo_fingerprint(const void* Q, const void* K, const void* V, int nN, int nM,
+                                   int d, int k, int dtype, const int* offN, const int* memN,
+                                   int PN, const int* offM, const int* memM, int PM,
+                                   const int* topk, int R) {
+  const unsigned long long v[] = {
+      (unsigned long long)reinterpret_cast<uintptr_t>(Q), (unsigned long long)reinterpret_cast<uintptr_t>(K),
+      (unsigned long long)reinterpret_cast<uintptr_t>(V), (unsigned long long)reinterpret_cast<uintptr_t>(offN),
+      (unsigned long long)reinterpret_cast<uintptr_t>(memN), (unsigned long long)reinterpret_cast<uintptr_t>(offM),
+      (unsigned long long)reinterpret_cast<uintptr_t>(memM), (unsigned long long)reinterpret_cast<uintptr_t>(topk),
+      (unsigned long long)nN, (unsigned long long)nM, (unsigned long long)d, (unsigned long long)k,
+      (unsigned long long)dtype, (unsigned long long)PN, (unsigned long long)PM, (unsigned long long)R};
+  unsigned long long h = 1469598103934665603ull;
+  for (unsigned long long x : v)
+    for (int b = 0; b < 8; ++b) {
+      h ^= (x >> (8 * b)) & 0xffull;
+      h *= 1099511628211ull;
+    }
+  return h;
 }
 
 bool ws_ok(void* ws, size_t have, size_t need) {
@@ -536,7 +560,9 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
       return SSC_ERR_CUDA;
   }
   e = launch_geo_schedule(offN, PN, nN, offM, PM, nM, topk, R, w.tiles, w.segs, w.counts,
-                          w.prefix, w.sched_scratch, ctl.status, st);
+                          w.prefix, w.sched_scratch, ctl.status, st, w.tag,
+                          geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
+                                          topk, R));
   return cuda_status(e);
 }
 
@@ -577,6 +603,12 @@ int geo_bwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, i
   if (!reuse && (rc = geo_setup(Q, ldq, K, ldk, V, ldv, nN, nM, d, k, dtype, offN, memN, PN, offM,
                                 memM, PM, topk, R, w, st, ctl)))
     return rc;
+  // the forward that filled the workspace must be this call's
+  if (reuse && launch_check_tag(w.tag,
+                                geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM,
+                                                memM, PM, topk, R),
+                                ctl.status, st) != cudaSuccess)
+    return SSC_ERR_CUDA;
   cudaError_t e;
   if (dtype == SSC_F32) {
     e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, nullptr, 0,

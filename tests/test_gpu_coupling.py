@@ -201,6 +201,13 @@ def test_geo_backward_reusing_the_forward_workspace(dtype):
             np.testing.assert_allclose(a.cpu().numpy(), other.cpu().numpy(), rtol=1e-4, atol=1e-6)
     with pytest.raises(ValueError):
         api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, *tabs, reuse_forward=True)
+    # the workspace holds the fingerprint of the forward that filled it: a reuse
+    # call with other operands (here another copy of Q) is reported on the device
+    api.ssc_device_status(clear=True)
+    Q2 = Q.clone()
+    api.ssc_geo_coupling_bwd(Q2, K, V, O, lse, dO, pair.scale, *tabs, workspace=ws,
+                             reuse_forward=True)
+    assert api.ssc_device_status(clear=True) == 1  # SSC_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("name", ["geo_60k", "geo_160k_warped"])
