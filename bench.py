@@ -160,11 +160,38 @@ def barrier(ws):
 GEO_SWEEP_N = (20000, 40000, 60000, 100000, 160000)
 
 
+def step_graph(step, torch, dev):
+    """The launches of one step captured once into a CUDA graph (after the
+    step has run eagerly, so every lazily made resource exists); a replay runs
+    every launch of the step again on the same device-resident inputs."""
+    gr = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(dev)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(gr, stream=cs):
+        step()
+    torch.cuda.synchronize()
+    return gr
+
+
+def timed_steps(run, flush, stream, torch, reps):
+    """Mean ms of `reps` runs, each bracketed by CUDA events on `stream`, with
+    L2 flushed (untimed) before each."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        run()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
 def run_geo_sweep(api, synth, torch, dev, need_dv, fpp, bpp):
     """Geo step (scores/top-R + fwd + bwd) against n with P = n/125 and R = 8:
     ms per step and peak device memory per size (160k is the warped,
     non-isometric pair).  Each size: patch tables once, 2 warm-up and 3 timed
-    steps, L2 flushed before each timed step."""
+    steps launched one by one, then 3 timed replays of the step as one CUDA
+    graph; L2 flushed before each timed step."""
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     bf = lambda a: torch.tensor(a).to(torch.bfloat16).to(dev)
@@ -189,17 +216,14 @@ def run_geo_sweep(api, synth, torch, dev, need_dv, fpp, bpp):
 
         for _ in range(2):
             step()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
-        for e in evs:
-            flush.zero_()
-            e[0].record(stream)
-            step()
-            e[1].record(stream)
-        torch.cuda.synchronize()
-        ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        eager_ms = timed_steps(step, flush, stream, torch, 3)
         peak = (torch.cuda.max_memory_allocated(dev) - flush.numel() - base) / 2**30
+        gr = step_graph(step, torch, dev)
+        ms = timed_steps(gr.replay, flush, stream, torch, 3)
+        del gr
         U = float(np.mean(np.diff(offM.cpu().numpy()))) * gp.R
         out.append({"n": n, "P": gp.P, "ms_per_step": round(ms, 4),
+                    "eager_ms_per_step": round(eager_ms, 4),
                     "tflops": round(float(n) * U * (fpp + bpp) / (ms * 1e-3) / 1e12, 2),
                     "peak_gib": round(peak, 3)})
         del Q, K, V, dO, offN, memN, offM, memM, gws
@@ -609,6 +633,28 @@ def run_ours(args, ws, rank, local):
             ("gather", api.PROF_GATHER))}
         geo_kern = {nm: (ms / gsteps, n // gsteps) for nm, (ms, n) in geo_kern.items()}
         geo_kern["_topk"] = topk_last
+        # the step on its own (no dense step between, so the clocks are not those
+        # of the dense step's power draw): K steps launched one by one through
+        # the API and K replays of the same step captured as one CUDA graph,
+        # alternating, L2 flushed before each
+        gr = step_graph(geo_step, torch, dev)
+        for _ in range(args.warmup):
+            geo_step()
+            gr.replay()
+        pairs_ev = []
+        for _ in range(args.steps):
+            for fn in (geo_step, gr.replay):
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                flush.zero_()
+                e[0].record(stream)
+                fn()
+                e[1].record(stream)
+                pairs_ev.append(e)
+        torch.cuda.synchronize()
+        tt = [a.elapsed_time(b) for a, b in pairs_ev]
+        geo_alone_ms = max_over_ranks(float(np.mean(tt[0::2])), ws)
+        geo_graph_ms = max_over_ranks(float(np.mean(tt[1::2])), ws)
+        del gr
     fps_timing = run_fps_timing(api, synth, torch, dev) if (geo and rank == 0) else None
 
     pk = peaks()
@@ -717,17 +763,23 @@ def run_ours(args, ws, rank, local):
                                 "per launch (L2 re-reads not counted)",
             "peak_source": pk["source"] + " (MEASURED_PEAKS.json: bf16_tflops, hbm_gbs)",
         }
-        res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_ms, 4),
-                      "tflops": round(gflops / (geo_ms * 1e-3) / 1e12, 2),
-                      "frac_of_peak": round(gflops / (geo_ms * 1e-3) / 1e12 / pk["tflops"], 4),
+        res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_graph_ms, 4),
+                      "eager_ms_per_step": round(geo_alone_ms, 4),
+                      "eager_ms_per_step_beside_dense": round(geo_ms, 4),
+                      "tflops": round(gflops / (geo_graph_ms * 1e-3) / 1e12, 2),
+                      "frac_of_peak": round(gflops / (geo_graph_ms * 1e-3) / 1e12 / pk["tflops"], 4),
                       "support_pairs": pairs, "tile_pairs": pairs_exec,
                       "tile_fill": round(pairs / pairs_exec, 4),
                       "support_per_row": round(pairs / gpair.n, 1),
                       "roofline": geo_roof,
                       "fps": fps_timing,
                       "note": "step = scores/top-R + fwd + bwd (the backward reuses the forward's "
-                              "patch-major operands and schedule from the workspace); FPS per "
-                              "shape, outside the step, timed warm on resident points"}
+                              "patch-major operands and schedule from the workspace); "
+                              "ms_per_step: the step's launches replayed as one CUDA graph, "
+                              "eager_ms_per_step: launched one by one through the API (the two "
+                              "alternating, Geo steps only); eager_ms_per_step_beside_dense: in "
+                              "the main timed region, each after a dense step; FPS per shape, "
+                              "outside the step, timed warm on resident points"}
     return res
 
 

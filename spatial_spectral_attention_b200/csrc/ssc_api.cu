@@ -1,7 +1,9 @@
 // ssc_api.cu -- the C ABI of libssc (declared in include/ssc.h): argument
 // checks, workspace carving and the launch sequence of every call.  No call
 // allocates device memory and none synchronises the host (except
-// ssc_device_status, whose job is to read the status word back).
+// ssc_device_status, whose job is to read the status word back).  Launches
+// that are independent of the ones before them go to a per-thread side stream
+// and are joined back into the caller's stream before their results are used.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -37,6 +39,60 @@ WaitCtl make_ctl() {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SSC_OK : SSC_ERR_CUDA; }
+
+// A side stream for launches that do not depend on the work just before them
+// on the caller's stream (the Geo patch-major gather runs beside the tile
+// schedule, the backward's accumulator zeroing beside its row prep).  One per
+// host thread and device, with its two events, made on the thread's first call
+// outside stream capture; when there is none (or the caller's stream is the
+// side stream) the work stays on the caller's stream, in the same order.
+struct Side {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+Side* side_for(cudaStream_t st) {
+  thread_local Side sides[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  Side& s = sides[dev];
+  if (!s.st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+      return nullptr;
+    Side n;
+    if (cudaStreamCreateWithFlags(&n.st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming) != cudaSuccess) {
+      if (n.fork) cudaEventDestroy(n.fork);
+      cudaStreamDestroy(n.st);
+      return nullptr;
+    }
+    s = n;
+  }
+  return s.st == st ? nullptr : &s;
+}
+
+// Starts a fork: the side stream waits for everything enqueued on st so far.
+// Returns the stream that the independent launches go to (st itself when
+// there is no side stream) and sets *side (nullptr when there is none).
+cudaError_t fork_begin(cudaStream_t st, Side** side, cudaStream_t* to) {
+  *side = side_for(st);
+  *to = st;
+  if (!*side) return cudaSuccess;
+  cudaError_t e = cudaEventRecord((*side)->fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent((*side)->st, (*side)->fork, 0);
+  if (e == cudaSuccess) *to = (*side)->st;
+  return e;
+}
+
+// Ends a fork: st waits for the side stream's launches since fork_begin.
+cudaError_t fork_end(cudaStream_t st, Side* side) {
+  if (!side) return cudaSuccess;
+  cudaError_t e = cudaEventRecord(side->join, side->st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+  return e;
+}
 
 }  // namespace
 
@@ -411,15 +467,22 @@ int ssc_dense_coupling_bwd(const void* Q, int ldq, const void* K, int ldk, const
     return cuda_status(launch_simt_bwd_dkdv(a, g, dO, lddo, lse, w.D, dK, lddk, dV, lddv, st));
   }
   const int kp = (int)kp_of(k);
-  e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
-                      nullptr, ctl.status, st);
-  if (e != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  const __nv_bfloat16* Vt;
-  int ldvt;
-  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  // the zeroing of the accumulators and the V re-pack run on the side stream
+  // beside the row prep (neither touches what the other reads or writes)
+  Side* side;
+  cudaStream_t zs;
+  if ((e = fork_begin(st, &side, &zs)) != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt = nullptr;
+  int ldvt = 0;
+  e = zero_matrix(dK, lddk, nM, d, zs);
+  if (e == cudaSuccess) e = zero_matrix(dQ, lddq, nN, d, zs);
+  if (e == cudaSuccess && dV) e = zero_matrix(dV, lddv, nM, k, zs);
+  if (e == cudaSuccess) e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, zs, ctl.status);
+  if (e == cudaSuccess)
+    e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
+                        nullptr, ctl.status, st);
+  const cudaError_t j = fork_end(st, side);
+  if (e != cudaSuccess || j != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Vt, ldq, ldk,
            ldvt, nN, nM, d, k, scale, w.tiles, w.segs, nullptr, dense_num_tiles(nN), w.prefix, nullptr,
            nullptr};
@@ -505,15 +568,22 @@ int ssc_dense_coupling_bwd_deterministic(const void* Q, int ldq, const void* K, 
   cudaError_t e = launch_dense_schedule(nN, nM, w.tiles, w.segs, w.prefix, st);
   if (e != cudaSuccess) return SSC_ERR_CUDA;
   const int kp = (int)kp_of(k);
-  e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
-                      nullptr, ctl.status, st);
-  if (e != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dK, lddk, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  const __nv_bfloat16* Vt;
-  int ldvt;
-  if ((e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, st, ctl.status)) != cudaSuccess) return SSC_ERR_CUDA;
+  // the zeroing of the accumulators and the V re-pack run on the side stream
+  // beside the row prep (neither touches what the other reads or writes)
+  Side* side;
+  cudaStream_t zs;
+  if ((e = fork_begin(st, &side, &zs)) != cudaSuccess) return SSC_ERR_CUDA;
+  const __nv_bfloat16* Vt = nullptr;
+  int ldvt = 0;
+  e = zero_matrix(dK, lddk, nM, d, zs);
+  if (e == cudaSuccess) e = zero_matrix(dQ, lddq, nN, d, zs);
+  if (e == cudaSuccess && dV) e = zero_matrix(dV, lddv, nM, k, zs);
+  if (e == cudaSuccess) e = dense_v(V, ldv, nM, k, w, &Vt, &ldvt, zs, ctl.status);
+  if (e == cudaSuccess)
+    e = launch_bwd_prep(dO, lddo, O, ldo, lse, nullptr, nN, nN, k, w.dOb, kp, nullptr, 0, w.D,
+                        nullptr, ctl.status, st);
+  const cudaError_t j = fork_end(st, side);
+  if (e != cudaSuccess || j != cudaSuccess) return SSC_ERR_CUDA;
   return cuda_status(launch_tc_bwd_deterministic(
       static_cast<const __nv_bfloat16*>(Q), ldq, static_cast<const __nv_bfloat16*>(K), ldk, Vt, ldvt,
       w.dOb, kp, lse, w.D, w.tiles, w.segs, w.prefix, nN, nM, d, k, scale, dQ, lddq, dK, lddk, dV,
@@ -534,7 +604,11 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
               int d, int k, int dtype, const int* offN, const int* memN, int PN, const int* offM,
               const int* memM, int PM, const int* topk, int R, const GeoWs& w, cudaStream_t st,
               const WaitCtl& ctl) {
-  cudaError_t e;
+  // the gather reads no top-R output: it runs on the side stream beside the schedule
+  Side* side;
+  cudaStream_t gs;
+  cudaError_t e = fork_begin(st, &side, &gs);
+  if (e != cudaSuccess) return SSC_ERR_CUDA;
   if (dtype == SSC_BF16) {
     // Q, K and V into patch-major order in one launch
     const __nv_bfloat16* in[3] = {static_cast<const __nv_bfloat16*>(Q),
@@ -547,23 +621,23 @@ int geo_setup(const void* Q, int ldq, const void* K, int ldk, const void* V, int
     __nv_bfloat16* out[3] = {static_cast<__nv_bfloat16*>(w.Qp), static_cast<__nv_bfloat16*>(w.Kp),
                              static_cast<__nv_bfloat16*>(w.Vp)};
     const int out_ld[3] = {w.ldq, w.ldk, w.ldv};
-    if ((e = launch_gather3_bf16(in, in_ld, map, rows, rows, cols, out, out_ld, ctl.status, st)) !=
-        cudaSuccess)
-      return SSC_ERR_CUDA;
+    e = launch_gather3_bf16(in, in_ld, map, rows, rows, cols, out, out_ld, ctl.status, gs);
   } else {
     if ((e = launch_gather_rows_f32(static_cast<const float*>(Q), ldq, memN, nN, nN, d,
-                                    static_cast<float*>(w.Qp), w.ldq, ctl.status, st)) != cudaSuccess ||
+                                    static_cast<float*>(w.Qp), w.ldq, ctl.status, gs)) == cudaSuccess &&
         (e = launch_gather_rows_f32(static_cast<const float*>(K), ldk, memM, nM, nM, d,
-                                    static_cast<float*>(w.Kp), w.ldk, ctl.status, st)) != cudaSuccess ||
-        (e = launch_gather_rows_f32(static_cast<const float*>(V), ldv, memM, nM, nM, k,
-                                    static_cast<float*>(w.Vp), w.ldv, ctl.status, st)) != cudaSuccess)
-      return SSC_ERR_CUDA;
+                                    static_cast<float*>(w.Kp), w.ldk, ctl.status, gs)) == cudaSuccess)
+      e = launch_gather_rows_f32(static_cast<const float*>(V), ldv, memM, nM, nM, k,
+                                 static_cast<float*>(w.Vp), w.ldv, ctl.status, gs);
   }
-  e = launch_geo_schedule(offN, PN, nN, offM, PM, nM, topk, R, w.tiles, w.segs, w.counts,
-                          w.prefix, w.sched_scratch, ctl.status, st, w.tag,
-                          geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM,
-                                          topk, R));
-  return cuda_status(e);
+  if (e == cudaSuccess)
+    e = launch_geo_schedule(offN, PN, nN, offM, PM, nM, topk, R, w.tiles, w.segs, w.counts,
+                            w.prefix, w.sched_scratch, ctl.status, st, w.tag,
+                            geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM,
+                                            memM, PM, topk, R));
+  // joined on every path, so that a captured stream is never left forked
+  const cudaError_t j = fork_end(st, side);
+  return cuda_status(e != cudaSuccess ? e : j);
 }
 
 }  // namespace
@@ -604,13 +678,12 @@ int geo_bwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, i
                                 memM, PM, topk, R, w, st, ctl)))
     return rc;
   // the forward that filled the workspace must be this call's
-  if (reuse && launch_check_tag(w.tag,
-                                geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM,
-                                                memM, PM, topk, R),
-                                ctl.status, st) != cudaSuccess)
-    return SSC_ERR_CUDA;
+  const unsigned long long fp =
+      reuse ? geo_fingerprint(Q, K, V, nN, nM, d, k, dtype, offN, memN, PN, offM, memM, PM, topk, R)
+            : 0;
   cudaError_t e;
   if (dtype == SSC_F32) {
+    if (reuse && launch_check_tag(w.tag, fp, ctl.status, st) != cudaSuccess) return SSC_ERR_CUDA;
     e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, nullptr, 0,
                         static_cast<float*>(w.dOp), w.ldg, w.D, w.lsep, ctl.status, st);
     if (e != cudaSuccess) return SSC_ERR_CUDA;
@@ -627,16 +700,24 @@ int geo_bwd_run(const void* Q, int ldq, const void* K, int ldk, const void* V, i
     return cuda_status(launch_simt_bwd_dkdv(a, g, static_cast<const float*>(w.dOp), w.ldg, w.lsep,
                                             w.D, dK, lddk, dV, lddv, st));
   }
-  e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, static_cast<__nv_bfloat16*>(w.dOp),
-                      w.ldg, nullptr, 0, w.D, w.lsep, ctl.status, st);
-  if (e != cudaSuccess) return SSC_ERR_CUDA;
   // dK is reduced in the patch-major key order (contiguous key rows, so TMA
   // reductions apply) and scattered to vertex order afterwards: memM lists
   // every source vertex once, so the scatter writes each row of dK once (with
-  // inconsistent tables the results are unspecified, as the header states)
-  if ((e = zero_matrix(w.dKg, d, nM, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if ((e = zero_matrix(dQ, lddq, nN, d, st)) != cudaSuccess) return SSC_ERR_CUDA;
-  if (dV && (e = zero_matrix(dV, lddv, nM, k, st)) != cudaSuccess) return SSC_ERR_CUDA;
+  // inconsistent tables the results are unspecified, as the header states).
+  // The fingerprint check and the zeroing of the accumulators touch nothing
+  // that the row prep reads or writes: they run on the side stream beside it.
+  Side* side;
+  cudaStream_t zs;
+  if ((e = fork_begin(st, &side, &zs)) != cudaSuccess) return SSC_ERR_CUDA;
+  if (reuse) e = launch_check_tag(w.tag, fp, ctl.status, zs);
+  if (e == cudaSuccess) e = zero_matrix(w.dKg, d, nM, d, zs);
+  if (e == cudaSuccess) e = zero_matrix(dQ, lddq, nN, d, zs);
+  if (e == cudaSuccess && dV) e = zero_matrix(dV, lddv, nM, k, zs);
+  if (e == cudaSuccess)
+    e = launch_bwd_prep(dO, lddo, O, ldo, lse, memN, nN, nN, k, static_cast<__nv_bfloat16*>(w.dOp),
+                        w.ldg, nullptr, 0, w.D, w.lsep, ctl.status, st);
+  const cudaError_t j = fork_end(st, side);
+  if (e != cudaSuccess || j != cudaSuccess) return SSC_ERR_CUDA;
   TcArgs a{static_cast<const __nv_bfloat16*>(w.Qp), static_cast<const __nv_bfloat16*>(w.Kp),
            static_cast<const __nv_bfloat16*>(w.Vp), w.ldq, w.ldk, w.ldv, nN, nM, d, k, scale,
            w.tiles, w.segs, w.counts, 0, w.prefix, memN, memM};

@@ -232,6 +232,58 @@ def test_geo_end_to_end_from_gpu_tables():
     assert_close(lse, lse64, TOL_BF16, "lse")
 
 
+def test_geo_step_captured_in_a_cuda_graph():
+    # scores/top-R + forward + reusing backward, captured once and replayed: the
+    # side-stream launches (gather beside the schedule, zeroing beside the row
+    # prep) join the capture; a replay after new values are copied into the
+    # same input buffers matches the oracle on those values
+    pair = synth.make_workload("geo_60k", n=6000)
+    P, R = 48, 8
+    (Q, K, V, dO), _ = _inputs(pair.F_N, pair.F_M, pair.Phi_M, pair.dO, "bf16")
+    t0 = _geo_tables(pair, P, R, "bf16")
+    offN, memN, offM, memM = [as_i32(t0[x]) for x in ("off_N", "mem_N", "off_M", "mem_M")]
+    nb = api.lib().ssc_geo_coupling_workspace_size(pair.n, pair.n, pair.d, pair.k, P, P, R, 0)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+
+    def step():
+        topk = api.ssc_patch_scores_topk(Q, K, offN, memN, offM, memM, R)
+        O, lse = api.ssc_geo_coupling_fwd(Q, K, V, pair.scale, offN, memN, offM, memM, topk,
+                                          workspace=ws)
+        dQ, dK, _ = api.ssc_geo_coupling_bwd(Q, K, V, O, lse, dO, pair.scale, offN, memN, offM,
+                                             memM, topk, workspace=ws, reuse_forward=True)
+        return topk, O, lse, dQ, dK
+
+    eager = step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cs):
+        out = step()
+    g.replay()
+    _status_ok()
+    np.testing.assert_array_equal(out[0].cpu().numpy(), eager[0].cpu().numpy())
+    for a, b in zip(out[1:3], eager[1:3]):
+        np.testing.assert_array_equal(a.cpu().numpy(), b.cpu().numpy())
+    for a, b in zip(out[3:], eager[3:]):
+        np.testing.assert_allclose(a.cpu().numpy(), b.cpu().numpy(), rtol=1e-4, atol=1e-6)
+    # new operand values in the captured buffers (another seed of the same recipe)
+    other = synth.make_workload("geo_60k", n=6000, seed=11)
+    (Q2, K2, V2, dO2), (Q64, K64, V64, dO64) = _inputs(other.F_N, other.F_M, other.Phi_M, other.dO,
+                                                       "bf16")
+    for dst, src in ((Q, Q2), (K, K2), (V, V2), (dO, dO2)):
+        dst.copy_(src)
+    g.replay()
+    _status_ok()
+    t = oracle.patch_pipeline(pair.pts_N, pair.pts_M, Q64, K64, P, P, R)
+    np.testing.assert_array_equal(out[0].cpu().numpy(), t["topk"])
+    ref = oracle.geo_bwd(Q64, K64, V64, dO64, pair.scale, t["off_N"], t["mem_N"], t["off_M"],
+                         t["mem_M"], t["topk"])
+    for a, nm in zip(out[1:], ("O", "lse", "dQ", "dK")):
+        assert_close(a, ref[nm], TOL_BF16, nm)
+    del g
+
+
 def test_constant_eigenfunction_reproduced():
     # rows of Pi sum to one, so the constant column Y_00 of Phi comes back exactly
     # up to the bf16 rounding of P (relative 2^-8 at worst per element)
