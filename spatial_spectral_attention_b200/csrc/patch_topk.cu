@@ -197,35 +197,51 @@ __global__ void __launch_bounds__(128) pool_rows_kernel(const PoolSet set_a, con
   if (c1 < d) mu[(size_t)p * d + c1] = __ddiv_rn(s1, cnt);
 }
 
-// Warp-per-patch pooling for d = 32 CPL (CPL = 2 or 4 channels per lane):
-// each lane sums its CPL channels as CPL independent chains, strictly in
-// member order (bit-identical to pool_kernel).  The warp stages the member
-// rows of its patch in shared memory with cp.async, kWarpRows rows per chunk
-// and two chunks in flight; member indices go through shared memory too.
-// Four warps (four patches) per block, both shapes in one launch.
+// fp32 -> fp64 from the bits, on the integer pipe (exact, like the
+// conversion instruction): a normal number keeps its sign and mantissa and
+// moves its exponent from the 127 to the 1023 bias; zeros, subnormals,
+// infinities and NaNs take the conversion instruction.
+__device__ __forceinline__ double widen_f32_bits(uint32_t u) {
+  const uint32_t e = (u >> 23) & 0xffu;
+  if (e - 1u < 254u)
+    return __longlong_as_double((long long)(((unsigned long long)(u >> 31) << 63) |
+                                            ((unsigned long long)(e + 896u) << 52) |
+                                            ((unsigned long long)(u & 0x7fffffu) << 29)));
+  return (double)__uint_as_float(u);
+}
+
+// Warp-sliced pooling for d = 32 CPL WPP: the WPP warps of a patch each take a
+// slice of 32 CPL channels, and each lane sums its CPL channels as CPL
+// independent chains, strictly in member order (bit-identical to
+// pool_kernel).  A warp stages its slice of the member rows in shared memory
+// with cp.async, kWarpRows rows per chunk and two chunks in flight; member
+// indices go through shared memory too.  Four warps per block, both shapes in
+// one launch.
 constexpr int kWarpRows = 32;
-template <bool F32, int CPL>
+template <bool F32, int CPL, int WPP>
 __global__ void __launch_bounds__(128) pool_warp_kernel(const PoolSet set_a, const PoolSet set_b,
                                                         unsigned* status) {
   constexpr int kEsz = F32 ? 4 : 2;
-  constexpr int kRowB = 32 * CPL * kEsz;    // bytes per descriptor row (d = 32 CPL)
-  constexpr int kPieces = kRowB / 16;       // 16-byte pieces per row
+  constexpr int kRowB = 32 * CPL * kEsz;    // bytes of this warp's slice of a row
+  constexpr int kPieces = kRowB / 16;       // 16-byte pieces per slice
   constexpr int kChunkB = kWarpRows * kRowB;
+  static_assert(kRowB % 16 == 0, "a slice is whole 16-byte pieces");
   extern __shared__ __align__(16) uint8_t s_pool[];  // [4 warps][2][kWarpRows][kRowB]
   __shared__ int s_idx[4][2][kWarpRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gp = blockIdx.x * 4 + warp;
+  const int gw = blockIdx.x * 4 + warp;
+  const int gp = gw / WPP, slice = gw % WPP;
   if (gp >= set_a.P + set_b.P) return;  // warp-uniform; no block barrier below
   const bool second = gp >= set_a.P;
   const PoolSet& S = second ? set_b : set_a;
   const int p = second ? gp - set_a.P : gp;
   const int n = S.n;
   const int* __restrict__ mem = S.mem;
-  const uint8_t* Fb = static_cast<const uint8_t*>(S.F);
+  const uint8_t* Fb = static_cast<const uint8_t*>(S.F) + slice * kRowB;
   const size_t ldb = (size_t)S.ld * kEsz;
   int b = S.off[p], e = S.off[p + 1];
   if (b < 0 || e <= b || e > n) {
-    if (lane == 0) atomicOr(status, kStatusBadIndex);
+    if (lane == 0 && slice == 0) atomicOr(status, kStatusBadIndex);
     b = min(max(b, 0), n);
     e = min(max(e, b), n);
   }
@@ -253,7 +269,7 @@ __global__ void __launch_bounds__(128) pool_warp_kernel(const PoolSet set_a, con
         v = mem[r0 + lane];
       }
       if (v < 0 || v >= n) {
-        atomicOr(status, kStatusBadIndex);
+        if (slice == 0) atomicOr(status, kStatusBadIndex);
         v = -1;
       }
     }
@@ -290,36 +306,28 @@ __global__ void __launch_bounds__(128) pool_warp_kernel(const PoolSet set_a, con
       for (int u = 0; u < 8; ++u) {
         const int r = r0 + u;
         ok[u] = r < nr && s_idx[warp][k & 1][r] >= 0;  // the same for every lane
+        // the element bits as fp32 (bf16 -> fp32 is exact: the bf16 bits are
+        // the high half of the float), widened to fp64 exactly
+        uint32_t h[CPL];
         if constexpr (F32) {
-          float v[CPL];
-          if (ok[u]) {
-            if constexpr (CPL == 4) {
-              const float4 t = *reinterpret_cast<const float4*>(buf + r * kRowB);
-              v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-            } else {
-              const float2 t = *reinterpret_cast<const float2*>(buf + r * kRowB);
-              v[0] = t.x; v[1] = t.y;
-            }
+          if constexpr (CPL == 1) {
+            h[0] = ok[u] ? *reinterpret_cast<const uint32_t*>(buf + r * kRowB) : 0u;
+          } else {
+            const uint2 t = ok[u] ? *reinterpret_cast<const uint2*>(buf + r * kRowB) : make_uint2(0u, 0u);
+            h[0] = t.x;
+            h[1] = t.y;
           }
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) x[u][c] = ok[u] ? (double)v[c] : 0.0;
         } else {
-          uint32_t w[CPL / 2];
-          if (ok[u]) {
-            if constexpr (CPL == 4) {
-              const uint2 t = *reinterpret_cast<const uint2*>(buf + r * kRowB);
-              w[0] = t.x; w[1] = t.y;
-            } else {
-              w[0] = *reinterpret_cast<const uint32_t*>(buf + r * kRowB);
-            }
-          }
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) {
-            // bf16 -> fp32 is exact: the bf16 bits are the high half of the float
-            const uint32_t h = ok[u] ? ((c & 1) ? (w[c >> 1] & 0xffff0000u) : (w[c >> 1] << 16)) : 0u;
-            x[u][c] = (double)__uint_as_float(h);
+          if constexpr (CPL == 1) {
+            h[0] = ok[u] ? (uint32_t)*reinterpret_cast<const uint16_t*>(buf + r * kRowB) << 16 : 0u;
+          } else {
+            const uint32_t w = ok[u] ? *reinterpret_cast<const uint32_t*>(buf + r * kRowB) : 0u;
+            h[0] = w << 16;
+            h[1] = w & 0xffff0000u;
           }
         }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) x[u][c] = widen_f32_bits(h[c]);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -332,7 +340,8 @@ __global__ void __launch_bounds__(128) pool_warp_kernel(const PoolSet set_a, con
   }
   const double cnt = (double)max(e - b, 1);
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) S.mu[(size_t)p * 32 * CPL + lane * CPL + c] = __ddiv_rn(acc[c], cnt);
+  for (int c = 0; c < CPL; ++c)
+    S.mu[(size_t)p * 32 * CPL * WPP + slice * 32 * CPL + lane * CPL + c] = __ddiv_rn(acc[c], cnt);
 }
 
 constexpr int kST = 32;  // score tile (target x source patches)
@@ -486,13 +495,17 @@ cudaError_t launch_scores_topk(const void* FN, int ldn, int nN, const void* FM, 
     // one warp per patch, both shapes in one launch
     const PoolSet a{FN, offN, memN, muN, ldn, batch * nN, batch * PN};
     const PoolSet b{FM, offM, memM, muM, ldm, batch * nM, batch * PM};
-    const int smem = 4 * 2 * kWarpRows * d * esz;
-    auto kern = dtype == 1 ? (d == 128 ? pool_warp_kernel<true, 4> : pool_warp_kernel<true, 2>)
-                           : (d == 128 ? pool_warp_kernel<false, 4> : pool_warp_kernel<false, 2>);
+    // bf16: one channel per lane (d / 32 warps per patch); fp32: two
+    // (d / 64 warps per patch), slices of 64 and 256 bytes of each row
+    const int cpl = dtype == 1 ? 2 : 1;
+    const int wpp = d / (32 * cpl);
+    const int smem = 4 * 2 * kWarpRows * 32 * cpl * esz;
+    auto kern = dtype == 1 ? (d == 128 ? pool_warp_kernel<true, 2, 2> : pool_warp_kernel<true, 2, 1>)
+                           : (d == 128 ? pool_warp_kernel<false, 1, 4> : pool_warp_kernel<false, 1, 2>);
     if ((pe = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return pe;
-    const int total = batch * (PN + PM);
+    const int total = batch * (PN + PM) * wpp;
     prof_launch_begin(st);
     kern<<<(total + 3) / 4, 128, smem, st>>>(a, b, status);
     prof_launch_end(st, SSC_PROF_POOL);
