@@ -45,8 +45,8 @@ def pair_flops(d, k, need_dv):
 # capture of this bench's own launch at n = 60k (dram__bytes_read.sum +
 # dram__bytes_write.sum, a 1-pass metric set).  It stands only while the
 # kernel's source text is the one that was captured.
-DQK_TRAFFIC = {"kernel_sha256_16": "198cc8e84387f42a", "n": 60000, "d": 128, "k": 196,
-               "read_bytes": 184.19e6, "write_bytes": 108.57e6}
+DQK_TRAFFIC = {"kernel_sha256_16": "d3a006df033c44d3", "n": 60000, "d": 128, "k": 196,
+               "read_bytes": 179.66e6, "write_bytes": 70.50e6}
 
 
 def dqk_kernel_hash():
@@ -54,8 +54,8 @@ def dqk_kernel_hash():
     path = os.path.join(ROOT, "spatial_spectral_attention_b200", "csrc", "coupling_tc.cu")
     try:
         s = open(path).read()
-        i = s.index("template <int NCG, int QCH, int VF, int VR, bool kNoDK>\n__global__ void "
-                    "__launch_bounds__(128 * (2 + NCG), 1)\n    tc_bwd_dqk_kernel(")
+        i = s.index("template <int NCG, int QCH, int VF, int VR, bool kNoDK, bool kDqFlush>\n"
+                    "__global__ void __launch_bounds__(128 * (2 + NCG), 1)\n    tc_bwd_dqk_kernel(")
         j = s.index("\n}\n", i) + 3
     except (OSError, ValueError):
         return None

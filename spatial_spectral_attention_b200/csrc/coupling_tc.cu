@@ -1101,9 +1101,12 @@ __global__ void __launch_bounds__(64 + 128 * NCG + 128, 1)
 //         V_j); warp 1: MMA issuer and TMEM owner; warps 2-3 idle.
 //   WG1.. (NCG softmax warpgroups): thread = query row (TMEM lane); the
 //         warpgroups split the key columns.  They write the row tile's dO into
-//         TMEM once and store dQ at the end of the row tile.
+//         TMEM once per row tile.
 //   last  (flush): thread = key row; reduces every key tile's partial dK into
-//         global memory while the other roles move on.
+//         global memory while the other roles move on, and at the end of each
+//         run of a row tile's key tiles reads dQ out of TMEM (handing the
+//         columns back to the MMA issuer at once) and stores it, so that the
+//         softmax warpgroups go on to the next row tile meanwhile.
 // TMEM columns: [0,128) S_j and then dP_j of the same key tile (dP is issued
 // once the softmax has read S, so its MMAs run under the softmax's exp2);
 // [128, 128 + kp/2) dO as bf16 pairs, the A operand of dP; [256, 256 + d) dQ;
@@ -1114,7 +1117,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG + 128, 1)
 //   dKp  = dS^T Q       (SS, MN-major views) -> flush warpgroup -> dK
 // Shared memory: Q, two K stages, V, dS (no dO tile), which leaves room for
 // the second K stage; a key tile's K load overlaps the previous tile's work.
-template <int NCG, int QCH, int VF, int VR, bool kNoDK>
+template <int NCG, int QCH, int VF, int VR, bool kNoDK, bool kDqFlush>
 __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     tc_bwd_dqk_kernel(const __grid_constant__ TensorMaps tm, const TcParams p) {
   static_assert(NCG == 2, "the register split assumes two softmax warpgroups");
@@ -1129,7 +1132,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q_full, bar_q_empty, bar_k_full[2], bar_k_empty[2], bar_v_full,
       bar_v_empty, bar_s_full, bar_s_read, bar_dp_full, bar_ds_full, bar_do_full, bar_dkp_full,
-      bar_dkp_empty, bar_dq_full, bar_drain, bar_dp_read, bar_never;
+      bar_dkp_empty, bar_dq_full, bar_dq_empty, bar_drain, bar_dp_read, bar_never;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_range[3];  // first tile, first segment in it, number of units
@@ -1165,6 +1168,7 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
     mbar_init(&bar_dkp_full, 1);
     mbar_init(&bar_dkp_empty, 128);
     mbar_init(&bar_dq_full, 1);
+    mbar_init(&bar_dq_empty, 128);
     mbar_init(&bar_drain, 1);
     mbar_init(&bar_never, 1);  // nothing arrives: the abort-path test hook waits here
     s_abort = 0;
@@ -1325,7 +1329,15 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
             break;
           }
           tc_fence_after();
-          // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major
+          // dQ += dS K_j : A = dS [q][keys] K-major, B = K_j [keys][d] MN-major; the
+          // run's first one overwrites the columns once the flush warpgroup has
+          // read the previous run's dQ out of them
+          if (kDqFlush && j == jb && tcount > 0 &&
+              !mbar_wait(&bar_dq_empty, (tcount - 1) & 1, p.ctl, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff = (kk >> 2) * kChunk + (kk & 3) * 32;
@@ -1475,6 +1487,12 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
         mbar_arrive(&bar_ds_full);
       }
       if (!ok) break;
+      if constexpr (kDqFlush) {
+        // the run's MMAs are complete (its dP read dO): the next run's dO may
+        // be written; the flush warpgroup stores this run's dQ
+        if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
+        continue;
+      }
       if (!mbar_wait(&bar_dq_full, tcount & 1, p.ctl, abort)) break;
       tc_fence_after();
       // dQ / s goes out through a 2 KB staging area inside this warp's own rows
@@ -1532,18 +1550,19 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
       }
     }
   } else {
-    // ---------------- flush (one warpgroup): thread = key row of the partial dK
+    // ---------------- flush (one warpgroup): thread = key row of the partial dK,
+    // and at the end of each run the query row of its dQ
     warpgroup_reg_alloc<176>();
     const int lrow = 32 * (warp & 3) + lane;
     const int qbase = lane & ~3;
     const uint32_t wstage = sStage + (warp & 3) * 8192;  // this warp's two 4 KB boxes
-    uint32_t it = 0, wblk = 0;
+    uint32_t it = 0, wblk = 0, rcount = 0;
     bool ok = true;
     UnitRange ur{s_range[0], s_range[1], s_range[2]};
     int t, jb, je;
-    while (ok && !kNoDK && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
+    while (ok && (kDqFlush || !kNoDK) && next_segment(ur, p.tiles, ntiles, t, jb, je)) {
       const RowTile tile = p.tiles[t];
-      for (int j = jb; j < je; ++j, ++it) {
+      for (int j = jb; j < je && !kNoDK; ++j, ++it) {
         const KeySeg sg = p.segs[tile.seg0 + j];
         const int krow = sg.key0 + lrow;
         int okey = (lrow < sg.nkeys && krow < p.nk) ? (p.col_map ? p.col_map[krow] : krow) : -1;
@@ -1638,6 +1657,83 @@ __global__ void __launch_bounds__(128 * (2 + NCG), 1)
           }
         }
       }
+      if (!ok) break;
+      if constexpr (!kDqFlush) continue;
+      // dQ / s of this run: its MMAs are complete; the columns are read in one
+      // TMEM round trip and handed back to the MMA issuer before the stores.
+      // Stored when the run covers all of the row tile's keys, else added
+      // (the row tile's keys are split over CTAs).
+      if (!mbar_wait(&bar_dq_full, rcount & 1, p.ctl, abort)) break;
+      tc_fence_after();
+      {
+        const uint32_t qa = tmem_lane_addr(tmem, warp, c_dq);
+        const bool whole = jb == 0 && je == tile.nseg;
+        const int qr = tile.row0 + lrow;
+        int orow = (lrow < tile.nrows && qr < p.nq) ? (p.row_map ? p.row_map[qr] : qr) : -1;
+        if (orow >= p.nq) orow = -1;
+        const bool live = orow >= 0;
+        if (!live) orow = 0;
+        const bool vec = (p.lddq & 3) == 0 && (whole || p.vec_atomics_dq);
+        // the output rows of this thread's lane quad
+        int qrow[4];
+        bool qlive[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          qrow[m] = __shfl_sync(0xffffffffu, orow, qbase + m);
+          qlive[m] = __shfl_sync(0xffffffffu, live ? 1 : 0, qbase + m) != 0;
+        }
+        // 16 columns of dQ / s: with float4 access each lane quad transposes
+        // its 4 x 16 values, so that a float4 of each lane covers 64
+        // contiguous bytes of a row with the quad's other lanes
+        auto put = [&](int q, const uint32_t (&o)[16]) {
+          if (vec) {
+            float4 v[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              v[c] = make_float4(__uint_as_float(o[4 * c]) * p.scale, __uint_as_float(o[4 * c + 1]) * p.scale,
+                                 __uint_as_float(o[4 * c + 2]) * p.scale,
+                                 __uint_as_float(o[4 * c + 3]) * p.scale);
+            quad_transpose4(v, lane & 3);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              if (!qlive[m]) continue;
+              float4* d4 = reinterpret_cast<float4*>(p.dQ + (size_t)qrow[m] * p.lddq + 16 * q + 4 * (lane & 3));
+              if (whole) *d4 = v[m];
+              else atomicAdd(d4, v[m]);
+            }
+          } else if (live) {
+            float* dst = p.dQ + (size_t)orow * p.lddq + 16 * q;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float v = __uint_as_float(o[i]) * p.scale;
+              if (whole) dst[i] = v;
+              else atomicAdd(dst + i, v);
+            }
+          }
+        };
+        if constexpr (kFixed) {
+          // all d = 128 columns in one TMEM round trip, handed back to the MMA
+          // issuer before the stores
+          uint32_t o[8][16];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) tmem_ld16(qa + 16 * q, o[q]);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&bar_dq_empty);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) put(q, o[q]);
+        } else {
+          for (int q = 0; q < d16; ++q) {
+            uint32_t o[16];
+            tmem_ld16(qa + 16 * q, o);
+            tmem_ld_wait();
+            put(q, o);
+          }
+          tc_fence_before();
+          mbar_arrive(&bar_dq_empty);
+        }
+      }
+      ++rcount;
     }
     // the reductions still in flight must finish before the CTA exits
     if (lane == 0 && p.dk_tma) bulk_wait_group_all();
@@ -2652,8 +2748,16 @@ cudaError_t launch_tc_bwd(const TcArgs& a, const __nv_bfloat16* dOb, int lddob, 
     p.dk_tma = !p.col_map && p.vec_atomics &&
                make_map_f32(&tm.dk, p.dK, a.nKrows, a.d, p.lddk, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
-    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, false>
-                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, false>;
+    // dQ stored by the flush warpgroup when row tiles run over many key tiles
+    // (dense: the softmax warpgroups then go straight on to the next row
+    // tile); by the softmax warpgroups when runs are short (Geo: a dozen key
+    // segments per row tile, where the flush warpgroup's extra stores would
+    // hold up the dK partials)
+    const bool dq_flush = a.ntiles_dev == nullptr;
+    auto kern = fixed ? (dq_flush ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, false, true>
+                                  : tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, false, false>)
+                      : (dq_flush ? tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, false, true>
+                                  : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     p.debug_stall = take_stall(2);
@@ -2782,8 +2886,8 @@ cudaError_t launch_tc_bwd_deterministic(const __nv_bfloat16* Q, int ldq, const _
   {
     // dQ: no more CTAs than row tiles, so a row tile's dQ gets at most two adds
     const int smem = 1024 + 3 * p.qch * kChunk + vb + 4 * kChunk;
-    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, true>
-                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, true>;
+    auto kern = fixed ? tc_bwd_dqk_kernel<kBwdComputeGroups, 2, 3, 16, true, true>
+                      : tc_bwd_dqk_kernel<kBwdComputeGroups, 0, 0, 0, true, true>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
