@@ -126,25 +126,37 @@ struct GatherJob {
   const __nv_bfloat16* in;
   const int* map;
   __nv_bfloat16* out;
-  int in_ld, rows, src_rows, cols, out_ld, vec;
-  long long begin;
+  int in_ld, rows, src_rows, cols, out_ld;
+  int vec;     // elements per output piece (8, 4 or 1)
+  int split;   // vec = 8 pieces read as two 8-byte halves (rows 8-byte aligned only)
+  int pieces;  // output pieces per row, out_ld / vec (< 512)
+  unsigned long long magic;  // floor(2^40 / pieces) + 1: r = (i * magic) >> 40 = i / pieces
 };
 struct GatherJobs {
   GatherJob j[3];
-  long long end;
 };
 
-__device__ __forceinline__ uint4 gather_piece(const GatherJob& g, int i, unsigned* status,
+// Output piece li of a job (row li / pieces, columns from (li % pieces) vec):
+// the row's source through the map, read in one or two loads when the piece
+// lies within the source columns, element by element (zero past them) else.
+// The division by the job's piece count is a multiply by its inverse (exact
+// for li < 2^30 and pieces < 512: li (magic pieces - 2^40) < 2^39).
+__device__ __forceinline__ uint4 gather_piece(const GatherJob& g, int li, unsigned* status,
                                               __nv_bfloat16** dst) {
-  const int pieces = g.out_ld / g.vec;
-  const int li = i - (int)g.begin;
-  const int r = li / pieces;
-  const int c0 = (li - r * pieces) * g.vec;
+  const int r = (int)(((unsigned long long)(unsigned)li * g.magic) >> 40);
+  const int c0 = (li - r * g.pieces) * g.vec;
   const int src = checked_src(g.map, r, g.src_rows, status);
   *dst = g.out + (size_t)r * g.out_ld + c0;
   if (src >= 0 && c0 + g.vec <= g.cols) {
     const __nv_bfloat16* a = g.in + (size_t)src * g.in_ld + c0;
-    if (g.vec == 8) return __ldg(reinterpret_cast<const uint4*>(a));
+    if (g.vec == 8) {
+      if (g.split) {
+        const uint2 x = __ldg(reinterpret_cast<const uint2*>(a));
+        const uint2 y = __ldg(reinterpret_cast<const uint2*>(a) + 1);
+        return make_uint4(x.x, x.y, y.x, y.y);
+      }
+      return __ldg(reinterpret_cast<const uint4*>(a));
+    }
     if (g.vec == 4) {
       const uint2 v = __ldg(reinterpret_cast<const uint2*>(a));
       return make_uint4(v.x, v.y, 0u, 0u);
@@ -166,28 +178,29 @@ __device__ __forceinline__ void put_piece(__nv_bfloat16* dst, int vec, uint4 v) 
   else *dst = __ushort_as_bfloat16((unsigned short)(v.x & 0xffffu));
 }
 
-// 32-bit piece indices (the launcher falls back to one launch per job when
-// the pieces do not fit).
-__global__ void gather_jobs_kernel(const GatherJobs jobs, unsigned* status) {
+// The three jobs one after the other, each over the whole grid, four pieces
+// per thread in flight (loads before stores); the job loop is unrolled so that
+// every job's parameters are read at fixed offsets.  32-bit piece indices (the
+// launcher falls back to one launch per job when the pieces do not fit).
+__global__ void gather_jobs_kernel(const __grid_constant__ GatherJobs jobs, unsigned* status) {
   const int stride = gridDim.x * blockDim.x;
-  const int end = (int)jobs.end, b1 = (int)jobs.j[1].begin, b2 = (int)jobs.j[2].begin;
-  for (int i0 = blockIdx.x * blockDim.x + threadIdx.x; i0 < end; i0 += 4 * stride) {
-    uint4 v[4];
-    __nv_bfloat16* dst[4];
-    int vec[4];
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * stride;
-      vec[u] = 0;
-      if (i < end) {
-        const int jj = i < b1 ? 0 : (i < b2 ? 1 : 2);
-        vec[u] = jobs.j[jj].vec;
-        v[u] = gather_piece(jobs.j[jj], i, status, &dst[u]);
+  for (int jj = 0; jj < 3; ++jj) {
+    const GatherJob& g = jobs.j[jj];
+    const int n = g.rows * g.pieces;
+    for (int i0 = tid; i0 < n; i0 += 4 * stride) {
+      uint4 v[4];
+      __nv_bfloat16* dst[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * stride;
+        if (i < n) v[u] = gather_piece(g, i, status, &dst[u]);
       }
-    }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (vec[u]) put_piece(dst[u], vec[u], v[u]);
+      for (int u = 0; u < 4; ++u)
+        if (i0 + u * stride < n) put_piece(dst[u], g.vec, v[u]);
+    }
   }
 }
 
@@ -870,13 +883,18 @@ cudaError_t launch_gather3_bf16(const __nv_bfloat16* const in[3], const int in_l
                                 const int cols[3], __nv_bfloat16* const out[3], const int out_ld[3],
                                 unsigned* status, cudaStream_t st) {
   GatherJobs jobs;
-  long long begin = 0;
+  long long total = 0;
+  bool small = true;
   for (int j = 0; j < 3; ++j) {
     GatherJob& g = jobs.j[j];
     const uintptr_t ia = reinterpret_cast<uintptr_t>(in[j]), oa = reinterpret_cast<uintptr_t>(out[j]);
-    g.vec = (in_ld[j] % 8 == 0 && out_ld[j] % 8 == 0 && ia % 16 == 0 && oa % 16 == 0)   ? 8
-            : (in_ld[j] % 4 == 0 && out_ld[j] % 4 == 0 && ia % 8 == 0 && oa % 8 == 0) ? 4
-                                                                                      : 1;
+    const bool out16 = out_ld[j] % 8 == 0 && oa % 16 == 0;
+    const bool in16 = in_ld[j] % 8 == 0 && ia % 16 == 0;
+    const bool in8 = in_ld[j] % 4 == 0 && ia % 8 == 0;
+    g.split = out16 && !in16 && in8;
+    g.vec = (out16 && (in16 || in8))                                         ? 8
+            : (in8 && out_ld[j] % 4 == 0 && oa % 8 == 0)                     ? 4
+                                                                             : 1;
     g.in = in[j];
     g.map = map[j];
     g.out = out[j];
@@ -885,13 +903,15 @@ cudaError_t launch_gather3_bf16(const __nv_bfloat16* const in[3], const int in_l
     g.src_rows = src_rows[j];
     g.cols = cols[j];
     g.out_ld = out_ld[j];
-    g.begin = begin;
-    begin += (long long)rows[j] * (out_ld[j] / g.vec);
+    g.pieces = out_ld[j] / g.vec;
+    g.magic = g.pieces > 0 ? (1ull << 40) / (unsigned long long)g.pieces + 1 : 0;
+    if (g.pieces >= 512) small = false;
+    total += (long long)rows[j] * g.pieces;
   }
-  jobs.end = begin;
-  if (begin == 0) return cudaSuccess;
-  if (begin >= (1LL << 30)) {
-    // too many pieces for 32-bit indices: one launch per matrix
+  if (total == 0) return cudaSuccess;
+  if (total >= (1LL << 30) || !small) {
+    // too many pieces for 32-bit indices (or rows too long for the inverse):
+    // one launch per matrix
     for (int j = 0; j < 3; ++j) {
       const cudaError_t e = launch_gather_rows_bf16(in[j], in_ld[j], 0, map[j], rows[j], src_rows[j],
                                                     cols[j], out[j], out_ld[j], status, st);
@@ -899,6 +919,7 @@ cudaError_t launch_gather3_bf16(const __nv_bfloat16* const in[3], const int in_l
     }
     return cudaSuccess;
   }
+  const long long begin = total;
   const int blocks = (int)std::max<long long>(1, std::min<long long>((begin + 1023) / 1024, 148LL * 8));
   prof_launch_begin(st);
   gather_jobs_kernel<<<blocks, 256, 0, st>>>(jobs, status);
