@@ -22,6 +22,14 @@
  *    asynchronously; no call synchronises the host.  Device-side failures
  *    (a bounded wait that ran out) are recorded in a library status word that
  *    ssc_device_status() reads back.
+ *  - Some launches that do not depend on the work just before them (the Geo
+ *    patch-major gather, the zeroing of the backward's accumulators) run on a
+ *    side stream of the library: one per host thread and device, created on
+ *    that thread's first call outside stream capture.  It waits for `stream`
+ *    before its launches and `stream` waits for it afterwards (events), so
+ *    the call's work is ordered on `stream` as a whole; a call inside stream
+ *    capture brings the side stream into the capture and joins it back.  When
+ *    the side stream cannot be made, everything runs on `stream`.
  *  - Matrices are row-major with an explicit leading dimension (`ld*`, in
  *    elements, >= the row length).  bf16 Q and K need 16-byte aligned base
  *    pointers and leading dimensions that are multiples of 8 elements (the

@@ -163,6 +163,14 @@ __device__ __forceinline__ uint4 gather_piece(const GatherJob& g, int li, unsign
     }
     return make_uint4(__bfloat16_as_ushort(a[0]), 0u, 0u, 0u);
   }
+  // wholly past the source columns (the padding of the row) or a dead row: zeros
+  if (src < 0 || c0 >= g.cols) return make_uint4(0u, 0u, 0u, 0u);
+  // an 8-element piece with 4 source columns left (k = 4 mod 8): one 8-byte
+  // load (vec = 8 pieces come from rows that are 8-byte aligned at least)
+  if (g.vec == 8 && c0 + 4 == g.cols) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(g.in + (size_t)src * g.in_ld + c0));
+    return make_uint4(v.x, v.y, 0u, 0u);
+  }
   uint32_t w[4] = {0u, 0u, 0u, 0u};
   for (int e = 0; e < g.vec; ++e) {
     const int c = c0 + e;
