@@ -485,6 +485,43 @@ def run_ours(args, ws, rank, local):
                                  workspace=g["ws"], reuse_forward=True)
         return topk
 
+    # ---- the Geo step on its own, before any dense step (after the dense work
+    # the clocks sit lower under the power cap for a while): K steps launched one
+    # by one through the API and K replays of the same step captured as one
+    # CUDA graph, alternating, L2 flushed before each; clocks sampled meanwhile
+    geo_alone = None
+    if geo:
+        for _ in range(args.warmup):
+            geo_step()
+        gr = step_graph(geo_step, torch, dev)
+        for _ in range(args.warmup):
+            geo_step()
+            gr.replay()
+        torch.cuda.synchronize()
+        reps = args.steps
+        gclk = ClockSampler(local).__enter__()
+        time.sleep(0.05)
+        pairs_ev = []
+        g0 = time.time()
+        for _ in range(reps):
+            for fn in (geo_step, gr.replay):
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                flush.zero_()
+                e[0].record(stream)
+                fn()
+                e[1].record(stream)
+                pairs_ev.append(e)
+        torch.cuda.synchronize()
+        g1 = time.time()
+        gclk.mark(g0, g1)
+        gclk.__exit__()
+        tt = [a.elapsed_time(b) for a, b in pairs_ev]
+        geo_alone = {"eager": max_over_ranks(float(np.mean(tt[0::2])), ws),
+                     "graph": max_over_ranks(float(np.mean(tt[1::2])), ws),
+                     "steps": reps, "clocks": gclk.summary()}
+        del gr
+        barrier(ws)
+
     clk = ClockSampler(local).__enter__()
     for _ in range(args.warmup):
         dense_step(Q, K, V, dO)
@@ -633,28 +670,6 @@ def run_ours(args, ws, rank, local):
             ("gather", api.PROF_GATHER))}
         geo_kern = {nm: (ms / gsteps, n // gsteps) for nm, (ms, n) in geo_kern.items()}
         geo_kern["_topk"] = topk_last
-        # the step on its own (no dense step between, so the clocks are not those
-        # of the dense step's power draw): K steps launched one by one through
-        # the API and K replays of the same step captured as one CUDA graph,
-        # alternating, L2 flushed before each
-        gr = step_graph(geo_step, torch, dev)
-        for _ in range(args.warmup):
-            geo_step()
-            gr.replay()
-        pairs_ev = []
-        for _ in range(args.steps):
-            for fn in (geo_step, gr.replay):
-                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                flush.zero_()
-                e[0].record(stream)
-                fn()
-                e[1].record(stream)
-                pairs_ev.append(e)
-        torch.cuda.synchronize()
-        tt = [a.elapsed_time(b) for a, b in pairs_ev]
-        geo_alone_ms = max_over_ranks(float(np.mean(tt[0::2])), ws)
-        geo_graph_ms = max_over_ranks(float(np.mean(tt[1::2])), ws)
-        del gr
     fps_timing = run_fps_timing(api, synth, torch, dev) if (geo and rank == 0) else None
 
     pk = peaks()
@@ -763,9 +778,11 @@ def run_ours(args, ws, rank, local):
                                 "per launch (L2 re-reads not counted)",
             "peak_source": pk["source"] + " (MEASURED_PEAKS.json: bf16_tflops, hbm_gbs)",
         }
+        geo_graph_ms = geo_alone["graph"]
         res["geo"] = {"workload": gpair.name, "ms_per_step": round(geo_graph_ms, 4),
-                      "eager_ms_per_step": round(geo_alone_ms, 4),
+                      "eager_ms_per_step": round(geo_alone["eager"], 4),
                       "eager_ms_per_step_beside_dense": round(geo_ms, 4),
+                      "steps": geo_alone["steps"], "clocks": geo_alone["clocks"],
                       "tflops": round(gflops / (geo_graph_ms * 1e-3) / 1e12, 2),
                       "frac_of_peak": round(gflops / (geo_graph_ms * 1e-3) / 1e12 / pk["tflops"], 4),
                       "support_pairs": pairs, "tile_pairs": pairs_exec,
@@ -777,9 +794,10 @@ def run_ours(args, ws, rank, local):
                               "patch-major operands and schedule from the workspace); "
                               "ms_per_step: the step's launches replayed as one CUDA graph, "
                               "eager_ms_per_step: launched one by one through the API (the two "
-                              "alternating, Geo steps only); eager_ms_per_step_beside_dense: in "
-                              "the main timed region, each after a dense step; FPS per shape, "
-                              "outside the step, timed warm on resident points"}
+                              "alternating, Geo steps only, before any dense step; clocks "
+                              "sampled meanwhile); eager_ms_per_step_beside_dense: in the main "
+                              "timed region, each after a dense step; FPS per shape, outside "
+                              "the step, timed warm on resident points"}
     return res
 
 
